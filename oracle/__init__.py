@@ -1,0 +1,252 @@
+"""The oracle: a plain CPU restatement of UNO's per-cycle sampling and
+verification step, in double precision (``uno_ref.c``), with a numpy wrapper.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  It shares no code with the CUDA library and the library never calls
+it.
+
+What pins each function (the tests under ``tests/test_oracle_*.py``):
+
+* ``philox`` / ``uniform``: the published Philox4x32-10 known-answer vectors
+  (``tests/golden/philox4x32_10_kat.txt``) and the counter layout checked on a
+  known-answer counter.
+* ``filter_softmax``: reduces to ``numpy.argmax`` for T = 0 or top_k = 1, to
+  ``scipy.special.softmax`` for top_p = 1 with top_k >= vocab, to a softmax
+  over a ``numpy.lexsort`` top-k for top_p = 1; the top-p cut is checked
+  against its defining property (the shortest prefix whose mass reaches
+  top_p); the draw is checked by a chi-square test against the filtered
+  probabilities.
+* ``linear_verify``: the emitted sequence is distributed exactly as the
+  target-only autoregressive process (chi-square on a tiny vocabulary with a
+  prefix-dependent target table); the mean accept length equals its closed
+  form; the invariants named by the method (counts in [0, B], equal p and q
+  accept all, disjoint one-hot p and q reject at the first position, top_k 1
+  is greedy speculative decoding).
+* ``tree_topk_expand``: brute-force enumeration of every path of the depth-B
+  trie, ranked by score; K = 1, V = B + 1 gives the argmax chain.
+* ``tree_verify``: emitted sequence distributed as the target-only process
+  (chi-square), mean accept length equals the sum over tree nodes of the
+  target path probability, one-hot targets equal greedy decoding.
+
+Parity unpinned: the boundary-event margin below which a GPU/oracle decision
+difference is excused (``BOUNDARY_EPS``) is a stated tolerance, not a value the
+pages fix.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from pathlib import Path
+
+import numpy as np
+
+_HERE = Path(__file__).resolve().parent
+_SRC = _HERE / "uno_ref.c"
+_LIB_PATH = _HERE / "_build" / "libuno_ref.so"
+
+F32, BF16 = 0, 1
+DRAW_PROPOSAL, DRAW_ACCEPT, DRAW_RESIDUAL, DRAW_TARGET = 0, 1, 2, 3
+FLAG_NONFINITE_ROW, FLAG_DRAFT_NOT_IN_SUPPORT, FLAG_RESIDUAL_EMPTY = 1, 2, 4
+
+# A decision whose distance from its flip point is below this is a boundary
+# event: the GPU may take the other branch there, and such cases are counted.
+BOUNDARY_EPS = 1e-6
+
+_lib = None
+
+
+def build(force: bool = False) -> Path:
+    """Compile ``uno_ref.c`` into ``oracle/_build/libuno_ref.so`` with gcc."""
+    _LIB_PATH.parent.mkdir(parents=True, exist_ok=True)
+    if force or not _LIB_PATH.exists() or _LIB_PATH.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB_PATH.with_suffix(".so.tmp%d" % os.getpid())
+        cmd = ["gcc", "-std=c11", "-O2", "-Wall", "-Wextra", "-fPIC", "-shared",
+               "-o", str(tmp), str(_SRC), "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _bind(lib):
+    P = ctypes.c_void_p
+    i32, i64, u32, u64, f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_float
+    lib.uno_ref_philox4x32_10.argtypes = [P, P, P]
+    lib.uno_ref_philox4x32_10.restype = None
+    lib.uno_ref_uniform.argtypes = [u64, u32, u32, u32, u32]
+    lib.uno_ref_uniform.restype = ctypes.c_double
+    lib.uno_ref_filter_softmax.argtypes = [P, ctypes.c_int, i64, i64, i64, i32, f32, i32, f32, i32,
+                                           P, P, P, P, ctypes.c_int, u64, u32, P, P, P]
+    lib.uno_ref_filter_softmax.restype = ctypes.c_int
+    lib.uno_ref_linear_verify.argtypes = [P, ctypes.c_int, i32, i32, i64, f32, i32, f32, P, P, P, P, i32,
+                                          u64, u32, P, P, P, P, P]
+    lib.uno_ref_linear_verify.restype = ctypes.c_int
+    lib.uno_ref_tree_topk_expand.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P]
+    lib.uno_ref_tree_topk_expand.restype = ctypes.c_int
+    lib.uno_ref_tree_verify.argtypes = [P, ctypes.c_int, i32, i32, i32, i64, f32, i32, f32, P, P, P,
+                                        u64, u32, P, P, P, P, P, P]
+    lib.uno_ref_tree_verify.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _bind(ctypes.CDLL(str(build())))
+    return _lib
+
+
+class use_library:
+    """Context manager: route the functions of this module to another build of
+    the oracle source (the tests use it to check that planted mistakes fail
+    the pins)."""
+
+    def __init__(self, so_path):
+        self._new = _bind(ctypes.CDLL(str(so_path)))
+
+    def __enter__(self):
+        global _lib
+        self._old = _load()
+        _lib = self._new
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self._old
+        return False
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _logits(arr, dtype):
+    """Return (contiguous array, dtype code).  bf16 rows travel as uint16 bits."""
+    if dtype == "bf16":
+        a = np.ascontiguousarray(arr, dtype=np.uint16)
+        return a, BF16
+    if dtype == "f32":
+        a = np.ascontiguousarray(arr, dtype=np.float32)
+        return a, F32
+    raise ValueError("dtype must be 'f32' or 'bf16'")
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise OracleError(f"{what}: oracle status {rc}")
+
+
+def philox(ctr, key):
+    """Philox4x32-10 of a 4-word counter under a 2-word key."""
+    lib = _load()
+    c = np.asarray(ctr, dtype=np.uint32).copy()
+    k = np.asarray(key, dtype=np.uint32).copy()
+    out = np.zeros(4, dtype=np.uint32)
+    lib.uno_ref_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def uniform(seed, request, position, draw, cycle=0):
+    return _load().uno_ref_uniform(int(seed), int(request), int(position), int(draw), int(cycle))
+
+
+def filter_softmax(logits, dtype, temperature, top_k, top_p, *, rows_per_request=1, cap=None,
+                   rng=None, dense=False):
+    """Filter each row of ``logits`` ([rows, vocab]); returns a dict with
+    ids [rows, cap], probs [rows, cap], count, flags, margin, and, on request,
+    sample (rng = (seed, cycle)) and dense [rows, vocab]."""
+    a, code = _logits(logits, dtype)
+    rows, vocab = a.shape
+    if cap is None:
+        cap = min(top_k, vocab)
+    ids = np.empty((rows, cap), dtype=np.int32)
+    probs = np.empty((rows, cap), dtype=np.float32)
+    count = np.empty(rows, dtype=np.int32)
+    flags = np.empty(rows, dtype=np.uint32)
+    margin = np.empty(rows, dtype=np.float64)
+    dn = np.empty((rows, vocab), dtype=np.float32) if dense else None
+    sample = np.empty(rows, dtype=np.int32) if rng is not None else None
+    seed, cycle = rng if rng is not None else (0, 0)
+    rc = _load().uno_ref_filter_softmax(_ptr(a), code, rows, vocab, vocab, rows_per_request,
+                                        float(temperature), int(top_k), float(top_p), cap,
+                                        _ptr(ids), _ptr(probs), _ptr(count), _ptr(dn),
+                                        1 if rng is not None else 0, int(seed), int(cycle),
+                                        _ptr(sample), _ptr(flags), _ptr(margin))
+    _check(rc, "filter_softmax")
+    out = dict(ids=ids, probs=probs, count=count, flags=flags, margin=margin)
+    if dense:
+        out["dense"] = dn
+    if rng is not None:
+        out["sample"] = sample
+    return out
+
+
+def linear_verify(target_logits, dtype, R, B, temperature, top_k, top_p, draft_ids, q_ids, q_probs,
+                  q_count, rng):
+    """Linear rejection sampling; target_logits [R*(B+1), vocab]."""
+    a, code = _logits(target_logits, dtype)
+    vocab = a.shape[-1]
+    assert a.size == R * (B + 1) * vocab
+    d = np.ascontiguousarray(draft_ids, dtype=np.int32).reshape(R, B)
+    qi = np.ascontiguousarray(q_ids, dtype=np.int32)
+    qp = np.ascontiguousarray(q_probs, dtype=np.float32)
+    qc = np.ascontiguousarray(q_count, dtype=np.int32)
+    q_cap = qi.shape[-1]
+    toks = np.empty((R, B + 1), dtype=np.int32)
+    acc = np.empty(R, dtype=np.int32)
+    ntok = np.empty(R, dtype=np.int32)
+    flags = np.empty(R, dtype=np.uint32)
+    margin = np.empty(R, dtype=np.float64)
+    seed, cycle = rng
+    rc = _load().uno_ref_linear_verify(_ptr(a), code, R, B, vocab, float(temperature), int(top_k),
+                                       float(top_p), _ptr(d), _ptr(qi), _ptr(qp), _ptr(qc), q_cap,
+                                       int(seed), int(cycle), _ptr(toks), _ptr(acc), _ptr(ntok),
+                                       _ptr(flags), _ptr(margin))
+    _check(rc, "linear_verify")
+    return dict(tokens=toks, accept_len=acc, num_tokens=ntok, flags=flags, margin=margin)
+
+
+def tree_topk_expand(q_ids, q_probs, q_count, R, B, K, V):
+    qi = np.ascontiguousarray(q_ids, dtype=np.int32)
+    qp = np.ascontiguousarray(q_probs, dtype=np.float32)
+    qc = np.ascontiguousarray(q_count, dtype=np.int32)
+    q_cap = qi.shape[-1]
+    tok = np.empty((R, V), dtype=np.int32)
+    par = np.empty((R, V), dtype=np.int32)
+    dep = np.empty((R, V), dtype=np.int32)
+    sco = np.empty((R, V), dtype=np.float32)
+    nn = np.empty(R, dtype=np.int32)
+    rc = _load().uno_ref_tree_topk_expand(_ptr(qi), _ptr(qp), _ptr(qc), q_cap, R, B, K, V,
+                                          _ptr(tok), _ptr(par), _ptr(dep), _ptr(sco), _ptr(nn))
+    _check(rc, "tree_topk_expand")
+    return dict(node_token=tok, node_parent=par, node_depth=dep, node_score=sco, num_nodes=nn)
+
+
+def tree_verify(target_logits, dtype, R, B, V, temperature, top_k, top_p, node_token, node_parent,
+                num_nodes, rng):
+    """Target-only tree verification; target_logits [R*V, vocab]."""
+    a, code = _logits(target_logits, dtype)
+    vocab = a.shape[-1]
+    assert a.size == R * V * vocab
+    tk = np.ascontiguousarray(node_token, dtype=np.int32)
+    pa = np.ascontiguousarray(node_parent, dtype=np.int32)
+    nn = np.ascontiguousarray(num_nodes, dtype=np.int32)
+    toks = np.empty((R, B + 1), dtype=np.int32)
+    path = np.empty((R, B + 1), dtype=np.int32)
+    acc = np.empty(R, dtype=np.int32)
+    ntok = np.empty(R, dtype=np.int32)
+    flags = np.empty(R, dtype=np.uint32)
+    margin = np.empty(R, dtype=np.float64)
+    seed, cycle = rng
+    rc = _load().uno_ref_tree_verify(_ptr(a), code, R, B, V, vocab, float(temperature), int(top_k),
+                                     float(top_p), _ptr(tk), _ptr(pa), _ptr(nn), int(seed), int(cycle),
+                                     _ptr(toks), _ptr(acc), _ptr(ntok), _ptr(path), _ptr(flags),
+                                     _ptr(margin))
+    _check(rc, "tree_verify")
+    return dict(tokens=toks, accept_len=acc, num_tokens=ntok, path_nodes=path, flags=flags,
+                margin=margin)
