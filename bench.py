@@ -1,0 +1,420 @@
+"""Benchmark of UNO's per-cycle sampling and verification step on B200.
+
+One step = one decode cycle of the linear 8/1/8 workload at 64 requests per
+GPU (the UNO PR page's batch-64 linear configuration, vocabulary 151,936,
+bf16, T = 1, top-k 50, top-p 0.95): uno_filter_softmax over the 512 draft
+marginal rows with the proposal draws, then uno_linear_verify over the 576
+target rows.  Inputs are seeded synthetic logits resident in HBM
+(330.6 MB per step, larger than the 126 MB L2).  Each step's two launches are
+captured once in two CUDA graphs and replayed; CUDA events around each replay
+give the per-kernel durations.
+
+Ranks (torchrun, one per GPU) each process their own 64 requests (global
+request indices rank*64 ..), with no collective on the data path; timing is
+the maximum over ranks.
+
+--impl reference times the oracle (oracle/uno_ref.c) on the host cores on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import numpy as np  # noqa: E402
+
+WORKLOAD_INDEX = 1
+METRIC = "verified draft blocks/sec and logits HBM GB/s (fraction of B200 peak)"
+UNIT = "blocks/s"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+BAD_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=WORKLOAD_INDEX, help="index into inputs.WORKLOADS (linear only)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget of the cpu_baseline")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(world):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(values, world, device):
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(world, device):
+    import torch
+    torch.cuda.synchronize(device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index])
+    torch.cuda.synchronize(device)
+
+
+# ---------------------------------------------------------------------------
+# clocks (NVML) sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.005):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # pragma: no cover - NVML missing
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                try:
+                    mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                except Exception:
+                    mask = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        return False
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# peaks and committed profile figures
+# ---------------------------------------------------------------------------
+def hbm_peak():
+    p = ROOT / "MEASURED_PEAKS.json"
+    try:
+        d = json.loads(p.read_text())
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in ("speculative_decoding_verification_filter_b200/csrc/uno_filter.cu",
+                "speculative_decoding_verification_filter_b200/csrc/uno_device.cuh"):
+        h.update((ROOT / rel).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic():
+    """DRAM bytes per launch of the verify kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    p = ROOT / "profiles" / "traffic.json"
+    try:
+        d = json.loads(p.read_text())
+    except Exception:
+        return None
+    if d.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    return d.get("verify_dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host (cpu_baseline and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_requests(w, reqs, cycle=0):
+    """Run the oracle over the given requests one by one; returns seconds."""
+    import oracle
+    from speculative_decoding_verification_filter_b200.inputs import linear_draft, linear_target
+    total = 0.0
+    for r in reqs:
+        q = linear_draft(w, [r])
+        p = linear_target(w, [r])
+        t0 = time.perf_counter()
+        rq = oracle.filter_softmax(q, w.dtype, w.temperature, w.top_k, w.top_p, rows_per_request=w.B,
+                                   rng=(w.seed, cycle, r))
+        oracle.linear_verify(p, w.dtype, 1, w.B, w.temperature, w.top_k, w.top_p, rq["sample"].reshape(1, w.B),
+                             rq["ids"], rq["probs"], rq["count"], rng=(w.seed, cycle, r))
+        total += time.perf_counter() - t0
+    return total
+
+
+def cpu_baseline(w, budget_s):
+    import oracle
+    oracle.build()
+    done, spent = 0, 0.0
+    while done < w.R and spent < budget_s:
+        spent += oracle_requests(w, [done])
+        done += 1
+    return {"value": done / spent, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{done} of {w.R} requests ({done * (2 * w.B + 1)} logit rows), single-threaded C oracle, "
+                      f"{spent:.1f} s of CPU work"}
+
+
+def run_reference(args, w):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    t_req = oracle_requests(w, [0])
+    budget = 150.0
+    steps = max(1, min(args.steps, int(budget / max(t_req, 1e-3))))
+    warm = min(args.warmup, 1)
+    oracle_requests(w, [1 % w.R] * warm)
+    secs = oracle_requests(w, [(2 + i) % w.R for i in range(steps)])
+    value = steps / secs
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
+        "warmup": warm, "ms_per_step": 1e3 * secs / steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, 1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"one request (its {2 * w.B + 1} logit rows) per step, {steps} steps "
+                                   f"(capped at ~{budget:.0f} s), single-threaded C oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, world):
+    return {"workload": f"{w.name}: R={w.R} requests/GPU, B={w.B}, vocab {w.vocab}, {w.dtype} logits, "
+                        f"T={w.temperature}, top-k {w.top_k}, top-p {w.top_p}",
+            "global_batch": w.R * world, "requests_per_gpu": w.R, "vocab": w.vocab, "B": w.B,
+            "logit_bytes_per_step_per_gpu": w.logit_bytes,
+            "l2": "inputs larger than L2 (no flush): %.1f MB of logits per step vs 126 MB L2" % (w.logit_bytes / 1e6),
+            "parallelism": f"requests sharded over {world} GPU(s), no collective on the data path"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, w):
+    import ctypes
+
+    import torch
+    from speculative_decoding_verification_filter_b200 import _binding as b
+    from speculative_decoding_verification_filter_b200.inputs import linear_draft, linear_target
+
+    rank, world, local = dist_env()
+    init_dist(world)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    lib = b.load_library()
+    first = rank * w.R
+    reqs = range(first, first + w.R)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def dev(a):
+        t = torch.from_numpy(a.view(np.int16) if w.dtype == "bf16" else a)
+        return t.to(device).view(tdt)
+
+    q_np = linear_draft(w, reqs)
+    p_np = linear_target(w, reqs)
+    q, p = dev(q_np), dev(p_np)
+    nq, npr, V = w.q_rows, w.p_rows, w.vocab
+    k = min(w.top_k, V)
+    i32 = dict(dtype=torch.int32, device=device)
+    q_ids, q_probs = torch.empty((nq, k), **i32), torch.empty((nq, k), dtype=torch.float32, device=device)
+    q_count, q_flags, drafts = torch.empty(nq, **i32), torch.empty(nq, **i32), torch.empty(nq, **i32)
+    toks, acc = torch.empty((w.R, w.B + 1), **i32), torch.empty(w.R, **i32)
+    ntok, rflags = torch.empty(w.R, **i32), torch.empty(w.R, **i32)
+    ws_q = torch.zeros(lib.uno_filter_softmax_workspace_bytes(nq, V, w.top_k), dtype=torch.uint8, device=device)
+    ws_p = torch.zeros(lib.uno_linear_verify_workspace_bytes(w.R, w.B, V, w.top_k), dtype=torch.uint8,
+                       device=device)
+    sp = b._Params(w.temperature, w.top_k, w.top_p)
+    dcode = b.UNO_BF16 if w.dtype == "bf16" else b.UNO_F32
+    P = ctypes.c_void_p
+    cycle_box = {"c": 0}
+
+    def filter_step(stream):
+        rng = b._Rng(w.seed, cycle_box["c"], first)
+        st = lib.uno_filter_softmax(P(q.data_ptr()), dcode, nq, V, V, w.B, sp, k, P(q_ids.data_ptr()),
+                                    P(q_probs.data_ptr()), P(q_count.data_ptr()), None, ctypes.byref(rng),
+                                    P(drafts.data_ptr()), P(q_flags.data_ptr()), P(ws_q.data_ptr()), ws_q.numel(),
+                                    P(stream.cuda_stream))
+        assert st == 0, b.STATUS.get(st, st)
+
+    def verify_step(stream):
+        rng = b._Rng(w.seed, cycle_box["c"], first)
+        st = lib.uno_linear_verify(P(p.data_ptr()), dcode, w.R, w.B, V, sp, P(drafts.data_ptr()),
+                                   P(q_ids.data_ptr()), P(q_probs.data_ptr()), P(q_count.data_ptr()), k, rng,
+                                   P(toks.data_ptr()), P(acc.data_ptr()), P(ntok.data_ptr()), P(rflags.data_ptr()),
+                                   P(ws_p.data_ptr()), ws_p.numel(), P(stream.cuda_stream))
+        assert st == 0, b.STATUS.get(st, st)
+
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            filter_step(stream)
+            verify_step(stream)
+    torch.cuda.synchronize(device)
+    gq, gp = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gq, stream=stream):
+        filter_step(torch.cuda.current_stream(device))
+    with torch.cuda.graph(gp, stream=stream):
+        verify_step(torch.cuda.current_stream(device))
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            gq.replay()
+            gp.replay()
+    torch.cuda.synchronize(device)
+
+    K = args.steps
+
+    def timed():
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world, device)
+        with ClockSampler(device.index) as clk, torch.cuda.stream(stream):
+            t0.record(stream)
+            for i in range(K):
+                ev[i][0].record(stream)
+                gq.replay()
+                ev[i][1].record(stream)
+                gp.replay()
+                ev[i][2].record(stream)
+            t1.record(stream)
+            stream.synchronize()
+        barrier(world, device)
+        total = t0.elapsed_time(t1)
+        fq = [e[0].elapsed_time(e[1]) for e in ev]
+        fp = [e[1].elapsed_time(e[2]) for e in ev]
+        return total, statistics.fmean(fq), statistics.fmean(fp), clk.summary()
+
+    total_ms, fq_ms, fp_ms, clocks = timed()
+    if any(r in clocks["reasons"] for r in BAD_REASONS):
+        total_ms, fq_ms, fp_ms, clocks = timed()  # re-measured once
+    total_ms, fq_ms, fp_ms = max_over_ranks([total_ms, fq_ms, fp_ms], world, device)
+    ms_step = total_ms / K
+    value = w.R * world / (ms_step / 1e3)
+
+    # end to end through the public API with pinned host buffers
+    from speculative_decoding_verification_filter_b200 import uno_filter_softmax, uno_linear_verify
+    q_host = torch.from_numpy(q_np.view(np.int16) if w.dtype == "bf16" else q_np).view(tdt).pin_memory()
+    p_host = torch.from_numpy(p_np.view(np.int16) if w.dtype == "bf16" else p_np).view(tdt).pin_memory()
+    sp_kw = dict(temperature=w.temperature, top_k=w.top_k, top_p=w.top_p)
+    K_e2e = max(3, min(K, 20))
+
+    def e2e_step(c):
+        fo = uno_filter_softmax(q_host, rows_per_request=w.B, rng=(w.seed, c, first), **sp_kw)
+        vo = uno_linear_verify(p_host, fo["sample"].reshape(w.R, w.B), fo["ids"], fo["probs"], fo["count"], R=w.R,
+                               B=w.B, rng=(w.seed, c, first), **sp_kw)
+        return fo, vo
+
+    for c in range(2):
+        e2e_step(c)
+    barrier(world, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for c in range(K_e2e):
+        fo, vo = e2e_step(c)
+    e1.record()
+    torch.cuda.synchronize(device)
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1) / K_e2e], world, device)
+    h2d = (q_host.numel() + p_host.numel()) * q_host.element_size() + sum(
+        t.numel() * t.element_size() for t in (fo["sample"], fo["ids"], fo["probs"], fo["count"]))
+    d2h = sum(t.numel() * t.element_size() for t in list(fo.values()) + list(vo.values()))
+
+    peak, peak_kind = hbm_peak()
+    verify_bytes = npr * V * w.elem_bytes
+    filter_bytes = nq * V * w.elem_bytes
+    achieved = verify_bytes / (fp_ms / 1e3) / 1e9
+    step_gbs = (verify_bytes + filter_bytes) / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, world),
+        "logits_gbs_per_gpu": step_gbs,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": committed_traffic(), "kernel": "row_kernel<bf16, linear> (uno_linear_verify)",
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback", "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+                     "filter_kernel_gbs": filter_bytes / (fq_ms / 1e3) / 1e9,
+                     "filter_ms": fq_ms, "verify_ms": fp_ms},
+        "e2e": {"value": w.R * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del gq, gp
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    from speculative_decoding_verification_filter_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if w.mode != "linear":
+        raise SystemExit("bench.py times the linear workloads")
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,221 @@
+/*
+ * uno_filter.h -- C ABI of libuno_filter.so: UNO's per-cycle sampling and
+ * verification step over vocabulary-wide logits, on one NVIDIA B200 (sm_100a).
+ *
+ * Method sources (web pages):
+ *   [UNO PR]     "sgl-project/sglang pull request 37667: UNO" -- "Motivation"
+ *                (lossless; linear sampler draws each of B tokens from its own
+ *                marginal; tree sampler keeps the top K candidates of each
+ *                marginal and considers V candidate sequences), "Modifications"
+ *                (sparse and dense proposal and rejection sampling for linear
+ *                UNO; tree UNO reuses EAGLE tree verification with compact-
+ *                support target sampling), review thread (top-k is applied and
+ *                renormalised before top-p).
+ *   [eval guide] "用 SGLang benchmark/uno 复现 UNO 全量数学评测：run_math_eval
+ *                实战与源码解析" -- "run_math_eval 全参数详解" (top_k > 0,
+ *                top_p in (0, 1], temperature >= 0), "B/K/V 参数映射" (B draft
+ *                width, K candidates per depth, V verification width) and
+ *                "启动期硬性约束" (V >= B, V <= 128, V*K <= 2048, acceptance
+ *                thresholds 1.0).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.  Every tensor argument is a DEVICE pointer owned by the caller;
+ *   the library keeps no pointer after a call returns and allocates no memory.
+ *   Logits may be binary32 (UNO_F32) or bfloat16 (UNO_BF16, the top half of a
+ *   binary32) and must be aligned to their element size; 16-byte-aligned rows
+ *   are read fastest.
+ * Stream.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream).  Calls are asynchronous: results are ready when the stream
+ *   reaches them.  A call enqueues one or two kernels and nothing else.
+ * Workspace.  Entry points that need scratch take (workspace, workspace_bytes),
+ *   caller-owned device memory of at least the size the matching
+ *   uno_*_workspace_bytes() returns (256-byte aligned).  Its first
+ *   UNO_WORKSPACE_COUNTER_BYTES hold arrival counters: zero-fill them once,
+ *   before the first use (zero-filling the whole buffer is simplest).  Every
+ *   call leaves them at zero again and writes nothing else there, so one
+ *   workspace serves any later call of any entry point and size.  The rest is
+ *   scratch the library overwrites.  Calls that run at the same time on the
+ *   GPU must not share a workspace.  Verifiers take at most
+ *   UNO_WORKSPACE_COUNTER_BYTES / 8 requests per call.
+ * Compact distributions.  A filtered row is stored as `count` pairs
+ *   (id, prob) in ascending id order, probabilities binary32, in slots
+ *   [0, count) of a row of `cap` slots; unused slots hold id -1 and prob 0.
+ * Randomness.  Each decision draws u in [0, 1) from Philox4x32-10 (Salmon et
+ *   al., SC'11) with key = seed (low word first) and counter
+ *   (request, position, draw, cycle); u = (x0 * 2^21 + (x1 >> 11)) * 2^-53.
+ *   draw = 0 proposal/sample, 1 accept test, 2 residual, 3 target/bonus.
+ * Filter.  Per row: keep the top_k finite logits ordered by (logit desc,
+ *   id asc); temperature 0 keeps the first alone (greedy); otherwise
+ *   w_j = exp((l_j - l_0) / T) and P_j = w_j / sum(w); keep j while the mass
+ *   before j is < top_p (always the first; top_p = 1 keeps all); the result
+ *   is w_j / sum of kept w_j.  The softmax over the kept support runs in
+ *   double precision; the scan over the vocabulary reads every logit once.
+ * Errors.  Arguments are checked on the host before anything is enqueued:
+ *   UNO_ERR_INVALID_ARG for null pointers, non-positive sizes, top_k < 1,
+ *   top_p outside (0, 1], temperature negative or non-finite, a bad tree
+ *   shape; UNO_ERR_UNSUPPORTED for cap < min(top_k, vocab) or
+ *   top_k > UNO_MAX_TOP_K; UNO_ERR_WORKSPACE for a null or short workspace;
+ *   UNO_ERR_CUDA when a launch fails (cudaGetLastError).  Data errors never
+ *   trap: they set per-row or per-request flag bits (UNO_FLAG_*).
+ */
+#ifndef UNO_FILTER_H
+#define UNO_FILTER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    UNO_OK = 0,
+    UNO_ERR_INVALID_ARG = 1,
+    UNO_ERR_UNSUPPORTED = 2,
+    UNO_ERR_CUDA = 3,
+    UNO_ERR_WORKSPACE = 4
+} uno_status;
+
+typedef enum { UNO_F32 = 0, UNO_BF16 = 1 } uno_dtype;
+
+/* Request sampling parameters ([eval guide, run_math_eval 全参数详解]). */
+typedef struct {
+    float temperature; /* >= 0; 0 = greedy                  */
+    int32_t top_k;     /* >= 1; clamped to the vocabulary     */
+    float top_p;       /* in (0, 1]                           */
+} uno_sampling_params;
+
+/* Counter-based RNG state of one decode cycle.  first_request is the global
+ * index of the call's first request: the counter's request word is
+ * first_request + local request index, so a batch split across calls or GPUs
+ * draws the same uniforms as one call over the whole batch. */
+typedef struct {
+    uint64_t seed;
+    uint32_t cycle;
+    uint32_t first_request;
+} uno_rng;
+
+#define UNO_MAX_TOP_K 1024
+#define UNO_WORKSPACE_COUNTER_BYTES (1 << 20)
+#define UNO_MAX_TREE_NODES 128   /* V <= 128   ([eval guide, 启动期硬性约束]) */
+#define UNO_MAX_TREE_FRONTIER 2048 /* V*K <= 2048 (same section) */
+
+/* Flag bits (per row of uno_filter_softmax, per request of the verifiers). */
+#define UNO_FLAG_NONFINITE_ROW 1u        /* NaN or +inf logit, or no finite logit */
+#define UNO_FLAG_DRAFT_NOT_IN_SUPPORT 2u /* draft token has q = 0: rejected      */
+#define UNO_FLAG_RESIDUAL_EMPTY 4u       /* max(0, p - q) summed to 0: drew p    */
+#define UNO_FLAG_TIMEOUT 8u              /* a bounded wait for the row's own     */
+                                         /* asynchronous copies gave up; the row */
+                                         /* result is not valid                  */
+
+/* ------------------------------------------------------------------------
+ * uno_filter_softmax -- filter each row and optionally draw from it.
+ * [UNO PR, review thread]: top-k first, renormalise, then top-p; [UNO PR,
+ * Motivation]: the linear sampler draws each draft token independently from
+ * its marginal.
+ *
+ * logits      [rows][row_stride] elements of dtype `dt` (row_stride >= vocab).
+ * rows_per_request  maps row -> (request = rng->first_request + row / rpr,
+ *             position = row % rpr) for the RNG counter (e.g. B for draft
+ *             marginals).
+ * cap         slots per compact row, >= min(top_k, vocab).
+ * out_ids     [rows][cap] int32, out_probs [rows][cap] float, out_count [rows].
+ * out_dense   nullable [rows][vocab] float: the filtered distribution.
+ * rng         nullable; when given, out_sample [rows] receives one token drawn
+ *             by inverse CDF (ascending id) with draw 0; -1 for a row with no
+ *             support.
+ * out_flags   [rows] UNO_FLAG_NONFINITE_ROW for rows with NaN/+inf/no finite.
+ * workspace   see uno_filter_softmax_workspace_bytes.
+ * ---------------------------------------------------------------------- */
+size_t uno_filter_softmax_workspace_bytes(int64_t rows, int64_t vocab, int32_t top_k);
+uno_status uno_filter_softmax(const void* logits, uno_dtype dt, int64_t rows, int64_t vocab, int64_t row_stride,
+                              int32_t rows_per_request, uno_sampling_params sp, int32_t cap, int32_t* out_ids,
+                              float* out_probs, int32_t* out_count, float* out_dense, const uno_rng* rng,
+                              int32_t* out_sample, uint32_t* out_flags, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/* ------------------------------------------------------------------------
+ * uno_linear_verify -- linear-mode rejection sampling for R requests.
+ * [UNO PR, Motivation]: lossless like speculative decoding; [UNO PR,
+ * Modifications]: proposal and rejection sampling for linear UNO.  Rule (the
+ * standard speculative-sampling rule; the pages print no formula): for draft
+ * position i = 0..B-1 accept x_i iff u_accept * q_i(x_i) < p_i(x_i); at the
+ * first rejection draw from normalise(max(0, p_i - q_i)) over supp p_i with
+ * the residual draw (from p_i, flagged, if that sums to 0) and stop; if all B
+ * are accepted draw a bonus token from p_B with the target draw.  p_i is
+ * target row i filtered as in uno_filter_softmax.
+ *
+ * target_logits [R][B+1][vocab] (dtype dt), contiguous.
+ * draft_ids     [R][B] int32 (ids outside supp q_i are rejected and flagged).
+ * q_ids/q_probs [R*B][q_cap], q_count [R*B]: the draft marginals as written by
+ *               uno_filter_softmax (ascending ids).
+ * out_tokens    [R][B+1]: accepted drafts then the correction/bonus token;
+ *               unused slots -1.  out_accept_len [R] in [0, B];
+ *               out_num_tokens [R] = accept_len + 1 (accept_len when a
+ *               non-finite target row is reached; its slot holds -1).
+ * out_flags     [R] OR of the request's flag bits.
+ * ---------------------------------------------------------------------- */
+size_t uno_linear_verify_workspace_bytes(int32_t R, int32_t B, int64_t vocab, int32_t top_k);
+uno_status uno_linear_verify(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int64_t vocab,
+                             uno_sampling_params sp, const int32_t* draft_ids, const int32_t* q_ids,
+                             const float* q_probs, const int32_t* q_count, int32_t q_cap, uno_rng rng,
+                             int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                             uint32_t* out_flags, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * uno_tree_topk_expand -- top-K candidates per marginal and a V-node tree.
+ * [UNO PR, Motivation]: the tree sampler considers V candidate sequences by
+ * selecting the top K candidates from each marginal, hyperparameters
+ * (B, K, V); [eval guide, 启动期硬性约束]: V >= B, V <= 128, V*K <= 2048.  The
+ * pages fix no construction rule.  This library's rule: candidates of depth
+ * d+1 are the first min(K, count_d) tokens of q_d by (prob desc, id asc);
+ * node 0 is the root; a child's score is its parent's score times q_d(token)
+ * (double); the frontier node with the highest score joins next, ties to the
+ * lower depth, then lower parent index, then lower candidate rank; stop at V
+ * nodes (root included) or an empty frontier.  Parents precede children.
+ *
+ * q_ids/q_probs [R*B][q_cap], q_count [R*B] (ascending ids, as written by
+ *               uno_filter_softmax).
+ * node_token, node_parent, node_depth [R][V] int32, node_score [R][V] float;
+ *               root: token -1, parent -1, depth 0, score 1; unused slots
+ *               token -1, parent -1, depth -1, score 0.  num_nodes [R].
+ * No workspace.
+ * ---------------------------------------------------------------------- */
+uno_status uno_tree_topk_expand(const int32_t* q_ids, const float* q_probs, const int32_t* q_count, int32_t q_cap,
+                                int32_t R, int32_t B, int32_t K, int32_t V, int32_t* node_token,
+                                int32_t* node_parent, int32_t* node_depth, float* node_score, int32_t* num_nodes,
+                                void* stream);
+
+/* ------------------------------------------------------------------------
+ * uno_tree_verify -- target-only verification of the candidate trees.
+ * [UNO PR, Modifications]: tree UNO reuses EAGLE tree verification with
+ * compact-support target sampling; [eval guide, 启动期硬性约束]: acceptance
+ * thresholds 1.0 (pure target sampling).  From the root: draw y from node j's
+ * filtered target row with the target draw at position j; if a child of j
+ * (lowest index first) carries y, emit y and continue from it; otherwise emit
+ * y and stop.  Stops after B+1 tokens at most.
+ *
+ * target_logits [R][V][vocab] (dtype dt), one row per node; rows at or past
+ *               num_nodes[r] are not read.
+ * node_token, node_parent [R][V], num_nodes [R]: as written by
+ *               uno_tree_topk_expand.
+ * out_tokens, out_path_nodes [R][B+1] (path_nodes[t] = node whose row drew
+ *               token t; unused -1); out_accept_len [R] = tokens - 1;
+ *               out_num_tokens [R]; out_flags [R].
+ * ---------------------------------------------------------------------- */
+size_t uno_tree_verify_workspace_bytes(int32_t R, int32_t V, int64_t vocab, int32_t top_k);
+uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int32_t V, int64_t vocab,
+                           uno_sampling_params sp, const int32_t* node_token, const int32_t* node_parent,
+                           const int32_t* num_nodes, uno_rng rng, int32_t* out_tokens, int32_t* out_accept_len,
+                           int32_t* out_num_tokens, int32_t* out_path_nodes, uint32_t* out_flags, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Text of a status code (static storage). */
+const char* uno_status_string(uno_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UNO_FILTER_H */

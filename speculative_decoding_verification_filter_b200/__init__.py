@@ -1,0 +1,19 @@
+"""UNO's per-cycle sampling and verification step on NVIDIA B200 (sm_100a).
+
+The computation lives in libuno_filter.so (CUDA, C ABI in include/uno_filter.h);
+this package is its thin Python binding plus the seeded synthetic-input
+generator used by the tests and the benchmark.
+"""
+from ._binding import (  # noqa: F401
+    EXPORTED,
+    FLAG_DRAFT_NOT_IN_SUPPORT,
+    FLAG_NONFINITE_ROW,
+    FLAG_RESIDUAL_EMPTY,
+    LIB_PATH,
+    UnoError,
+    load_library,
+    uno_filter_softmax,
+    uno_linear_verify,
+    uno_tree_topk_expand,
+    uno_tree_verify,
+)

@@ -1,0 +1,281 @@
+"""Thin Python binding of libuno_filter.so (include/uno_filter.h).
+
+The functions carry the C entry points' names and only marshal arguments:
+they check shapes, allocate output tensors and a zero-filled workspace with
+PyTorch, pass raw device pointers and the current CUDA stream, and raise when
+the library returns an error.  Every step of the computation runs in the
+library's CUDA kernels.  Host (CPU) input tensors are copied to the current
+CUDA device first and results are copied back, which is what the end-to-end
+benchmark measures.
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libuno_filter.so"
+
+UNO_F32, UNO_BF16 = 0, 1
+FLAG_NONFINITE_ROW, FLAG_DRAFT_NOT_IN_SUPPORT, FLAG_RESIDUAL_EMPTY = 1, 2, 4
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported argument", 3: "CUDA launch error",
+          4: "workspace missing or too small"}
+
+EXPORTED = (
+    "uno_filter_softmax_workspace_bytes", "uno_filter_softmax",
+    "uno_linear_verify_workspace_bytes", "uno_linear_verify",
+    "uno_tree_topk_expand",
+    "uno_tree_verify_workspace_bytes", "uno_tree_verify",
+    "uno_status_string",
+)
+
+
+class UnoError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn}: {STATUS.get(status, 'status %d' % status)}")
+        self.status = status
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_float), ("top_k", ctypes.c_int32), ("top_p", ctypes.c_float)]
+
+
+class _Rng(ctypes.Structure):
+    _fields_ = [("seed", ctypes.c_uint64), ("cycle", ctypes.c_uint32), ("first_request", ctypes.c_uint32)]
+
+
+def _rng(rng):
+    """(seed, cycle) or (seed, cycle, first_request) -> _Rng."""
+    seed, cycle = int(rng[0]), int(rng[1])
+    first = int(rng[2]) if len(rng) > 2 else 0
+    return _Rng(seed, cycle, first)
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def load_library():
+    """Load libuno_filter.so; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not LIB_PATH.exists():
+            raise RuntimeError(f"{LIB_PATH.name} is not built: run `python -m "
+                               "speculative_decoding_verification_filter_b200.build` (needs nvcc)")
+        lib = ctypes.CDLL(str(LIB_PATH))
+        P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        lib.uno_filter_softmax_workspace_bytes.argtypes = [i64, i64, i32]
+        lib.uno_filter_softmax_workspace_bytes.restype = sz
+        lib.uno_filter_softmax.argtypes = [P, ctypes.c_int, i64, i64, i64, i32, _Params, i32, P, P, P, P,
+                                           ctypes.POINTER(_Rng), P, P, P, sz, P]
+        lib.uno_filter_softmax.restype = ctypes.c_int
+        lib.uno_linear_verify_workspace_bytes.argtypes = [i32, i32, i64, i32]
+        lib.uno_linear_verify_workspace_bytes.restype = sz
+        lib.uno_linear_verify.argtypes = [P, ctypes.c_int, i32, i32, i64, _Params, P, P, P, P, i32, _Rng,
+                                          P, P, P, P, P, sz, P]
+        lib.uno_linear_verify.restype = ctypes.c_int
+        lib.uno_tree_topk_expand.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P]
+        lib.uno_tree_topk_expand.restype = ctypes.c_int
+        lib.uno_tree_verify_workspace_bytes.argtypes = [i32, i32, i64, i32]
+        lib.uno_tree_verify_workspace_bytes.restype = sz
+        lib.uno_tree_verify.argtypes = [P, ctypes.c_int, i32, i32, i32, i64, _Params, P, P, P, _Rng,
+                                        P, P, P, P, P, P, sz, P]
+        lib.uno_tree_verify.restype = ctypes.c_int
+        lib.uno_status_string.argtypes = [ctypes.c_int]
+        lib.uno_status_string.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers
+# ---------------------------------------------------------------------------
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int, device: torch.device, stream: torch.cuda.Stream) -> torch.Tensor:
+    """A zero-filled workspace of at least nbytes for this device and stream.
+
+    The library leaves its counters at zero after each call, so the buffer is
+    zero-filled once, when it is created or grown."""
+    key = (device.index, stream.cuda_stream)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return UNO_F32
+    if t.dtype == torch.bfloat16:
+        return UNO_BF16
+    raise TypeError(f"logits must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(fn, status):
+    if status != 0:
+        raise UnoError(fn, status)
+
+
+def _dev(t: torch.Tensor, device) -> torch.Tensor:
+    return t if t.device == device else t.to(device, non_blocking=True)
+
+
+def _device_of(*ts):
+    for t in ts:
+        if isinstance(t, torch.Tensor) and t.is_cuda:
+            return t.device
+    return torch.device("cuda", torch.cuda.current_device())
+
+
+def _host_back(out: dict, host: bool) -> dict:
+    if not host:
+        return out
+    return {k: v.to("cpu", non_blocking=False) for k, v in out.items()}
+
+
+# ---------------------------------------------------------------------------
+# entry points
+# ---------------------------------------------------------------------------
+def uno_filter_softmax(logits, *, temperature, top_k, top_p, rows_per_request=1, cap=None, rng=None,
+                       dense=False):
+    """Filter each row of logits [rows, vocab] (top-k, then top-p, softmax).
+
+    Returns dict(ids [rows, cap] int32, probs [rows, cap] float32, count [rows],
+    flags [rows] uint32 as int32, and sample [rows] when rng=(seed, cycle),
+    dense [rows, vocab] when dense=True)."""
+    lib = load_library()
+    host = not logits.is_cuda
+    device = _device_of(logits)
+    x = _dev(logits, device)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("logits must be [rows, vocab] with unit inner stride")
+    rows, vocab = x.shape
+    if cap is None:
+        cap = min(int(top_k), vocab)
+    stream = torch.cuda.current_stream(device)
+    kw = dict(dtype=torch.int32, device=device)
+    ids = torch.empty((rows, cap), **kw)
+    probs = torch.empty((rows, cap), dtype=torch.float32, device=device)
+    count = torch.empty(rows, **kw)
+    flags = torch.empty(rows, **kw)
+    dn = torch.empty((rows, vocab), dtype=torch.float32, device=device) if dense else None
+    sample = torch.empty(rows, **kw) if rng is not None else None
+    rng_c = ctypes.byref(_rng(rng)) if rng is not None else None
+    nbytes = lib.uno_filter_softmax_workspace_bytes(rows, vocab, int(top_k))
+    ws = workspace(nbytes, device, stream)
+    st = lib.uno_filter_softmax(_ptr(x), _dtype_code(x), rows, vocab, x.stride(0), int(rows_per_request),
+                                _Params(float(temperature), int(top_k), float(top_p)), int(cap), _ptr(ids),
+                                _ptr(probs), _ptr(count), _ptr(dn), rng_c, _ptr(sample), _ptr(flags),
+                                _ptr(ws), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
+    _check("uno_filter_softmax", st)
+    out = dict(ids=ids, probs=probs, count=count, flags=flags)
+    if dense:
+        out["dense"] = dn
+    if rng is not None:
+        out["sample"] = sample
+    return _host_back(out, host)
+
+
+def uno_linear_verify(target_logits, draft_ids, q_ids, q_probs, q_count, *, R, B, temperature, top_k, top_p,
+                      rng):
+    """Linear rejection sampling.  target_logits [R*(B+1), vocab] (or
+    [R, B+1, vocab]); draft_ids [R, B]; q_* as returned by uno_filter_softmax
+    for the R*B draft rows.  Returns dict(tokens [R, B+1], accept_len,
+    num_tokens, flags)."""
+    lib = load_library()
+    host = not target_logits.is_cuda
+    device = _device_of(target_logits, draft_ids, q_ids)
+    x = _dev(target_logits, device).contiguous()
+    vocab = x.shape[-1]
+    if x.numel() != R * (B + 1) * vocab:
+        raise ValueError("target_logits must hold R*(B+1) rows")
+    d = _dev(draft_ids, device).to(torch.int32).contiguous()
+    qi = _dev(q_ids, device).to(torch.int32).contiguous()
+    qp = _dev(q_probs, device).to(torch.float32).contiguous()
+    qc = _dev(q_count, device).to(torch.int32).contiguous()
+    if d.numel() != R * B or qi.shape[0] != R * B or qc.numel() != R * B:
+        raise ValueError("draft_ids / q rows must cover R*B draft positions")
+    stream = torch.cuda.current_stream(device)
+    kw = dict(dtype=torch.int32, device=device)
+    toks = torch.empty((R, B + 1), **kw)
+    acc = torch.empty(R, **kw)
+    ntok = torch.empty(R, **kw)
+    flags = torch.empty(R, **kw)
+    nbytes = lib.uno_linear_verify_workspace_bytes(R, B, vocab, int(top_k))
+    ws = workspace(nbytes, device, stream)
+    st = lib.uno_linear_verify(_ptr(x), _dtype_code(x), R, B, vocab,
+                               _Params(float(temperature), int(top_k), float(top_p)), _ptr(d), _ptr(qi),
+                               _ptr(qp), _ptr(qc), qi.shape[1], _rng(rng), _ptr(toks),
+                               _ptr(acc), _ptr(ntok), _ptr(flags), _ptr(ws), ws.numel(),
+                               ctypes.c_void_p(stream.cuda_stream))
+    _check("uno_linear_verify", st)
+    return _host_back(dict(tokens=toks, accept_len=acc, num_tokens=ntok, flags=flags), host)
+
+
+def uno_tree_topk_expand(q_ids, q_probs, q_count, *, R, B, K, V):
+    """Top-K candidates per marginal and best-first V-node trees.  Returns
+    dict(node_token, node_parent, node_depth [R, V] int32, node_score [R, V]
+    float32, num_nodes [R])."""
+    lib = load_library()
+    host = not q_ids.is_cuda
+    device = _device_of(q_ids)
+    qi = _dev(q_ids, device).to(torch.int32).contiguous()
+    qp = _dev(q_probs, device).to(torch.float32).contiguous()
+    qc = _dev(q_count, device).to(torch.int32).contiguous()
+    if qi.shape[0] != R * B:
+        raise ValueError("q rows must cover R*B marginals")
+    stream = torch.cuda.current_stream(device)
+    kw = dict(dtype=torch.int32, device=device)
+    tok = torch.empty((R, V), **kw)
+    par = torch.empty((R, V), **kw)
+    dep = torch.empty((R, V), **kw)
+    sco = torch.empty((R, V), dtype=torch.float32, device=device)
+    nn = torch.empty(R, **kw)
+    st = lib.uno_tree_topk_expand(_ptr(qi), _ptr(qp), _ptr(qc), qi.shape[1], R, B, K, V, _ptr(tok), _ptr(par),
+                                  _ptr(dep), _ptr(sco), _ptr(nn), ctypes.c_void_p(stream.cuda_stream))
+    _check("uno_tree_topk_expand", st)
+    return _host_back(dict(node_token=tok, node_parent=par, node_depth=dep, node_score=sco, num_nodes=nn), host)
+
+
+def uno_tree_verify(target_logits, node_token, node_parent, num_nodes, *, R, B, V, temperature, top_k, top_p,
+                    rng):
+    """Target-only tree verification.  target_logits [R*V, vocab] (one row
+    per node).  Returns dict(tokens [R, B+1], accept_len, num_tokens,
+    path_nodes [R, B+1], flags)."""
+    lib = load_library()
+    host = not target_logits.is_cuda
+    device = _device_of(target_logits, node_token)
+    x = _dev(target_logits, device).contiguous()
+    vocab = x.shape[-1]
+    if x.numel() != R * V * vocab:
+        raise ValueError("target_logits must hold R*V rows")
+    tk = _dev(node_token, device).to(torch.int32).contiguous()
+    pa = _dev(node_parent, device).to(torch.int32).contiguous()
+    nn = _dev(num_nodes, device).to(torch.int32).contiguous()
+    stream = torch.cuda.current_stream(device)
+    kw = dict(dtype=torch.int32, device=device)
+    toks = torch.empty((R, B + 1), **kw)
+    path = torch.empty((R, B + 1), **kw)
+    acc = torch.empty(R, **kw)
+    ntok = torch.empty(R, **kw)
+    flags = torch.empty(R, **kw)
+    nbytes = lib.uno_tree_verify_workspace_bytes(R, V, vocab, int(top_k))
+    ws = workspace(nbytes, device, stream)
+    st = lib.uno_tree_verify(_ptr(x), _dtype_code(x), R, B, V, vocab,
+                             _Params(float(temperature), int(top_k), float(top_p)), _ptr(tk), _ptr(pa), _ptr(nn),
+                             _rng(rng), _ptr(toks), _ptr(acc), _ptr(ntok), _ptr(path),
+                             _ptr(flags), _ptr(ws), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
+    _check("uno_tree_verify", st)
+    return _host_back(dict(tokens=toks, accept_len=acc, num_tokens=ntok, path_nodes=path, flags=flags), host)

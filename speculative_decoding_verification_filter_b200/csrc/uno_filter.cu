@@ -1,0 +1,1809 @@
+// uno_filter.cu -- libuno_filter: UNO's per-cycle sampling and verification
+// step on sm_100a, behind the C ABI of include/uno_filter.h.
+//
+// Hot path.  Every entry point that reads logits runs one row kernel: a CTA
+// (or `S` CTAs, for few rows) streams one row of vocabulary logits from HBM
+// exactly once with 16-byte non-allocating loads, keeps only the elements that
+// can still be among the row's top_k (a per-warp candidate buffer in shared
+// memory behind a threshold the warps share), and finishes the row with an
+// exact top-k select, a double-precision softmax over the kept support, the
+// top-p cut and renormalisation, and then, depending on the entry point:
+//   * filter:  write the compact row (and the dense row / one draw);
+//   * linear:  write the compact target row to the workspace; the last CTA of
+//              a request runs the request's accept / residual / bonus steps;
+//   * tree:    the same, the last CTA walks the request's tree.
+// No tensor cores: nothing on this path is a contraction.  The filter order
+// (top-k, renormalise, then top-p) follows the UNO PR page's review thread;
+// the verification rules follow its "Motivation" and "Modifications"
+// sections (see include/uno_filter.h for the full statement).
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <climits>
+#include <cmath>
+#include <cstddef>
+#include <mutex>
+
+#include "uno_filter.h"
+#include "uno_device.cuh"
+
+namespace uno {
+
+enum Mode { kModeFilter = 0, kModeLinear = 1, kModeTree = 2 };
+
+
+struct RowJob {
+    // logits and shape
+    const unsigned char* logits;
+    int64_t rows, vocab, row_stride;  // row_stride in elements
+    int32_t rpr;                      // rows per request
+    int32_t S;                        // CTAs per row
+    // sampling parameters
+    float temperature, top_p;
+    int32_t k;                        // min(top_k, vocab)
+    int32_t hw, cap_w;                // warp buffer high-water mark / capacity
+    int32_t merge_cap;                // entries of the merge area
+    int32_t fin_off;                  // shared-memory offset of the finishing area (0: the ring)
+    // filter outputs
+    int32_t* out_ids;
+    float* out_probs;
+    int32_t* out_count;
+    int32_t cap;
+    float* out_dense;
+    int32_t* out_sample;
+    uint32_t* out_flags;
+    int32_t has_rng;
+    uint64_t seed;
+    uint32_t cycle;
+    uint32_t first_request;  // global index of request 0 of this call
+    // workspace
+    uint32_t* row_ticket;
+    uint32_t* req_ticket;
+    uint64_t* part_keys;   // [rows*S][k]
+    int32_t* part_count;   // [rows*S]
+    uint32_t* part_flags;  // [rows*S]
+    int32_t* c_ids;        // [rows][k]   compact target rows (verifiers)
+    float* c_probs;        // [rows][k]
+    int32_t* c_count;      // [rows]
+    uint32_t* c_flags;     // [rows]
+    // linear verification
+    int32_t B;
+    const int32_t* draft_ids;
+    const int32_t* q_ids;
+    const float* q_probs;
+    const int32_t* q_count;
+    int32_t q_cap;
+    int32_t* out_tokens;
+    int32_t* out_accept_len;
+    int32_t* out_num_tokens;
+    uint32_t* out_req_flags;
+    // tree verification
+    int32_t V;
+    const int32_t* node_token;
+    const int32_t* node_parent;
+    const int32_t* num_nodes;
+    int32_t* out_path_nodes;
+};
+
+// ---------------------------------------------------------------------------
+// Element traits.  A lane examines 16-byte units (8 bf16 or 4 fp32), four
+// per ring stage.
+// ---------------------------------------------------------------------------
+constexpr int kUnits = 4;  // 16-byte units per lane per stage
+
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr int kPerUnit = 8;
+    static constexpr int kBytes = 2;
+    typedef __nv_bfloat162 Tau;
+    __device__ static Tau make_tau(float t) {
+        const __nv_bfloat16 b = __float2bfloat16_rd(t);  // largest bf16 <= t
+        return __halves2bfloat162(b, b);
+    }
+    __device__ static __nv_bfloat162 w2(uint32_t w) { return *reinterpret_cast<const __nv_bfloat162*>(&w); }
+    // elementwise maximum of a unit (NaN propagates)
+    __device__ static __nv_bfloat162 umax(const uint4& r) {
+        return __hmax2_nan(__hmax2_nan(w2(r.x), w2(r.y)), __hmax2_nan(w2(r.z), w2(r.w)));
+    }
+    // true when some element of the unit may be >= tau, or is NaN
+    __device__ static bool maybe(const uint4& r, Tau tau) { return !__hblt2(umax(r), tau); }
+    __device__ static bool chunk_maybe(const uint4* c, Tau tau) {
+        return !__hblt2(__hmax2_nan(__hmax2_nan(umax(c[0]), umax(c[1])), __hmax2_nan(umax(c[2]), umax(c[3]))), tau);
+    }
+    __device__ static float get(const uint4& r, int e) {
+        const uint32_t w = (e < 2) ? r.x : (e < 4) ? r.y : (e < 6) ? r.z : r.w;
+        return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+    }
+    __device__ static float load_scalar(const unsigned char* p) {
+        const uint16_t h = *reinterpret_cast<const uint16_t*>(p);
+        return __uint_as_float((uint32_t)h << 16);
+    }
+    __device__ static uint4 neg_inf_unit() { return make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u); }
+    // Running top-2 of a lane's elements (per bf16x2 half); NaN is skipped
+    // by the min/max, the -inf fill never counts, and +inf only arises in a
+    // row that is flagged non-finite anyway.
+    typedef __nv_bfloat162 Top;
+    __device__ static Top top_init() {
+        const __nv_bfloat16 ninf = __ushort_as_bfloat16((unsigned short)0xff80u);
+        return __halves2bfloat162(ninf, ninf);
+    }
+    __device__ static void top2_update(Top& m1, Top& m2, const uint4* c) {
+#pragma unroll
+        for (int u = 0; u < kUnits; ++u) {
+            const uint32_t w[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const __nv_bfloat162 x = w2(w[q]);
+                const __nv_bfloat162 t = __hmin2(m1, x);
+                m1 = __hmax2(m1, x);
+                m2 = __hmax2(m2, t);
+            }
+        }
+    }
+    // ordered bits of the second largest tracked element, 0 when there is none
+    __device__ static uint32_t second_ord(Top m1, Top m2) {
+        const float a1 = __low2float(m1), b1 = __high2float(m1), a2 = __low2float(m2), b2 = __high2float(m2);
+        const float second = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
+        if (!(second > -__int_as_float(0x7f800000))) return 0u;
+        return ord_of_float(__fadd_rn(second, 0.0f));
+    }
+    // ordered bits of the lane's two largest tracked elements (0 = none)
+    __device__ static void lane_top2_ord(Top m1, Top m2, uint32_t& t1, uint32_t& t2) {
+        const float a1 = __low2float(m1), b1 = __high2float(m1), a2 = __low2float(m2), b2 = __high2float(m2);
+        const float first = fmaxf(a1, b1);
+        const float second = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
+        t1 = (first > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(first, 0.0f)) : 0u;
+        t2 = (second > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(second, 0.0f)) : 0u;
+    }
+    // bit u*8+e set when element e of unit u is >= tau (rounded down) or NaN
+    __device__ static unsigned cand_mask4(const uint4* c, Tau tau) {
+        unsigned m = 0;
+#pragma unroll
+        for (int u = 0; u < kUnits; ++u) {
+            if (maybe(c[u], tau)) {
+                const uint32_t w[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const unsigned g = __hgeu2_mask(w2(w[q]), tau);
+                    m |= ((g & 1u) | ((g >> 15) & 2u)) << (u * 8 + 2 * q);
+                }
+            }
+        }
+        return m;
+    }
+    // bit u*8+e set when element e of unit u is >= tau (rounded down) or NaN
+    __device__ static unsigned cand_mask(const uint4* c, Tau tau) {
+        unsigned m = 0;
+#pragma unroll
+        for (int u = 0; u < kUnits; ++u) {
+            if (maybe(c[u], tau)) {
+                const uint32_t w[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const unsigned g = __hgeu2_mask(w2(w[q]), tau);
+                    m |= ((g & 1u) | ((g >> 15) & 2u)) << (u * 8 + 2 * q);
+                }
+            }
+        }
+        return m;
+    }
+};
+
+template <>
+struct Elem<float> {
+    static constexpr int kPerUnit = 4;
+    static constexpr int kBytes = 4;
+    typedef float Tau;
+    __device__ static Tau make_tau(float t) { return t; }
+    __device__ static float max_nan(float a, float b) {
+        float r;
+        asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+        return r;
+    }
+    __device__ static float umax(const uint4& r) {
+        return max_nan(max_nan(__uint_as_float(r.x), __uint_as_float(r.y)),
+                       max_nan(__uint_as_float(r.z), __uint_as_float(r.w)));
+    }
+    __device__ static bool maybe(const uint4& r, Tau tau) { return !(umax(r) < tau); }
+    __device__ static bool chunk_maybe(const uint4* c, Tau tau) {
+        return !(max_nan(max_nan(umax(c[0]), umax(c[1])), max_nan(umax(c[2]), umax(c[3]))) < tau);
+    }
+    __device__ static float get(const uint4& r, int e) {
+        const uint32_t w = (e == 0) ? r.x : (e == 1) ? r.y : (e == 2) ? r.z : r.w;
+        return __uint_as_float(w);
+    }
+    __device__ static float load_scalar(const unsigned char* p) { return *reinterpret_cast<const float*>(p); }
+    __device__ static uint4 neg_inf_unit() { return make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u); }
+    typedef float Top;
+    __device__ static Top top_init() { return -__int_as_float(0x7f800000); }
+    __device__ static void top2_update(Top& m1, Top& m2, const uint4* c) {
+#pragma unroll
+        for (int u = 0; u < kUnits; ++u) {
+            const float x[4] = {__uint_as_float(c[u].x), __uint_as_float(c[u].y), __uint_as_float(c[u].z),
+                                __uint_as_float(c[u].w)};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float t = fminf(m1, x[q]);
+                m1 = fmaxf(m1, x[q]);
+                m2 = fmaxf(m2, t);
+            }
+        }
+    }
+    __device__ static uint32_t second_ord(Top m1, Top m2) {
+        (void)m1;
+        if (!(m2 > -__int_as_float(0x7f800000))) return 0u;
+        return ord_of_float(__fadd_rn(m2, 0.0f));
+    }
+    __device__ static void lane_top2_ord(Top m1, Top m2, uint32_t& t1, uint32_t& t2) {
+        t1 = (m1 > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(m1, 0.0f)) : 0u;
+        t2 = (m2 > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(m2, 0.0f)) : 0u;
+    }
+    // bit u*4+e set when element e of unit u is >= tau or NaN
+    __device__ static unsigned cand_mask4(const uint4* c, Tau tau) {
+        unsigned m = 0;
+#pragma unroll
+        for (int u = 0; u < kUnits; ++u) {
+            const float x[4] = {__uint_as_float(c[u].x), __uint_as_float(c[u].y), __uint_as_float(c[u].z),
+                                __uint_as_float(c[u].w)};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) m |= (!(x[q] < tau) ? 1u : 0u) << (u * 4 + q);
+        }
+        return m;
+    }
+    // bit u*4+e set when element e of unit u is >= tau or NaN
+    __device__ static unsigned cand_mask(const uint4* c, Tau tau) {
+        unsigned m = 0;
+#pragma unroll
+        for (int u = 0; u < kUnits; ++u) {
+            const float x[4] = {__uint_as_float(c[u].x), __uint_as_float(c[u].y), __uint_as_float(c[u].z),
+                                __uint_as_float(c[u].w)};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) m |= (!(x[q] < tau) ? 1u : 0u) << (u * 4 + q);
+        }
+        return m;
+    }
+};
+
+// 32-byte streaming load (bypasses L1, 256-byte L2 prefetch hint).  The
+// address is 32-byte aligned.
+__device__ __forceinline__ void ld_stream32(const void* p, uint4& lo, uint4& hi) {
+    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+                 : "l"(p));
+}
+
+// Per-warp streaming state.  Candidates are appended by single lanes with a
+// shared-memory counter (*wcnt); cnt is the warp-uniform copy of it.
+struct WarpState {
+    uint64_t* buf;    // candidate keys (shared memory)
+    int* wcnt;        // this warp's candidate count (shared memory)
+    int cnt;          // warp-uniform copy of *wcnt
+    uint64_t tau;     // threshold key (warp-uniform): every key < tau is out
+    uint32_t bad;     // this lane saw NaN / +inf
+};
+
+struct Compacted {
+    int cnt;
+    uint64_t tau;
+};
+
+// Drop candidates below the threshold, cut to the k best if more remain, and
+// publish the threshold to the CTA.  Every threshold a warp holds is a lower
+// bound of the CTA's k-th best key, so dropping below it loses nothing.
+// Rare; kept out of line so the streaming loop stays small.
+__device__ __noinline__ Compacted warp_compact(uint64_t* buf, int* wcnt, int cnt, uint64_t tau, int k,
+                                               unsigned long long* s_tau, int lane) {
+    cnt = warp_keep_ge(buf, cnt, tau, lane);
+    if (cnt > k) {
+        const uint64_t t = warp_select_kth(buf, cnt, k, lane);
+        cnt = warp_keep_ge(buf, cnt, t, lane);
+        if (t > tau) tau = t;
+        if (lane == 0) atomicMax(s_tau, (unsigned long long)tau);
+    }
+    if (lane == 0) *wcnt = cnt;
+    __syncwarp();
+    return Compacted{cnt, tau};
+}
+
+// One lane's slow path for one 16-byte unit: append every finite element
+// whose key beats the threshold (ids id0 ..); flag NaN / +inf.
+template <typename T>
+__device__ __forceinline__ void append_lane_unit(const uint4& r, uint32_t id0, float tau_f, uint64_t tau,
+                                                 uint64_t* buf, int* wcnt, uint32_t& bad) {
+#pragma unroll
+    for (int e = 0; e < Elem<T>::kPerUnit; ++e) {
+        const float v = Elem<T>::get(r, e);
+        if (!(v < tau_f)) {  // v >= threshold value, or NaN
+            if (v != v || v == __int_as_float(0x7f800000)) {
+                bad = 1u;
+            } else if (v != -__int_as_float(0x7f800000)) {
+                const uint64_t key = make_key(v, id0 + (uint32_t)e);
+                if (key > tau) buf[atomicAdd(wcnt, 1)] = key;
+            }
+        }
+    }
+}
+
+// Geometry of a row: `head` scalar elements up to the first 16-byte boundary,
+// then nunit aligned 16-byte units, then the tail.
+struct RowGeom {
+    const unsigned char* base;  // first element of the row
+    int64_t head, nunit, tail_begin;
+};
+
+template <typename T>
+__device__ __forceinline__ RowGeom row_geom(const RowJob& J, int64_t row) {
+    RowGeom g;
+    g.base = J.logits + (size_t)row * (size_t)J.row_stride * Elem<T>::kBytes;
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(g.base);
+    int64_t head = (int64_t)(((16u - (addr & 15u)) & 15u) / Elem<T>::kBytes);
+    if (head > J.vocab) head = J.vocab;
+    g.head = head;
+    g.nunit = (J.vocab - head) / Elem<T>::kPerUnit;
+    g.tail_begin = head + g.nunit * Elem<T>::kPerUnit;
+    return g;
+}
+
+
+// Element j (0 .. kUnits*kPerUnit-1) of a lane's units, j not known at compile time.
+template <typename T>
+__device__ __forceinline__ float lane_elem(const uint4* c, int j) {
+    const int u = j / Elem<T>::kPerUnit;
+    const uint4 r = (u == 0) ? c[0] : (u == 1) ? c[1] : (u == 2) ? c[2] : c[3];
+    const int e = j % Elem<T>::kPerUnit;
+    if (Elem<T>::kBytes == 2) {
+        const int q = e >> 1;
+        const uint32_t w = (q == 0) ? r.x : (q == 1) ? r.y : (q == 2) ? r.z : r.w;
+        return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+    }
+    const uint32_t w = (e == 0) ? r.x : (e == 1) ? r.y : (e == 2) ? r.z : r.w;
+    return __uint_as_float(w);
+}
+
+// Streaming ring of the CTA.  A stage is kStageBytes of consecutive logits,
+// brought in by ONE bulk copy (TMA, no multicast) with an mbarrier tracking
+// its bytes.  Warp w owns bytes [w*2KB, (w+1)*2KB) of a stage: four rows of
+// 32 16-byte units, lane l taking unit l of each row (conflict-free shared
+// loads).  The last warp to finish with a stage refills it (a shared-memory
+// arrival counter: no warp ever waits for another to release a stage).
+constexpr int kStages = 2;
+constexpr int kStageBytes = 16384;
+constexpr int kStageUnits = kStageBytes / 16;         // 16-byte units per stage
+constexpr int kWarpUnits = kStageUnits / kWarps;      // 128 per warp per stage
+constexpr int kRowsPerWarp = kWarpUnits / 32;         // 4 = kUnits
+static_assert(kRowsPerWarp == kUnits, "one unit per lane per row");
+// Stages whose elements seed the CTA threshold; the CTA reads them twice
+// (seed, then select), the second time from L2.
+constexpr int kBootStages = 4;
+// Elements per lane handled at a time when a burst of candidates arrives.
+constexpr int kPiece = 4;
+
+struct Ring {
+    unsigned char* stages;  // [kStages][kStageBytes]
+    uint64_t* full;         // [kStages] mbarriers (bytes arrived)
+    int* done;              // [kStages] warps finished with the stage
+    const unsigned char* ubase;
+    int ub, ue;             // the CTA's 16-byte units
+    int nA, total;          // sequence: nA seed stages, then every stage
+};
+
+__device__ __forceinline__ int ring_stage_index(const Ring& R, int q) { return q < R.nA ? q : q - R.nA; }
+
+// one thread: start copying sequence element q into its stage buffer
+__device__ __forceinline__ void ring_issue(const Ring& R, int q) {
+    const int u0 = R.ub + ring_stage_index(R, q) * kStageUnits;
+    const int nu = (R.ue - u0) < kStageUnits ? (R.ue - u0) : kStageUnits;
+    const uint32_t bytes = (uint32_t)nu * 16u;
+    uint64_t* bar = R.full + (q % kStages);
+    mbar_expect_tx(bar, bytes);
+    bulk_g2s(R.stages + (q % kStages) * kStageBytes, R.ubase + (size_t)u0 * 16, bytes, bar);
+}
+
+// Wait for sequence element q and load this warp's lane units (the -inf fill
+// past the end of the slice).  Returns false if the wait gave up.
+template <typename T>
+__device__ __forceinline__ bool ring_take(const Ring& R, int q, int warp, int lane, uint4* c) {
+    uint64_t* bar = R.full + (q % kStages);
+    const uint32_t par = (uint32_t)((q / kStages) & 1);
+    bool got = mbar_try_wait(bar, par);
+    if (!got) got = mbar_wait_bounded(bar, par);
+    const bool ok = __all_sync(kFull, got);
+    const int u0 = R.ub + ring_stage_index(R, q) * kStageUnits + warp * kWarpUnits + lane;
+    const uint4* sp = reinterpret_cast<const uint4*>(R.stages + (q % kStages) * kStageBytes) + warp * kWarpUnits + lane;
+#pragma unroll
+    for (int u = 0; u < kUnits; ++u) c[u] = (ok && u0 + u * 32 < R.ue) ? sp[u * 32] : Elem<T>::neg_inf_unit();
+    return ok;
+}
+
+// After every lane of the warp has used its units (its shared loads are
+// complete): count the warp out of the stage; the last warp refills it.
+__device__ __forceinline__ void ring_release(const Ring& R, int q, int lane) {
+    __syncwarp();
+    if (lane == 0) {
+        int* d = R.done + (q % kStages);
+        if (atomicAdd(d, 1) == kWarps - 1) {
+            atomicExch(d, 0);
+            if (q + kStages < R.total) {
+                fence_proxy_async();
+                ring_issue(R, q + kStages);
+            }
+        }
+    }
+}
+
+// After a timeout: wait (bounded) for the copies that may still be in flight.
+__device__ __forceinline__ void ring_drain(const Ring& R, int q) {
+    for (int d = q; d < R.total && d < q + kStages; ++d)
+        (void)mbar_wait_bounded(R.full + (d % kStages), (uint32_t)((d / kStages) & 1));
+}
+
+// Element id of bit j of a lane's mask (unit j / kPerUnit, element j % kPerUnit).
+template <typename T>
+__device__ __forceinline__ uint32_t lane_id(uint32_t uid0, int j) {
+    return (uid0 + (uint32_t)(j / Elem<T>::kPerUnit) * 32u) * Elem<T>::kPerUnit + (uint32_t)(j % Elem<T>::kPerUnit);
+}
+
+// Append the candidates of mask cm (bit j = element j of the lane's units;
+// uid0 = the lane's first unit, relative to element 0 of the row's units).
+template <typename T>
+__device__ __forceinline__ void append_mask(WarpState& ws, unsigned cm, const uint4* c, uint32_t id_base,
+                                            uint32_t uid0) {
+    while (cm) {
+        const int j = __ffs(cm) - 1;
+        cm &= cm - 1;
+        const float x = lane_elem<T>(c, j);
+        if (x != x || x == __int_as_float(0x7f800000)) {
+            ws.bad |= 1u;
+        } else if (x != -__int_as_float(0x7f800000)) {
+            const uint64_t key = make_key(x, id_base + lane_id<T>(uid0, j));
+            if (key > ws.tau) ws.buf[atomicAdd(ws.wcnt, 1)] = key;
+        }
+    }
+}
+
+// Stream this CTA's share of the row: 16-byte units [ub, ue) plus, for split
+// 0, the head and tail scalars.  All threads of the CTA call it.  ws.bad gets
+// bit 0 for a NaN / +inf logit, bit 1 when a wait gave up.
+//
+// Phase A (threshold seed): every lane tracks the two largest elements of its
+// share of the first kBootStages stages; the k-th largest of those (real,
+// distinct) elements is a valid lower bound of the CTA's k-th largest
+// (k <= 2*kThreads).
+// Phase B (select): every stage again; a lane whose units may hold an element
+// >= the threshold (or a NaN) appends its candidates; a warp whose buffer
+// passes the high-water mark cuts it to its best k, which raises the
+// threshold for the whole CTA.
+template <typename T>
+__device__ void scan_slice(const RowJob& J, const RowGeom& g, int64_t ub64, int64_t ue64, bool do_scalars,
+                           WarpState& ws, unsigned long long* s_tau, const Ring& ring_in, uint64_t* boot, int warp,
+                           int lane) {
+    typedef typename Elem<T>::Tau Tau;
+    constexpr int NE = kUnits * Elem<T>::kPerUnit;  // elements per lane per stage
+    Ring R = ring_in;
+    R.ubase = g.base + (size_t)g.head * Elem<T>::kBytes;  // 16-byte aligned
+    R.ub = (int)ub64;                                     // unit indices fit in 32 bits
+    R.ue = (int)ue64;
+    const int nstage = (R.ue - R.ub + kStageUnits - 1) / kStageUnits;
+    R.nA = nstage < kBootStages ? nstage : kBootStages;
+    R.total = R.nA + nstage;
+    const uint32_t id_base = (uint32_t)g.head;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(R.full + s, 1);
+            R.done[s] = 0;
+        }
+        fence_mbar_init();
+        for (int q = 0; q < kStages && q < R.total; ++q) ring_issue(R, q);
+    }
+    __syncthreads();
+
+    bool ok = true;
+    int q = 0;
+    // ---- phase A: seed the threshold
+    {
+        typename Elem<T>::Top m1 = Elem<T>::top_init(), m2 = m1;
+        for (; q < R.nA; ++q) {
+            uint4 c[kUnits];
+            ok = ring_take<T>(R, q, warp, lane, c);
+            if (!ok) break;
+            Elem<T>::top2_update(m1, m2, c);
+            ring_release(R, q, lane);
+        }
+        uint32_t t1, t2;
+        Elem<T>::lane_top2_ord(m1, m2, t1, t2);
+        // the k-th largest lane maximum: at least k (distinct) elements are
+        // >= it, so it is a valid lower bound of the CTA's k-th largest
+        uint32_t* bv = reinterpret_cast<uint32_t*>(boot);
+        bv[threadIdx.x] = t1;  // 0: no element
+        __syncthreads();
+        if (J.k <= kThreads && t1 > kOrdNegInf) {
+            int gt = 0, ge = 0;
+            for (int j = 0; j < kThreads; j += 8) {
+                const uint4 a = *reinterpret_cast<const uint4*>(bv + j);
+                const uint4 b = *reinterpret_cast<const uint4*>(bv + j + 4);
+                const uint32_t v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    gt += v[q] > t1;
+                    ge += v[q] >= t1;
+                }
+            }
+            if (gt < J.k && J.k <= ge) *s_tau = (uint64_t)t1 << 32;  // every writer holds the same value
+        }
+        (void)t2;
+        __syncthreads();
+        ws.tau = *reinterpret_cast<volatile unsigned long long*>(s_tau);
+    }
+
+    // row head / tail scalars (split 0, warp 0)
+    if (do_scalars && warp == 0) {
+        const int64_t ntail = J.vocab - g.tail_begin;
+        const int64_t nsc = g.head + ntail;  // < 2 * 8 = 16
+        if (lane < nsc) {
+            const int64_t id = (lane < g.head) ? (int64_t)lane : g.tail_begin + (lane - g.head);
+            const float v = Elem<T>::load_scalar(g.base + (size_t)id * Elem<T>::kBytes);
+            if (v != v || v == __int_as_float(0x7f800000)) {
+                ws.bad |= 1u;
+            } else if (v != -__int_as_float(0x7f800000)) {
+                const uint64_t key = make_key(v, (uint32_t)id);
+                if (key > ws.tau) ws.buf[atomicAdd(ws.wcnt, 1)] = key;
+            }
+        }
+        __syncwarp();
+        ws.cnt = *reinterpret_cast<volatile int*>(ws.wcnt);
+    }
+
+    // ---- phase B: select
+    Tau tau_v = Elem<T>::make_tau(tau_value(ws.tau));
+    float tau_f = tau_value(ws.tau);
+    for (; ok && q < R.total; ++q) {
+        uint4 c[kUnits];
+        ok = ring_take<T>(R, q, warp, lane, c);
+        if (!ok) break;
+        bool need = false;
+#pragma unroll
+        for (int u = 0; u < kUnits; ++u) need |= Elem<T>::maybe(c[u], tau_v);
+        if (__any_sync(kFull, need)) {
+            const uint32_t uid0 = (uint32_t)(R.ub + ring_stage_index(R, q) * kStageUnits + warp * kWarpUnits + lane);
+            unsigned cm = need ? Elem<T>::cand_mask4(c, tau_v) : 0u;
+            const int nc = (int)__reduce_add_sync(kFull, (unsigned)__popc(cm));
+            if (ws.cnt + nc <= J.cap_w) {
+                append_mask<T>(ws, cm, c, id_base, uid0);
+                __syncwarp();
+                ws.cnt = *reinterpret_cast<volatile int*>(ws.wcnt);
+            } else {
+                // a burst: kPiece elements per lane at a time, compacting between
+#pragma unroll 1
+                for (int p = 0; p < NE; p += kPiece) {
+                    if (ws.cnt > J.hw) {
+                        const Compacted cp = warp_compact(ws.buf, ws.wcnt, ws.cnt, ws.tau, J.k, s_tau, lane);
+                        ws.cnt = cp.cnt;
+                        ws.tau = cp.tau;
+                        tau_v = Elem<T>::make_tau(tau_value(ws.tau));
+                        tau_f = tau_value(ws.tau);
+                    }
+                    unsigned pm = 0;
+                    for (int e = 0; e < kPiece; ++e) pm |= (!(lane_elem<T>(c, p + e) < tau_f) ? 1u : 0u) << (p + e);
+                    append_mask<T>(ws, pm, c, id_base, uid0);
+                    __syncwarp();
+                    ws.cnt = *reinterpret_cast<volatile int*>(ws.wcnt);
+                }
+            }
+            if (ws.cnt > J.hw) {
+                const Compacted cp = warp_compact(ws.buf, ws.wcnt, ws.cnt, ws.tau, J.k, s_tau, lane);
+                ws.cnt = cp.cnt;
+                ws.tau = cp.tau;
+                tau_v = Elem<T>::make_tau(tau_value(ws.tau));
+                tau_f = tau_value(ws.tau);
+            }
+        }
+        ring_release(R, q, lane);
+        // adopt a better threshold found by another warp of this CTA
+        const unsigned long long st = *reinterpret_cast<volatile unsigned long long*>(s_tau);
+        if (st > ws.tau) {
+            ws.tau = st;
+            tau_v = Elem<T>::make_tau(tau_value(ws.tau));
+            tau_f = tau_value(ws.tau);
+        }
+    }
+    if (!ok) {
+        ring_drain(R, q);
+        ws.bad |= 2u;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Request tails (one warp of the last CTA of a request).
+// ---------------------------------------------------------------------------
+
+// Probability of `tok` in a compact row with ascending ids (binary search).
+__device__ __forceinline__ double lookup_sorted(const int32_t* ids, const float* probs, int n, int32_t tok) {
+    int lo = 0, hi = n - 1;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        const int32_t m = __ldcg(ids + mid);
+        if (m == tok) return (double)__ldcg(probs + mid);
+        if (m < tok)
+            lo = mid + 1;
+        else
+            hi = mid - 1;
+    }
+    return 0.0;
+}
+
+__device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd, int lane) {
+    const int32_t B = J.B;
+    const int64_t base = (int64_t)r * (B + 1);
+    const int kc = J.k;
+    uint32_t flags = 0;
+    for (int i = lane; i <= B; i += 32) flags |= __ldcg(J.c_flags + base + i);
+    flags = __reduce_or_sync(kFull, flags);
+    int32_t acc = B, ntok = B + 1;
+    int32_t* toks = J.out_tokens + (size_t)r * (B + 1);
+    for (int i = lane; i <= B; i += 32) toks[i] = -1;
+    __syncwarp();
+    bool stopped = false;
+    for (int i = 0; i < B && !stopped; ++i) {
+        const int pc = __ldcg(J.c_count + base + i);
+        const int32_t* pid = J.c_ids + (size_t)(base + i) * kc;
+        const float* ppr = J.c_probs + (size_t)(base + i) * kc;
+        if (pc == 0) {
+            acc = i;
+            ntok = i;
+            stopped = true;
+            break;
+        }
+        const int64_t qrow = (int64_t)r * B + i;
+        int qc = J.q_count[qrow];
+        qc = qc < 0 ? 0 : (qc > J.q_cap ? J.q_cap : qc);
+        const int32_t* qid = J.q_ids + (size_t)qrow * J.q_cap;
+        const float* qpr = J.q_probs + (size_t)qrow * J.q_cap;
+        const int32_t x = J.draft_ids[(size_t)r * B + i];
+        const bool xin = x >= 0 && (int64_t)x < J.vocab;
+        const double a = xin ? lookup_sorted(qid, qpr, qc, x) : 0.0;
+        const double px = xin ? lookup_sorted(pid, ppr, pc, x) : 0.0;
+        bool accept = false;
+        if (a > 0.0) {
+            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)i, kDrawAccept, J.cycle);
+            accept = (u * a < px);
+        } else {
+            flags |= kFlagDraftNotInSupport;
+        }
+        if (accept) {
+            if (lane == 0) toks[i] = x;
+            continue;
+        }
+        // residual max(0, p_i - q_i) over supp p_i (ascending ids)
+        for (int j = lane; j < pc; j += 32) {
+            const double d = (double)__ldcg(ppr + j) - lookup_sorted(qid, qpr, qc, __ldcg(pid + j));
+            wd[j] = d > 0.0 ? d : 0.0;
+        }
+        __syncwarp();
+        int pick = -1;
+        if (lane == 0) {
+            double tot = 0.0;
+            for (int j = 0; j < pc; ++j) tot += wd[j];
+            if (!(tot > 0.0)) {
+                flags |= kFlagResidualEmpty;
+                for (int j = 0; j < pc; ++j) wd[j] = (double)__ldcg(ppr + j);
+            }
+            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)i, kDrawResidual, J.cycle);
+            pick = inv_cdf_serial(wd, pc, u);
+            toks[i] = pick >= 0 ? __ldcg(pid + pick) : -1;
+        }
+        flags = __shfl_sync(kFull, flags, 0);
+        __syncwarp();
+        acc = i;
+        ntok = i + 1;
+        stopped = true;
+    }
+    if (!stopped) {
+        const int pc = __ldcg(J.c_count + base + B);
+        if (pc == 0) {
+            ntok = B;
+        } else if (lane == 0) {
+            const int32_t* pid = J.c_ids + (size_t)(base + B) * kc;
+            const float* ppr = J.c_probs + (size_t)(base + B) * kc;
+            for (int j = 0; j < pc; ++j) wd[j] = (double)__ldcg(ppr + j);
+            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)B, kDrawTarget, J.cycle);
+            const int pick = inv_cdf_serial(wd, pc, u);
+            toks[B] = pick >= 0 ? __ldcg(pid + pick) : -1;
+        }
+    }
+    if (lane == 0) {
+        J.out_accept_len[r] = acc;
+        J.out_num_tokens[r] = ntok;
+        J.out_req_flags[r] = flags;
+    }
+}
+
+__device__ __noinline__ void tree_tail(const RowJob& J, int32_t r, double* wd, int lane) {
+    const int32_t B = J.B, V = J.V;
+    const int64_t base = (int64_t)r * V;
+    const int kc = J.k;
+    int32_t n = J.num_nodes[r];
+    n = n < 1 ? 1 : (n > V ? V : n);
+    const int32_t* tk = J.node_token + (size_t)r * V;
+    const int32_t* pa = J.node_parent + (size_t)r * V;
+    uint32_t flags = 0;
+    for (int j = lane; j < n; j += 32) flags |= __ldcg(J.c_flags + base + j);
+    flags = __reduce_or_sync(kFull, flags);
+    int32_t* toks = J.out_tokens + (size_t)r * (B + 1);
+    int32_t* path = J.out_path_nodes + (size_t)r * (B + 1);
+    for (int t = lane; t <= B; t += 32) {
+        toks[t] = -1;
+        path[t] = -1;
+    }
+    __syncwarp();
+    int32_t j = 0, t = 0, acc = 0, ntok = 0;
+    for (;;) {
+        const int pc = __ldcg(J.c_count + base + j);
+        if (pc == 0) {
+            if (lane == 0) path[t] = j;
+            ntok = t;
+            acc = t;
+            break;
+        }
+        int32_t y = -1;
+        if (lane == 0) {
+            const int32_t* pid = J.c_ids + (size_t)(base + j) * kc;
+            const float* ppr = J.c_probs + (size_t)(base + j) * kc;
+            for (int q = 0; q < pc; ++q) wd[q] = (double)__ldcg(ppr + q);
+            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)j, kDrawTarget, J.cycle);
+            const int pick = inv_cdf_serial(wd, pc, u);
+            y = pick >= 0 ? __ldcg(pid + pick) : -1;
+            toks[t] = y;
+            path[t] = j;
+        }
+        y = __shfl_sync(kFull, y, 0);
+        __syncwarp();
+        ++t;
+        ntok = t;
+        acc = t - 1;
+        // the lowest-index child of j carrying token y
+        int32_t next = -1;
+        for (int c0 = 1; c0 < n && next < 0; c0 += 32) {
+            const int c = c0 + lane;
+            const bool hit = c < n && pa[c] == j && tk[c] == y;
+            const unsigned bal = __ballot_sync(kFull, hit);
+            if (bal) next = c0 + __ffs(bal) - 1;
+        }
+        if (next < 0 || t > B) break;
+        j = next;
+    }
+    if (lane == 0) {
+        J.out_accept_len[r] = acc;
+        J.out_num_tokens[r] = ntok;
+        J.out_req_flags[r] = flags;
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Finishing a row (all threads of the CTA).
+// ---------------------------------------------------------------------------
+struct FinishShared {
+    double S, W;
+    int kept, last, n;
+};
+
+// Exact top k of the unique keys uni[0..U): each key's rank is the number of
+// larger keys; ranks below k land in sel[rank], so sel comes out sorted
+// (descending).  All threads call it.
+__device__ __forceinline__ void cta_rank_topk(const uint64_t* uni, int U, int k, uint64_t* sel) {
+    for (int i = threadIdx.x; i < U; i += kThreads) {
+        const uint64_t key = uni[i];
+        int rank = 0;
+        int j = 0;
+        for (; j + 8 <= U; j += 8) {  // independent loads ahead of the compares
+            ulonglong2 p[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) p[q] = *reinterpret_cast<const ulonglong2*>(uni + j + 2 * q);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) rank += (p[q].x > key) + (p[q].y > key);
+        }
+        for (; j < U; ++j) rank += (uni[j] > key);
+        if (rank < k) sel[rank] = key;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Warp-level finishing for k <= 64: lane l holds ranks l and l + 32.  Sums
+// and scans run as warp reductions (a fixed order; it differs from a serial
+// sum only in the last bits, which can flip a decision only within the
+// boundary margin the library documents).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+__device__ __forceinline__ double warp_incl_scan_d(double v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+// Ascending bitonic sort of 64 keys, element e = lane in a, e = lane + 32 in b.
+__device__ __forceinline__ void warp_sort64(uint64_t& a, uint64_t& b, int lane) {
+#pragma unroll
+    for (int size = 2; size <= 64; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride == 32) {
+                const uint64_t lo = a < b ? a : b, hi = a < b ? b : a;
+                a = lo;
+                b = hi;
+            } else {
+                const uint64_t pa = __shfl_xor_sync(kFull, a, stride), pb = __shfl_xor_sync(kFull, b, stride);
+                const bool lower = (lane & stride) == 0;
+                const bool upa = size == 64 || (lane & size) == 0;
+                const bool upb = size == 64 || ((lane + 32) & size) == 0;
+                a = (lower == upa) ? (a < pa ? a : pa) : (a < pa ? pa : a);
+                b = (lower == upb) ? (b < pb ? b : pb) : (b < pb ? pb : b);
+            }
+        }
+    }
+}
+
+// First j (of weights wa at index lane, wb at lane + 32; ascending id order)
+// with u * S < prefix_j, else the last positive weight; -1 if all are zero.
+__device__ __forceinline__ int warp_inv_cdf(double wa, double wb, double u, int lane) {
+    const double S = warp_sum_d(wa + wb);
+    if (!(S > 0.0)) return -1;
+    const double x = u * S;
+    const double ia = warp_incl_scan_d(wa, lane);
+    const double ta = __shfl_sync(kFull, ia, 31);
+    const double ib = warp_incl_scan_d(wb, lane) + ta;
+    const unsigned ba = __ballot_sync(kFull, x < ia), bb = __ballot_sync(kFull, x < ib);
+    if (ba) return __ffs(ba) - 1;
+    if (bb) return 32 + __ffs(bb) - 1;
+    const unsigned pa = __ballot_sync(kFull, wa > 0.0), pb = __ballot_sync(kFull, wb > 0.0);
+    if (pb) return 32 + 31 - __clz(pb);
+    if (pa) return 31 - __clz(pa);
+    return -1;
+}
+
+template <int MODE>
+__device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n, uint32_t rowbad,
+                                const uint64_t* sel, double* wd, FinishShared& fs, int lane) {
+    const bool bad = rowbad != 0u || n == 0;
+    int kept = 0;
+    uint64_t oa = ~0ull, ob = ~0ull;  // (id, prob) pairs, ascending id after the sort
+    if (!bad) {
+        const uint64_t ka = lane < n ? sel[lane] : 0ull, kb = lane + 32 < n ? sel[lane + 32] : 0ull;
+        double wa = 0.0, wb = 0.0;
+        if (J.temperature == 0.0f) {
+            kept = 1;
+            wa = lane == 0 ? 1.0 : 0.0;
+        } else {
+            const double v0 = (double)key_value(sel[0]);
+            const double temp = (double)J.temperature;
+            if (lane < n) wa = exp(((double)key_value(ka) - v0) / temp);
+            if (lane + 32 < n) wb = exp(((double)key_value(kb) - v0) / temp);
+            if (J.top_p >= 1.0f) {
+                kept = n;
+            } else {
+                const double S = warp_sum_d(wa + wb);
+                const double pa = wa / S, pb = wb / S;
+                // mass before rank j
+                const double ia = warp_incl_scan_d(pa, lane);
+                const double ta = __shfl_sync(kFull, ia, 31);
+                const double ib = warp_incl_scan_d(pb, lane) + ta;
+                double ea = __shfl_up_sync(kFull, ia, 1), eb = __shfl_up_sync(kFull, ib, 1);
+                if (lane == 0) {
+                    ea = 0.0;
+                    eb = ta;
+                }
+                const double tp = (double)J.top_p;
+                const bool keepa = lane < n && (lane == 0 || ea < tp);
+                const bool keepb = lane + 32 < n && eb < tp;
+                kept = __popc(__ballot_sync(kFull, keepa)) + __popc(__ballot_sync(kFull, keepb));
+            }
+        }
+        const double ra = lane < kept ? wa : 0.0, rb = lane + 32 < kept ? wb : 0.0;
+        const double W = warp_sum_d(ra + rb);
+        if (lane < kept)
+            oa = ((uint64_t)(uint32_t)key_id(ka) << 32) | (uint64_t)__float_as_uint((float)(wa / W));
+        if (lane + 32 < kept)
+            ob = ((uint64_t)(uint32_t)key_id(kb) << 32) | (uint64_t)__float_as_uint((float)(wb / W));
+        warp_sort64(oa, ob, lane);
+    }
+    // bit 0 of rowbad: NaN / +inf (or no finite logit); bit 1: a wait gave up
+    const uint32_t rflags = !bad ? 0u : (rowbad & 2u) ? (kFlagTimeout | ((rowbad & 1u) ? kFlagNonfinite : 0u))
+                                                       : kFlagNonfinite;
+    if (MODE == kModeFilter) {
+        int32_t* ids = J.out_ids + (size_t)row * J.cap;
+        float* pr = J.out_probs + (size_t)row * J.cap;
+        // lanes write their own two slots, then the rest of the row's slots
+        if (lane < J.cap) {
+            ids[lane] = lane < kept ? (int32_t)(oa >> 32) : -1;
+            pr[lane] = lane < kept ? __uint_as_float((uint32_t)oa) : 0.0f;
+        }
+        if (lane + 32 < J.cap) {
+            ids[lane + 32] = lane + 32 < kept ? (int32_t)(ob >> 32) : -1;
+            pr[lane + 32] = lane + 32 < kept ? __uint_as_float((uint32_t)ob) : 0.0f;
+        }
+        for (int j = 64 + lane; j < J.cap; j += 32) {
+            ids[j] = -1;
+            pr[j] = 0.0f;
+        }
+        if (J.out_dense != nullptr) {
+            float* d = J.out_dense + (size_t)row * (size_t)J.vocab;
+            if (lane < kept) d[(int32_t)(oa >> 32)] = __uint_as_float((uint32_t)oa);
+            if (lane + 32 < kept) d[(int32_t)(ob >> 32)] = __uint_as_float((uint32_t)ob);
+        }
+        int32_t tok = -1;
+        if (J.has_rng && kept > 0) {
+            const double u = uniform53(J.seed, J.first_request + (uint32_t)(row / J.rpr), (uint32_t)(row % J.rpr),
+                                       kDrawProposal, J.cycle);
+            const double wa = lane < kept ? (double)__uint_as_float((uint32_t)oa) : 0.0;
+            const double wb = lane + 32 < kept ? (double)__uint_as_float((uint32_t)ob) : 0.0;
+            const int pick = warp_inv_cdf(wa, wb, u, lane);
+            if (pick >= 0) tok = (int32_t)(__shfl_sync(kFull, pick < 32 ? oa : ob, pick & 31) >> 32);
+        }
+        if (lane == 0) {
+            J.out_count[row] = kept;
+            J.out_flags[row] = rflags;
+            if (J.has_rng) J.out_sample[row] = tok;
+        }
+    } else {
+        int32_t* ids = J.c_ids + (size_t)row * J.k;
+        float* pr = J.c_probs + (size_t)row * J.k;
+        if (lane < kept) {
+            ids[lane] = (int32_t)(oa >> 32);
+            pr[lane] = __uint_as_float((uint32_t)oa);
+        }
+        if (lane + 32 < kept) {
+            ids[lane + 32] = (int32_t)(ob >> 32);
+            pr[lane + 32] = __uint_as_float((uint32_t)ob);
+        }
+        if (lane == 0) {
+            J.c_count[row] = kept;
+            J.c_flags[row] = rflags;
+        }
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            __threadfence();
+            const uint32_t t = atomicAdd(J.req_ticket + req, 1u);
+            last = (t == (uint32_t)(J.rpr - 1));
+            if (last) {
+                atomicExch(J.req_ticket + req, 0u);
+                __threadfence();
+            }
+        }
+        last = __shfl_sync(kFull, last, 0);
+        if (last) {
+            if (MODE == kModeLinear)
+                linear_tail(J, req, wd, lane);
+            else
+                tree_tail(J, req, wd, lane);
+        }
+    }
+}
+
+// Softmax in double over the sorted top n, top-p cut, renormalise, and write
+// the row (filter: output; verifiers: workspace + request tail).
+template <int MODE>
+__device__ void finish_row(const RowJob& J, int64_t row, int32_t req, int n, uint32_t rowbad, const uint64_t* sel,
+                           uint64_t* outk, double* wd, double* pd, FinishShared& fs, int warp, int lane) {
+    const int tid = threadIdx.x;
+    const bool bad = rowbad != 0u || n == 0;
+    int kept = 0;
+    if (!bad) {
+        const double v0 = (double)key_value(sel[0]);
+        if (J.temperature == 0.0f) {
+            kept = 1;
+            if (tid == 0) fs.W = 1.0;
+            if (tid == 0) wd[0] = 1.0;
+        } else {
+            const double temp = (double)J.temperature;
+            for (int j = tid; j < n; j += kThreads) wd[j] = exp(((double)key_value(sel[j]) - v0) / temp);
+            __syncthreads();
+            if (tid == 0) fs.S = serial_sum(wd, n);  // the defined (descending) order
+            __syncthreads();
+            const double S = fs.S;
+            for (int j = tid; j < n; j += kThreads) pd[j] = wd[j] / S;
+            __syncthreads();
+            if (tid == 0) {
+                int kk = 0;
+                if (J.top_p >= 1.0f) {
+                    kk = n;
+                } else {
+                    const double tp = (double)J.top_p;
+                    double m = 0.0;
+                    int j = 0;
+                    for (; j + 8 <= n; j += 8) {  // loads ahead of the dependent walk
+                        double b[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) b[q] = pd[j + q];
+                        bool stop = false;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (!stop) {
+                                if (j + q > 0 && !(m < tp)) {
+                                    stop = true;
+                                } else {
+                                    m += b[q];
+                                    ++kk;
+                                }
+                            }
+                        }
+                        if (stop) break;
+                    }
+                    if (kk == j) {
+                        for (; j < n; ++j) {
+                            if (j > 0 && !(m < tp)) break;
+                            m += pd[j];
+                            ++kk;
+                        }
+                    }
+                }
+                fs.kept = kk;
+                fs.W = serial_sum(wd, kk);
+            }
+        }
+        __syncthreads();
+        if (J.temperature != 0.0f) kept = fs.kept;
+        const double W = fs.W;
+        // (id, prob) pairs in ascending id order
+        for (int j = tid; j < kept; j += kThreads) {
+            const float p = (float)(wd[j] / W);
+            const uint32_t id = (uint32_t)key_id(sel[j]);
+            int r = 0;
+            int i = 0;
+            for (; i + 8 <= kept; i += 8) {
+                uint64_t b[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) b[q] = sel[i + q];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) r += ((uint32_t)key_id(b[q]) < id);
+            }
+            for (; i < kept; ++i) r += ((uint32_t)key_id(sel[i]) < id);
+            outk[r] = ((uint64_t)id << 32) | (uint64_t)__float_as_uint(p);
+        }
+        __syncthreads();
+    }
+    // bit 0 of rowbad: NaN / +inf (or no finite logit); bit 1: a wait gave up
+    const uint32_t rflags = !bad ? 0u : (rowbad & 2u) ? (kFlagTimeout | ((rowbad & 1u) ? kFlagNonfinite : 0u))
+                                                       : kFlagNonfinite;
+
+    if (MODE == kModeFilter) {
+        int32_t* ids = J.out_ids + (size_t)row * J.cap;
+        float* pr = J.out_probs + (size_t)row * J.cap;
+        for (int j = tid; j < J.cap; j += kThreads) {
+            if (j < kept) {
+                ids[j] = (int32_t)(outk[j] >> 32);
+                pr[j] = __uint_as_float((uint32_t)outk[j]);
+            } else {
+                ids[j] = -1;
+                pr[j] = 0.0f;
+            }
+        }
+        if (J.out_dense != nullptr) {
+            float* d = J.out_dense + (size_t)row * (size_t)J.vocab;
+            for (int j = tid; j < kept; j += kThreads) d[(int32_t)(outk[j] >> 32)] = __uint_as_float((uint32_t)outk[j]);
+        }
+        if (tid == 0) {
+            J.out_count[row] = kept;
+            J.out_flags[row] = rflags;
+            if (J.has_rng) {
+                int32_t tok = -1;
+                if (kept > 0) {
+                    for (int j = 0; j < kept; ++j) wd[j] = (double)__uint_as_float((uint32_t)outk[j]);
+                    const double u = uniform53(J.seed, J.first_request + (uint32_t)(row / J.rpr),
+                                               (uint32_t)(row % J.rpr), kDrawProposal, J.cycle);
+                    const int pick = inv_cdf_serial(wd, kept, u);
+                    tok = pick >= 0 ? (int32_t)(outk[pick] >> 32) : -1;
+                }
+                J.out_sample[row] = tok;
+            }
+        }
+    } else {
+        int32_t* ids = J.c_ids + (size_t)row * J.k;
+        float* pr = J.c_probs + (size_t)row * J.k;
+        for (int j = tid; j < kept; j += kThreads) {
+            ids[j] = (int32_t)(outk[j] >> 32);
+            pr[j] = __uint_as_float((uint32_t)outk[j]);
+        }
+        if (tid == 0) {
+            J.c_count[row] = kept;
+            J.c_flags[row] = rflags;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            const uint32_t t = atomicAdd(J.req_ticket + req, 1u);
+            fs.last = (t == (uint32_t)(J.rpr - 1));
+            if (fs.last) {
+                atomicExch(J.req_ticket + req, 0u);
+                __threadfence();
+            }
+        }
+        __syncthreads();
+        if (fs.last && warp == 0) {
+            if (MODE == kModeLinear)
+                linear_tail(J, req, wd, lane);
+            else
+                tree_tail(J, req, wd, lane);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The row kernel.
+// ---------------------------------------------------------------------------
+template <typename T, int MODE>
+__global__ void __launch_bounds__(kThreads, 4) row_kernel(const RowJob J) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    // streaming: ring stages | barriers | counters | warp buffers
+    unsigned char* stages = smem;                                                   // [kStages][kStageBytes]
+    uint64_t* full = reinterpret_cast<uint64_t*>(stages + kStages * kStageBytes);   // [kStages]
+    int* done = reinterpret_cast<int*>(full + kStages);                             // [kStages] (+pad)
+    uint64_t* wbufs = reinterpret_cast<uint64_t*>(full + 2 * kStages);
+    // finishing (after streaming): in the ring stages when it fits there
+    unsigned char* fin = J.fin_off ? smem + J.fin_off : smem;
+    uint64_t* uni = reinterpret_cast<uint64_t*>(fin);   // [merge_cap]
+    uint64_t* sel = uni + J.merge_cap;                  // [k]
+    uint64_t* outk = sel + J.k;                         // [k]
+    double* wd = reinterpret_cast<double*>(outk + J.k); // [k]
+    double* pd = wd + J.k;                              // [k]
+
+    __shared__ unsigned long long s_tau;
+    __shared__ int s_wcnt[kWarps];
+    __shared__ int s_cnt[kWarps];
+    __shared__ uint32_t s_bad;
+    __shared__ FinishShared fs;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = blockIdx.x / J.S;
+    const int split = (int)(blockIdx.x % J.S);
+    const int32_t req = (int32_t)(row / J.rpr);
+
+    // Tree rows past the request's node count are neither read nor used.
+    if (MODE == kModeTree) {
+        int32_t nn = J.num_nodes[req];
+        nn = nn < 1 ? 1 : (nn > J.V ? J.V : nn);
+        if ((int32_t)(row % J.V) >= nn) {
+            if (split != 0) return;
+            if (threadIdx.x == 0) {
+                __threadfence();
+                const uint32_t t = atomicAdd(J.req_ticket + req, 1u);
+                fs.last = (t == (uint32_t)(J.rpr - 1));
+                if (fs.last) {
+                    atomicExch(J.req_ticket + req, 0u);
+                    __threadfence();
+                }
+            }
+            __syncthreads();
+            if (fs.last && warp == 0) tree_tail(J, req, wd, lane);
+            return;
+        }
+    }
+
+    if (threadIdx.x == 0) {
+        s_tau = 0ull;
+        s_bad = 0u;
+    }
+    if (threadIdx.x < kWarps) s_wcnt[threadIdx.x] = 0;
+
+    const RowGeom g = row_geom<T>(J, row);
+    const int64_t per = (g.nunit + J.S - 1) / J.S;
+    const int64_t vb = per * split < g.nunit ? per * split : g.nunit;
+    const int64_t ve = vb + per < g.nunit ? vb + per : g.nunit;
+
+    // Zero the dense row over this CTA's element range before any value is
+    // written (the last CTA of the row writes the values after the ticket).
+    if (MODE == kModeFilter && J.out_dense != nullptr) {
+        const int64_t e0 = (split == 0) ? 0 : g.head + vb * Elem<T>::kPerUnit;
+        const int64_t e1 = (split == J.S - 1) ? J.vocab : g.head + ve * Elem<T>::kPerUnit;
+        float* d = J.out_dense + (size_t)row * (size_t)J.vocab;
+        for (int64_t e = e0 + threadIdx.x; e < e1; e += kThreads) d[e] = 0.0f;
+    }
+    __syncthreads();
+
+    WarpState ws;
+    ws.buf = wbufs + (size_t)warp * J.cap_w;
+    ws.wcnt = &s_wcnt[warp];
+    ws.cnt = 0;
+    ws.tau = 0ull;
+    ws.bad = 0u;
+    Ring ring;
+    ring.stages = stages;
+    ring.full = full;
+    ring.done = done;
+    scan_slice<T>(J, g, vb, ve, split == 0, ws, &s_tau, ring, wbufs, warp, lane);
+
+    // each warp drops what the CTA's threshold has ruled out
+    {
+        const unsigned long long st = *reinterpret_cast<volatile unsigned long long*>(&s_tau);
+        if (st > ws.tau) ws.tau = st;
+        ws.cnt = warp_keep_ge(ws.buf, ws.cnt, ws.tau, lane);
+    }
+    const uint32_t wbad = __reduce_or_sync(kFull, ws.bad);
+    if (lane == 0) {
+        s_cnt[warp] = ws.cnt;
+        if (wbad) atomicOr(&s_bad, wbad);
+    }
+    __syncthreads();
+    int U = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) U += s_cnt[w];
+    if (U > J.merge_cap) {  // rare: cut every warp to its own best k first
+        const Compacted cp = warp_compact(ws.buf, ws.wcnt, ws.cnt, ws.tau, J.k, &s_tau, lane);
+        ws.cnt = cp.cnt;
+        if (lane == 0) s_cnt[warp] = ws.cnt;
+        __syncthreads();
+        U = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) U += s_cnt[w];
+    }
+    {
+        int off = 0;
+        for (int w = 0; w < warp; ++w) off += s_cnt[w];
+        for (int i = lane; i < ws.cnt; i += 32) uni[off + i] = ws.buf[i];
+    }
+    __syncthreads();
+    cta_rank_topk(uni, U, J.k, sel);
+    int n = U < J.k ? U : J.k;
+    uint32_t rowbad = s_bad;
+    __syncthreads();
+
+    // Split rows: publish this CTA's best k; the last CTA of the row merges.
+    if (J.S > 1) {
+        const size_t pslot = (size_t)row * J.S + split;
+        uint64_t* pk = J.part_keys + pslot * J.k;
+        for (int i = threadIdx.x; i < n; i += kThreads) pk[i] = sel[i];
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            J.part_count[pslot] = n;
+            J.part_flags[pslot] = rowbad;
+            __threadfence();
+            const uint32_t t = atomicAdd(J.row_ticket + row, 1u);
+            fs.last = (t == (uint32_t)(J.S - 1));
+            if (fs.last) {
+                atomicExch(J.row_ticket + row, 0u);
+                __threadfence();
+            }
+        }
+        __syncthreads();
+        if (!fs.last) return;
+        U = 0;
+        rowbad = 0;
+        for (int s = 0; s < J.S; ++s) {
+            const size_t ps = (size_t)row * J.S + s;
+            const int c = __ldcg(J.part_count + ps);
+            rowbad |= __ldcg(J.part_flags + ps);
+            const unsigned long long* src = reinterpret_cast<const unsigned long long*>(J.part_keys + ps * J.k);
+            for (int i = threadIdx.x; i < c; i += kThreads) uni[U + i] = __ldcg(src + i);
+            U += c;
+        }
+        __syncthreads();
+        cta_rank_topk(uni, U, J.k, sel);
+        n = U < J.k ? U : J.k;
+        __syncthreads();
+    }
+
+    if (J.k <= 64) {
+        if (warp == 0) finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, fs, lane);
+    } else {
+        finish_row<MODE>(J, row, req, n, rowbad, sel, outk, wd, pd, fs, warp, lane);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Tree expansion: one warp per request.
+// ---------------------------------------------------------------------------
+struct TreeJob {
+    const int32_t* q_ids;
+    const float* q_probs;
+    const int32_t* q_count;
+    int32_t q_cap, R, B, K, V, sort_cap;
+    int32_t* node_token;
+    int32_t* node_parent;
+    int32_t* node_depth;
+    float* node_score;
+    int32_t* num_nodes;
+};
+
+__global__ void __launch_bounds__(32) tree_expand_kernel(const TreeJob J) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int B = J.B, K = J.K, V = J.V;
+    uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem);            // [sort_cap]
+    double* nscore = reinterpret_cast<double*>(sortbuf + J.sort_cap);  // [V]
+    double* fscore = nscore + V;                                       // [V + 1]
+    int32_t* cand_id = reinterpret_cast<int32_t*>(fscore + V + 1);     // [B*K]
+    float* cand_p = reinterpret_cast<float*>(cand_id + B * K);         // [B*K]
+    int32_t* ncand = reinterpret_cast<int32_t*>(cand_p + B * K);       // [B]
+    int32_t* fdep = ncand + B;                                         // [V + 1]
+    int32_t* fpar = fdep + V + 1;                                      // [V + 1]
+    int32_t* frank = fpar + V + 1;                                     // [V + 1]
+
+    const int lane = threadIdx.x;
+    const int r = blockIdx.x;
+
+    // 1. top-K of each marginal by (prob desc, id asc)
+    for (int d = 0; d < B; ++d) {
+        const int64_t row = (int64_t)r * B + d;
+        int c = J.q_count[row];
+        c = c < 0 ? 0 : (c > J.q_cap ? J.q_cap : c);
+        const int np2 = next_pow2(c < 1 ? 1 : c);
+        for (int i = lane; i < np2; i += 32) {
+            uint64_t key = 0ull;
+            if (i < c) {
+                const float p = __fadd_rn(J.q_probs[(size_t)row * J.q_cap + i], 0.0f);
+                const int32_t id = J.q_ids[(size_t)row * J.q_cap + i];
+                key = ((uint64_t)ord_of_float(p) << 32) | (uint64_t)(~(uint32_t)id);
+            }
+            sortbuf[i] = key;
+        }
+        __syncwarp();
+        warp_bitonic_sort(sortbuf, np2, true, lane);
+        const int nk = c < K ? c : K;
+        for (int i = lane; i < nk; i += 32) {
+            cand_id[d * K + i] = key_id(sortbuf[i]);
+            cand_p[d * K + i] = float_of_ord((uint32_t)(sortbuf[i] >> 32));
+        }
+        if (lane == 0) ncand[d] = nk;
+        __syncwarp();
+    }
+
+    int32_t* tok = J.node_token + (size_t)r * V;
+    int32_t* par = J.node_parent + (size_t)r * V;
+    int32_t* dep = J.node_depth + (size_t)r * V;
+    float* sco = J.node_score + (size_t)r * V;
+    for (int j = lane; j < V; j += 32) {
+        tok[j] = -1;
+        par[j] = -1;
+        dep[j] = -1;
+        sco[j] = 0.0f;
+    }
+    __syncwarp();
+
+    // 2. best-first expansion with a lazy frontier: a tree node keeps only its
+    // best unexpanded child in the frontier; popping a child brings in its own
+    // first child and its next sibling.  Scores never rise along those links
+    // and the tie order never falls, so this pops nodes in the same order as
+    // a frontier that holds every child.
+    int nf = 0;
+    if (lane == 0) {
+        nscore[0] = 1.0;
+        tok[0] = -1;
+        par[0] = -1;
+        dep[0] = 0;
+        sco[0] = 1.0f;
+        if (ncand[0] > 0) {
+            fscore[0] = 1.0 * (double)cand_p[0];
+            fdep[0] = 1;
+            fpar[0] = 0;
+            frank[0] = 0;
+            nf = 1;
+        }
+    }
+    nf = __shfl_sync(kFull, nf, 0);
+    __syncwarp();
+    int n = 1;
+    while (n < V && nf > 0) {
+        // lane-local best over entries lane, lane+32, ...
+        int best = -1;
+        double bs = 0.0;
+        uint32_t btie = 0xffffffffu;
+        for (int f = lane; f < nf; f += 32) {
+            const double s = fscore[f];
+            const uint32_t tie = ((uint32_t)fdep[f] << 24) | ((uint32_t)fpar[f] << 12) | (uint32_t)frank[f];
+            if (best < 0 || s > bs || (s == bs && tie < btie)) {
+                best = f;
+                bs = s;
+                btie = tie;
+            }
+        }
+        // warp maximum of the score, then the smallest tie key among lanes
+        // holding it (depth < 256, parent < 4096, rank < 4096)
+        double ms = best >= 0 ? bs : -1.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const double other = __shfl_xor_sync(kFull, ms, o);
+            ms = other > ms ? other : ms;
+        }
+        const uint32_t mytie = (best >= 0 && bs == ms) ? btie : 0xffffffffu;
+        const uint32_t mtie = __reduce_min_sync(kFull, mytie);
+        const unsigned owner_bal = __ballot_sync(kFull, best >= 0 && bs == ms && btie == mtie);
+        const int owner = __ffs(owner_bal) - 1;
+        const int f = __shfl_sync(kFull, best, owner);
+        if (lane == 0) {
+            const double s = fscore[f];
+            const int32_t d = fdep[f], p = fpar[f], rk = frank[f];
+            // remove f (move the last entry into its slot)
+            const int lastf = nf - 1;
+            fscore[f] = fscore[lastf];
+            fdep[f] = fdep[lastf];
+            fpar[f] = fpar[lastf];
+            frank[f] = frank[lastf];
+            int m = lastf;
+            const int idx = n;
+            nscore[idx] = s;
+            tok[idx] = cand_id[(d - 1) * K + rk];
+            par[idx] = p;
+            dep[idx] = d;
+            sco[idx] = (float)s;
+            if (d < B && ncand[d] > 0) {  // first child of the new node
+                fscore[m] = s * (double)cand_p[d * K + 0];
+                fdep[m] = d + 1;
+                fpar[m] = idx;
+                frank[m] = 0;
+                ++m;
+            }
+            if (rk + 1 < ncand[d - 1]) {  // next sibling
+                fscore[m] = nscore[p] * (double)cand_p[(d - 1) * K + rk + 1];
+                fdep[m] = d;
+                fpar[m] = p;
+                frank[m] = rk + 1;
+                ++m;
+            }
+            nf = m;
+        }
+        nf = __shfl_sync(kFull, nf, 0);
+        ++n;
+        __syncwarp();
+    }
+    if (lane == 0) J.num_nodes[r] = n;
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+static int sm_count() {
+    static int cached[64];
+    static std::once_flag flags[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::call_once(flags[dev], [dev]() {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    });
+    return cached[dev];
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Largest split count the workspace is sized for.
+static int split_bound(int64_t rows) {
+    if (rows <= 0) return 1;
+    int64_t s = 4096 / rows;
+    if (s < 1) s = 1;
+    if (s > kMaxSplits) s = kMaxSplits;
+    return (int)s;
+}
+
+// Workspace layout.  The first kCounterBytes hold the library's arrival
+// counters: row counters (split rows) in the first half, request counters in
+// the second.  Every call leaves them at zero, and nothing else is ever
+// written there, so one zero-fill serves every later call of any entry point
+// and size.  Scratch (partial selections, compact target rows) follows.
+constexpr int64_t kCounterWords = UNO_WORKSPACE_COUNTER_BYTES / 4;
+constexpr int64_t kRowCounterWords = kCounterWords / 2;
+
+struct WsLayout {
+    size_t row_ticket, req_ticket, part_keys, part_count, part_flags, c_ids, c_probs, c_count, c_flags, total;
+};
+
+static WsLayout ws_layout(int64_t rows, int32_t k, bool compact) {
+    WsLayout L{};
+    const int sb = split_bound(rows);
+    const size_t nslot = sb > 1 ? (size_t)rows * sb : 0;
+    L.row_ticket = 0;
+    L.req_ticket = (size_t)kRowCounterWords * 4;
+    size_t off = (size_t)UNO_WORKSPACE_COUNTER_BYTES;
+    L.part_keys = off;
+    off = align_up(off + nslot * (size_t)k * 8, 256);
+    L.part_count = off;
+    off = align_up(off + nslot * 4, 256);
+    L.part_flags = off;
+    off = align_up(off + nslot * 4, 256);
+    L.c_ids = off;
+    const size_t crow = compact ? (size_t)rows : 0;
+    off = align_up(off + crow * (size_t)k * 4, 256);
+    L.c_probs = off;
+    off = align_up(off + crow * (size_t)k * 4, 256);
+    L.c_count = off;
+    off = align_up(off + crow * 4, 256);
+    L.c_flags = off;
+    off = align_up(off + crow * 4, 256);
+    L.total = off;
+    return L;
+}
+
+static bool params_ok(const uno_sampling_params& sp) {
+    if (!(sp.temperature >= 0.0f) || std::isinf(sp.temperature)) return false;
+    if (sp.top_k < 1) return false;
+    if (!(sp.top_p > 0.0f && sp.top_p <= 1.0f)) return false;
+    return true;
+}
+
+// Shared memory of the streaming phase; the finishing area reuses the ring
+// stages when it fits there, else it is appended (fin_off).
+template <typename T, int MODE>
+static size_t row_smem_bytes(RowJob& J) {
+    const size_t stream = (size_t)kStages * kStageBytes + 32 + (size_t)kWarps * J.cap_w * 8;
+    const size_t finish = (size_t)J.merge_cap * 8 + (size_t)J.k * 32;
+    if (finish <= (size_t)kStages * kStageBytes) {
+        J.fin_off = 0;
+        return stream;
+    }
+    J.fin_off = (int32_t)((stream + 127) / 128 * 128);
+    return (size_t)J.fin_off + finish;
+}
+
+template <typename T, int MODE>
+static uno_status launch_rows(RowJob J, cudaStream_t stream) {
+    // warp buffer: high-water mark, plus room for one piece of appends from
+    // every lane; it also holds the threshold seed (2 keys per thread)
+    J.hw = J.k + 16 > 64 ? J.k + 16 : 64;
+    J.cap_w = J.hw + 32 * kPiece;
+    // split count: fill the GPU when rows are few (each split streams at
+    // least two stages)
+    const int64_t nunit_row = J.vocab / Elem<T>::kPerUnit;
+    const int64_t slots = (int64_t)sm_count() * 4;
+    int S = 1;
+    if (J.rows < slots && J.rows <= kRowCounterWords) {
+        int64_t s = slots / J.rows;
+        const int64_t by_work = nunit_row / (2 * kStageUnits);
+        if (s > by_work) s = by_work;
+        if (s > split_bound(J.rows)) s = split_bound(J.rows);
+        S = s < 1 ? 1 : (int)s;
+    }
+    // fewer splits if the merge area would not fit in shared memory
+    size_t smem = 0;
+    for (;;) {
+        J.S = S;
+        J.merge_cap = (S > kWarps ? S : kWarps) * J.k;
+        smem = row_smem_bytes<T, MODE>(J);
+        if (smem <= 227 * 1024 || S <= kWarps) break;
+        --S;
+    }
+    if (smem > 227 * 1024) return UNO_ERR_UNSUPPORTED;
+    auto kern = row_kernel<T, MODE>;
+    if (smem > 48 * 1024) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return UNO_ERR_CUDA;
+    }
+    const int64_t grid = J.rows * S;
+    if (grid <= 0) return UNO_OK;
+    if (grid > INT_MAX) return UNO_ERR_UNSUPPORTED;
+    kern<<<(unsigned)grid, kThreads, smem, stream>>>(J);
+    return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
+}
+
+static void bind_workspace(RowJob& J, void* ws, const WsLayout& L) {
+    unsigned char* b = static_cast<unsigned char*>(ws);
+    J.row_ticket = reinterpret_cast<uint32_t*>(b + L.row_ticket);
+    J.req_ticket = reinterpret_cast<uint32_t*>(b + L.req_ticket);
+    J.part_keys = reinterpret_cast<uint64_t*>(b + L.part_keys);
+    J.part_count = reinterpret_cast<int32_t*>(b + L.part_count);
+    J.part_flags = reinterpret_cast<uint32_t*>(b + L.part_flags);
+    J.c_ids = reinterpret_cast<int32_t*>(b + L.c_ids);
+    J.c_probs = reinterpret_cast<float*>(b + L.c_probs);
+    J.c_count = reinterpret_cast<int32_t*>(b + L.c_count);
+    J.c_flags = reinterpret_cast<uint32_t*>(b + L.c_flags);
+}
+
+}  // namespace uno
+
+using namespace uno;
+
+extern "C" {
+
+const char* uno_status_string(uno_status s) {
+    switch (s) {
+        case UNO_OK: return "ok";
+        case UNO_ERR_INVALID_ARG: return "invalid argument";
+        case UNO_ERR_UNSUPPORTED: return "unsupported argument";
+        case UNO_ERR_CUDA: return "CUDA launch error";
+        case UNO_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+size_t uno_filter_softmax_workspace_bytes(int64_t rows, int64_t vocab, int32_t top_k) {
+    if (rows <= 0 || vocab <= 0 || top_k < 1) return 0;
+    const int32_t k = (int32_t)(top_k < vocab ? top_k : vocab);
+    return ws_layout(rows, k, false).total;
+}
+
+size_t uno_linear_verify_workspace_bytes(int32_t R, int32_t B, int64_t vocab, int32_t top_k) {
+    if (R <= 0 || B <= 0 || vocab <= 0 || top_k < 1) return 0;
+    const int32_t k = (int32_t)(top_k < vocab ? top_k : vocab);
+    return ws_layout((int64_t)R * (B + 1), k, true).total;
+}
+
+size_t uno_tree_verify_workspace_bytes(int32_t R, int32_t V, int64_t vocab, int32_t top_k) {
+    if (R <= 0 || V <= 0 || vocab <= 0 || top_k < 1) return 0;
+    const int32_t k = (int32_t)(top_k < vocab ? top_k : vocab);
+    return ws_layout((int64_t)R * V, k, true).total;
+}
+
+static bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+uno_status uno_filter_softmax(const void* logits, uno_dtype dt, int64_t rows, int64_t vocab, int64_t row_stride,
+                              int32_t rows_per_request, uno_sampling_params sp, int32_t cap, int32_t* out_ids,
+                              float* out_probs, int32_t* out_count, float* out_dense, const uno_rng* rng,
+                              int32_t* out_sample, uint32_t* out_flags, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    if (!logits || !out_ids || !out_probs || !out_count || !out_flags) return UNO_ERR_INVALID_ARG;
+    if (rows <= 0 || vocab <= 0 || vocab > INT32_MAX || row_stride < vocab || rows_per_request < 1)
+        return UNO_ERR_INVALID_ARG;
+    if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
+    if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    if (rng && !out_sample) return UNO_ERR_INVALID_ARG;
+    if (!aligned_to(logits, dt == UNO_F32 ? 4 : 2)) return UNO_ERR_INVALID_ARG;
+    if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
+    const int32_t k = (int32_t)(sp.top_k < vocab ? sp.top_k : vocab);
+    if (cap < k) return UNO_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(rows, k, false);
+    if (!workspace || workspace_bytes < L.total || !aligned_to(workspace, 16)) return UNO_ERR_WORKSPACE;
+
+    RowJob J{};
+    J.logits = static_cast<const unsigned char*>(logits);
+    J.rows = rows;
+    J.vocab = vocab;
+    J.row_stride = row_stride;
+    J.rpr = rows_per_request;
+    J.temperature = sp.temperature;
+    J.top_p = sp.top_p;
+    J.k = k;
+    J.out_ids = out_ids;
+    J.out_probs = out_probs;
+    J.out_count = out_count;
+    J.cap = cap;
+    J.out_dense = out_dense;
+    J.out_sample = out_sample;
+    J.out_flags = out_flags;
+    J.has_rng = rng ? 1 : 0;
+    J.seed = rng ? rng->seed : 0;
+    J.cycle = rng ? rng->cycle : 0;
+    J.first_request = rng ? rng->first_request : 0;
+    bind_workspace(J, workspace, L);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeFilter>(J, s) : launch_rows<float, kModeFilter>(J, s);
+}
+
+uno_status uno_linear_verify(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int64_t vocab,
+                             uno_sampling_params sp, const int32_t* draft_ids, const int32_t* q_ids,
+                             const float* q_probs, const int32_t* q_count, int32_t q_cap, uno_rng rng,
+                             int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                             uint32_t* out_flags, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!target_logits || !draft_ids || !q_ids || !q_probs || !q_count || !out_tokens || !out_accept_len ||
+        !out_num_tokens || !out_flags)
+        return UNO_ERR_INVALID_ARG;
+    if (R <= 0 || B <= 0 || vocab <= 0 || vocab > INT32_MAX || q_cap < 1) return UNO_ERR_INVALID_ARG;
+    if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
+    if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    if (!aligned_to(target_logits, dt == UNO_F32 ? 4 : 2)) return UNO_ERR_INVALID_ARG;
+    if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
+    const int32_t k = (int32_t)(sp.top_k < vocab ? sp.top_k : vocab);
+    const int64_t rows = (int64_t)R * (B + 1);
+    if ((int64_t)R > kCounterWords - kRowCounterWords) return UNO_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(rows, k, true);
+    if (!workspace || workspace_bytes < L.total || !aligned_to(workspace, 16)) return UNO_ERR_WORKSPACE;
+
+    RowJob J{};
+    J.logits = static_cast<const unsigned char*>(target_logits);
+    J.rows = rows;
+    J.vocab = vocab;
+    J.row_stride = vocab;
+    J.rpr = B + 1;
+    J.temperature = sp.temperature;
+    J.top_p = sp.top_p;
+    J.k = k;
+    J.seed = rng.seed;
+    J.cycle = rng.cycle;
+    J.first_request = rng.first_request;
+    J.B = B;
+    J.draft_ids = draft_ids;
+    J.q_ids = q_ids;
+    J.q_probs = q_probs;
+    J.q_count = q_count;
+    J.q_cap = q_cap;
+    J.out_tokens = out_tokens;
+    J.out_accept_len = out_accept_len;
+    J.out_num_tokens = out_num_tokens;
+    J.out_req_flags = out_flags;
+    bind_workspace(J, workspace, L);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeLinear>(J, s) : launch_rows<float, kModeLinear>(J, s);
+}
+
+uno_status uno_tree_topk_expand(const int32_t* q_ids, const float* q_probs, const int32_t* q_count, int32_t q_cap,
+                                int32_t R, int32_t B, int32_t K, int32_t V, int32_t* node_token,
+                                int32_t* node_parent, int32_t* node_depth, float* node_score, int32_t* num_nodes,
+                                void* stream) {
+    if (!q_ids || !q_probs || !q_count || !node_token || !node_parent || !node_depth || !node_score || !num_nodes)
+        return UNO_ERR_INVALID_ARG;
+    if (R <= 0 || B <= 0 || K <= 0 || V <= 0 || q_cap < 1) return UNO_ERR_INVALID_ARG;
+    if (V < B || V > UNO_MAX_TREE_NODES || (int64_t)V * K > UNO_MAX_TREE_FRONTIER) return UNO_ERR_INVALID_ARG;
+    if (q_cap > 4096) return UNO_ERR_UNSUPPORTED;
+    TreeJob J{};
+    J.q_ids = q_ids;
+    J.q_probs = q_probs;
+    J.q_count = q_count;
+    J.q_cap = q_cap;
+    J.R = R;
+    J.B = B;
+    J.K = K;
+    J.V = V;
+    J.sort_cap = next_pow2(q_cap);
+    J.node_token = node_token;
+    J.node_parent = node_parent;
+    J.node_depth = node_depth;
+    J.node_score = node_score;
+    J.num_nodes = num_nodes;
+    const size_t smem = (size_t)J.sort_cap * 8 + (size_t)(2 * V + 1) * 8 + (size_t)B * K * 8 + (size_t)B * 4 +
+                        (size_t)3 * (V + 1) * 4;
+    if (smem > 227 * 1024) return UNO_ERR_UNSUPPORTED;
+    if (smem > 48 * 1024) {
+        if (cudaFuncSetAttribute(tree_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return UNO_ERR_CUDA;
+    }
+    tree_expand_kernel<<<(unsigned)R, 32, smem, static_cast<cudaStream_t>(stream)>>>(J);
+    return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
+}
+
+uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int32_t V, int64_t vocab,
+                           uno_sampling_params sp, const int32_t* node_token, const int32_t* node_parent,
+                           const int32_t* num_nodes, uno_rng rng, int32_t* out_tokens, int32_t* out_accept_len,
+                           int32_t* out_num_tokens, int32_t* out_path_nodes, uint32_t* out_flags, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    if (!target_logits || !node_token || !node_parent || !num_nodes || !out_tokens || !out_accept_len ||
+        !out_num_tokens || !out_path_nodes || !out_flags)
+        return UNO_ERR_INVALID_ARG;
+    if (R <= 0 || B <= 0 || V <= 0 || vocab <= 0 || vocab > INT32_MAX) return UNO_ERR_INVALID_ARG;
+    if (V < B || V > UNO_MAX_TREE_NODES) return UNO_ERR_INVALID_ARG;
+    if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
+    if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    if (!aligned_to(target_logits, dt == UNO_F32 ? 4 : 2)) return UNO_ERR_INVALID_ARG;
+    if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
+    const int32_t k = (int32_t)(sp.top_k < vocab ? sp.top_k : vocab);
+    const int64_t rows = (int64_t)R * V;
+    if ((int64_t)R > kCounterWords - kRowCounterWords) return UNO_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(rows, k, true);
+    if (!workspace || workspace_bytes < L.total || !aligned_to(workspace, 16)) return UNO_ERR_WORKSPACE;
+
+    RowJob J{};
+    J.logits = static_cast<const unsigned char*>(target_logits);
+    J.rows = rows;
+    J.vocab = vocab;
+    J.row_stride = vocab;
+    J.rpr = V;
+    J.temperature = sp.temperature;
+    J.top_p = sp.top_p;
+    J.k = k;
+    J.seed = rng.seed;
+    J.cycle = rng.cycle;
+    J.first_request = rng.first_request;
+    J.B = B;
+    J.V = V;
+    J.node_token = node_token;
+    J.node_parent = node_parent;
+    J.num_nodes = num_nodes;
+    J.out_tokens = out_tokens;
+    J.out_accept_len = out_accept_len;
+    J.out_num_tokens = out_num_tokens;
+    J.out_path_nodes = out_path_nodes;
+    J.out_req_flags = out_flags;
+    bind_workspace(J, workspace, L);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeTree>(J, s) : launch_rows<float, kModeTree>(J, s);
+}
+
+}  // extern "C"

@@ -42,8 +42,8 @@ MUTATIONS = {
     "bonus from wrong row": ("for (int j = 0; j < p_cnt[B]; ++j) wts[j] = (double)p_probs[(size_t)B * (size_t)cap + (size_t)j];",
                              "for (int j = 0; j < p_cnt[B]; ++j) wts[j] = (double)p_probs[(size_t)(B - 1) * (size_t)cap + (size_t)j];",
                              lambda: tl.test_linear_output_is_the_target_process(4, 2, 1.0, 4, 1.0, 11)),
-    "accept and residual share a draw": ("double u = uno_ref_uniform(seed, (uint32_t)r, (uint32_t)i, DRAW_RESIDUAL, cycle);",
-                                         "double u = uno_ref_uniform(seed, (uint32_t)r, (uint32_t)i, DRAW_ACCEPT, cycle);",
+    "accept and residual share a draw": ("uno_ref_uniform(seed, first_request + (uint32_t)r, (uint32_t)i, DRAW_RESIDUAL, cycle);",
+                                         "uno_ref_uniform(seed, first_request + (uint32_t)r, (uint32_t)i, DRAW_ACCEPT, cycle);",
                                          lambda: tl.test_linear_output_is_the_target_process(4, 2, 1.0, 4, 1.0, 11)),
     "tree tie by deeper first": ("if (a->depth != b->depth) return a->depth < b->depth;",
                                  "if (a->depth != b->depth) return a->depth > b->depth;",
