@@ -211,6 +211,34 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
                            int32_t* out_num_tokens, int32_t* out_path_nodes, uint32_t* out_flags, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * uno_linear_verify_noalloc -- uno_linear_verify without a caller workspace.
+ * This entry point has no counterpart on the method's pages: it only changes
+ * where the scratch memory comes from.  It is for callers that cannot
+ * allocate device memory for the library -- a serving loop that has given all
+ * free memory to its KV-cache pool, or a host that loads this library as a
+ * plugin and offers it no allocator.  Its scratch is a library-owned device
+ * array of UNO_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU which loads the
+ * library holds until the process exits.
+ *
+ * Arguments, results and errors are those of uno_linear_verify, minus the
+ * workspace.  Sizes whose uno_linear_verify_workspace_bytes exceeds
+ * UNO_NOALLOC_SCRATCH_BYTES return UNO_ERR_UNSUPPORTED before anything is
+ * enqueued: the 8 MiB hold R*(B+1) * min(top_k, vocab) up to about 880,000
+ * (512 requests with B = 16 at top_k 50 fit; at top_k 200 they do not).  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  The call itself allocates nothing: it enqueues
+ * cudaMemsetAsync of the counters it uses, then the kernel.  Every call
+ * shares the one array, so calls that overlap on the GPU (other streams,
+ * other host threads) race; serialise them.
+ * ---------------------------------------------------------------------- */
+#define UNO_NOALLOC_SCRATCH_BYTES (8u << 20)
+uno_status uno_linear_verify_noalloc(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int64_t vocab,
+                                     uno_sampling_params sp, const int32_t* draft_ids, const int32_t* q_ids,
+                                     const float* q_probs, const int32_t* q_count, int32_t q_cap, uno_rng rng,
+                                     int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                                     uint32_t* out_flags, void* stream);
+
 /* Text of a status code (static storage). */
 const char* uno_status_string(uno_status s);
 

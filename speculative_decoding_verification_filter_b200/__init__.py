@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     load_library,
     uno_filter_softmax,
     uno_linear_verify,
+    uno_linear_verify_noalloc,
     uno_tree_topk_expand,
     uno_tree_verify,
 )

@@ -29,6 +29,7 @@ EXPORTED = (
     "uno_linear_verify_workspace_bytes", "uno_linear_verify",
     "uno_tree_topk_expand",
     "uno_tree_verify_workspace_bytes", "uno_tree_verify",
+    "uno_linear_verify_noalloc",
     "uno_status_string",
 )
 
@@ -86,6 +87,9 @@ def load_library():
         lib.uno_tree_verify.argtypes = [P, ctypes.c_int, i32, i32, i32, i64, _Params, P, P, P, _Rng,
                                         P, P, P, P, P, P, sz, P]
         lib.uno_tree_verify.restype = ctypes.c_int
+        lib.uno_linear_verify_noalloc.argtypes = [P, ctypes.c_int, i32, i32, i64, _Params, P, P, P, P, i32, _Rng,
+                                                  P, P, P, P, P]
+        lib.uno_linear_verify_noalloc.restype = ctypes.c_int
         lib.uno_status_string.argtypes = [ctypes.c_int]
         lib.uno_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -279,3 +283,35 @@ def uno_tree_verify(target_logits, node_token, node_parent, num_nodes, *, R, B, 
                              _ptr(flags), _ptr(ws), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
     _check("uno_tree_verify", st)
     return _host_back(dict(tokens=toks, accept_len=acc, num_tokens=ntok, path_nodes=path, flags=flags), host)
+
+
+def uno_linear_verify_noalloc(target_logits, draft_ids, q_ids, q_probs, q_count, *, R, B, temperature, top_k,
+                              top_p, rng):
+    """uno_linear_verify for callers that cannot give the library a workspace
+    (for instance a serving loop whose free device memory all belongs to its
+    KV-cache pool): the scratch is a fixed 8 MiB device array owned by the
+    library.  Same arguments and results as uno_linear_verify; only the output
+    tensors are allocated here, by PyTorch, as for every entry point."""
+    lib = load_library()
+    host = not target_logits.is_cuda
+    device = _device_of(target_logits, draft_ids, q_ids)
+    x = _dev(target_logits, device).contiguous()
+    vocab = x.shape[-1]
+    if x.numel() != R * (B + 1) * vocab:
+        raise ValueError("target_logits must hold R*(B+1) rows")
+    d = _dev(draft_ids, device).to(torch.int32).contiguous()
+    qi = _dev(q_ids, device).to(torch.int32).contiguous()
+    qp = _dev(q_probs, device).to(torch.float32).contiguous()
+    qc = _dev(q_count, device).to(torch.int32).contiguous()
+    stream = torch.cuda.current_stream(device)
+    kw = dict(dtype=torch.int32, device=device)
+    toks = torch.empty((R, B + 1), **kw)
+    acc = torch.empty(R, **kw)
+    ntok = torch.empty(R, **kw)
+    flags = torch.empty(R, **kw)
+    st = lib.uno_linear_verify_noalloc(_ptr(x), _dtype_code(x), R, B, vocab,
+                                       _Params(float(temperature), int(top_k), float(top_p)), _ptr(d), _ptr(qi),
+                                       _ptr(qp), _ptr(qc), qi.shape[1], _rng(rng), _ptr(toks), _ptr(acc), _ptr(ntok),
+                                       _ptr(flags), ctypes.c_void_p(stream.cuda_stream))
+    _check("uno_linear_verify_noalloc", st)
+    return _host_back(dict(tokens=toks, accept_len=acc, num_tokens=ntok, flags=flags), host)

@@ -1806,4 +1806,87 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
     return dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeTree>(J, s) : launch_rows<float, kModeTree>(J, s);
 }
 
+// ---------------------------------------------------------------------------
+// uno_linear_verify_noalloc: uno_linear_verify with library-owned scratch.
+//
+// Some callers cannot hand the library a workspace: a serving loop that has
+// already given all free device memory to its KV-cache pool, or a host
+// program that loads this library as a plugin and offers it no allocator.
+// For them the scratch lives in a file-scope device array that every GPU
+// which loads the library holds until the process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[UNO_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name is only a stand-in, so the address is looked up once per
+// device, with that device current, on the first call there.
+static uno_status noalloc_scratch(unsigned char** out) {
+    static std::mutex mu;
+    static unsigned char* addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return UNO_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return UNO_ERR_CUDA;
+        addr[dev] = static_cast<unsigned char*>(p);
+    }
+    *out = addr[dev];
+    return UNO_OK;
+}
+
+uno_status uno_linear_verify_noalloc(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int64_t vocab,
+                                     uno_sampling_params sp, const int32_t* draft_ids, const int32_t* q_ids,
+                                     const float* q_probs, const int32_t* q_count, int32_t q_cap, uno_rng rng,
+                                     int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                                     uint32_t* out_flags, void* stream) {
+    if (!target_logits || !draft_ids || !q_ids || !q_probs || !q_count || !out_tokens || !out_accept_len ||
+        !out_num_tokens || !out_flags)
+        return UNO_ERR_INVALID_ARG;
+    if (R <= 0 || B <= 0 || vocab <= 0 || vocab > INT32_MAX || q_cap < 1) return UNO_ERR_INVALID_ARG;
+    if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
+    if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    if (!aligned_to(target_logits, dt == UNO_F32 ? 4 : 2)) return UNO_ERR_INVALID_ARG;
+    if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
+    if ((int64_t)R > kCounterWords - kRowCounterWords) return UNO_ERR_UNSUPPORTED;
+    const int32_t k = (int32_t)(sp.top_k < vocab ? sp.top_k : vocab);
+    const int64_t rows = (int64_t)R * (B + 1);
+    const WsLayout L = ws_layout(rows, k, true);
+    if (L.total > (size_t)UNO_NOALLOC_SCRATCH_BYTES) return UNO_ERR_UNSUPPORTED;  // beyond the fixed scratch
+    unsigned char* scratch = nullptr;
+    const uno_status st = noalloc_scratch(&scratch);
+    if (st != UNO_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the array keeps the last call's contents: clear the counters this call
+    // uses (row counters only matter for split rows, which need rows < 4096)
+    if (cudaMemsetAsync(scratch + L.req_ticket, 0, (size_t)R * 4, s) != cudaSuccess) return UNO_ERR_CUDA;
+    if (rows < 4096 && cudaMemsetAsync(scratch + L.row_ticket, 0, (size_t)rows * 4, s) != cudaSuccess)
+        return UNO_ERR_CUDA;
+
+    RowJob J{};
+    J.logits = static_cast<const unsigned char*>(target_logits);
+    J.rows = rows;
+    J.vocab = vocab;
+    J.row_stride = vocab;
+    J.rpr = B + 1;
+    J.temperature = sp.temperature;
+    J.top_p = sp.top_p;
+    J.k = k;
+    J.seed = rng.seed;
+    J.cycle = rng.cycle;
+    J.first_request = rng.first_request;
+    J.B = B;
+    J.draft_ids = draft_ids;
+    J.q_ids = q_ids;
+    J.q_probs = q_probs;
+    J.q_count = q_count;
+    J.q_cap = q_cap;
+    J.out_tokens = out_tokens;
+    J.out_accept_len = out_accept_len;
+    J.out_num_tokens = out_num_tokens;
+    J.out_req_flags = out_flags;
+    bind_workspace(J, scratch, L);
+    return dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeLinear>(J, s) : launch_rows<float, kModeLinear>(J, s);
+}
+
 }  // extern "C"
