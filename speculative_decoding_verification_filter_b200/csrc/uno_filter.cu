@@ -46,6 +46,7 @@ struct RowJob {
     int32_t hw, cap_w;                // warp buffer high-water mark / capacity
     int32_t merge_cap;                // entries of the merge area
     int32_t fin_off;                  // shared-memory offset of the finishing area (0: the ring)
+    int32_t tail_off, tail_bytes;     // shared-memory scratch of the request tails
     // filter outputs
     int32_t* out_ids;
     float* out_probs;
@@ -784,35 +785,6 @@ __device__ __noinline__ void tree_tail(const RowJob& J, int32_t r, double* wd, i
     }
 }
 
-
-// ---------------------------------------------------------------------------
-// Finishing a row (all threads of the CTA).
-// ---------------------------------------------------------------------------
-struct FinishShared {
-    double S, W;
-    int kept, last, n;
-};
-
-// Exact top k of the unique keys uni[0..U): each key's rank is the number of
-// larger keys; ranks below k land in sel[rank], so sel comes out sorted
-// (descending).  All threads call it.
-__device__ __forceinline__ void cta_rank_topk(const uint64_t* uni, int U, int k, uint64_t* sel) {
-    for (int i = threadIdx.x; i < U; i += kThreads) {
-        const uint64_t key = uni[i];
-        int rank = 0;
-        int j = 0;
-        for (; j + 8 <= U; j += 8) {  // independent loads ahead of the compares
-            ulonglong2 p[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) p[q] = *reinterpret_cast<const ulonglong2*>(uni + j + 2 * q);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) rank += (p[q].x > key) + (p[q].y > key);
-        }
-        for (; j < U; ++j) rank += (uni[j] > key);
-        if (rank < k) sel[rank] = key;
-    }
-}
-
 // ---------------------------------------------------------------------------
 // Warp-level finishing for k <= 64: lane l holds ranks l and l + 32.  Sums
 // and scans run as warp reductions (a fixed order; it differs from a serial
@@ -872,9 +844,296 @@ __device__ __forceinline__ int warp_inv_cdf(double wa, double wb, double u, int 
     return -1;
 }
 
+// ---------------------------------------------------------------------------
+// Request tails from shared memory (k <= 64): the last CTA of a request first
+// copies the request's compact rows into its idle ring buffer with all
+// lanes, then runs the sequential decisions with warp-parallel lookups and
+// inverse-CDF draws.  They return false (and the callers fall back to the
+// tails above) when the rows do not fit.
+// ---------------------------------------------------------------------------
+
+// Probability of token x in a compact row held in shared memory (0 if absent).
+__device__ __forceinline__ double warp_lookup(const int32_t* ids, const float* pr, int n, int32_t x, int lane) {
+    float v = 0.0f;
+    bool hit = false;
+    for (int j = lane; j < n; j += 32)
+        if (ids[j] == x) {
+            v = pr[j];
+            hit = true;
+        }
+    const unsigned bal = __ballot_sync(kFull, hit);
+    if (!bal) return 0.0;
+    return (double)__shfl_sync(kFull, v, __ffs(bal) - 1);
+}
+
+// Probability of token x in a compact row with ascending ids (one lane,
+// binary search in shared memory).
+__device__ __forceinline__ double smem_lookup(const int32_t* ids, const float* pr, int n, int32_t x) {
+    int lo = 0, hi = n - 1;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        const int32_t m = ids[mid];
+        if (m == x) return (double)pr[mid];
+        if (m < x)
+            lo = mid + 1;
+        else
+            hi = mid - 1;
+    }
+    return 0.0;
+}
+
+__device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsigned char* sm, int lane) {
+    const int32_t B = J.B;
+    const int kc = J.k;
+    constexpr int QS = 64;  // q entries kept per row
+    if (kc > 64) return false;
+    const size_t need = (size_t)(B + 1) * kc * 8 + (size_t)B * QS * 8 + (size_t)(4 * B + 2) * 4;
+    if (need > (size_t)J.tail_bytes) return false;
+    int32_t* pid = reinterpret_cast<int32_t*>(sm);           // [B+1][kc]
+    float* ppr = reinterpret_cast<float*>(pid + (B + 1) * kc);  // [B+1][kc]
+    int32_t* qid = reinterpret_cast<int32_t*>(ppr + (B + 1) * kc);  // [B][QS]
+    float* qpr = reinterpret_cast<float*>(qid + B * QS);        // [B][QS]
+    int32_t* pcnt = reinterpret_cast<int32_t*>(qpr + B * QS);  // [B+1]
+    int32_t* qcnt = pcnt + (B + 1);                             // [B]
+    int32_t* dft = qcnt + B;                                    // [B]
+    int32_t* otok = dft + B;                                    // [B+1] emitted tokens
+    const int64_t base = (int64_t)r * (B + 1);
+    uint32_t flags = 0;
+    bool qbig = false;
+    for (int i = lane; i <= B; i += 32) {
+        pcnt[i] = __ldcg(J.c_count + base + i);
+        flags |= __ldcg(J.c_flags + base + i);
+    }
+    for (int i = lane; i < B; i += 32) {
+        int qc = J.q_count[(int64_t)r * B + i];
+        qc = qc < 0 ? 0 : (qc > J.q_cap ? J.q_cap : qc);
+        qbig |= qc > QS;
+        qcnt[i] = qc;
+        dft[i] = J.draft_ids[(size_t)r * B + i];
+    }
+    for (int i = lane; i <= B; i += 32) otok[i] = -1;
+    flags = __reduce_or_sync(kFull, flags);
+    if (__any_sync(kFull, qbig)) return false;
+    __syncwarp();
+    for (int i = 0; i <= B; ++i) {
+        const int c = pcnt[i];
+        for (int j = lane; j < c; j += 32) {
+            pid[i * kc + j] = __ldcg(J.c_ids + (size_t)(base + i) * kc + j);
+            ppr[i * kc + j] = __ldcg(J.c_probs + (size_t)(base + i) * kc + j);
+        }
+    }
+    for (int i = 0; i < B; ++i) {
+        const int c = qcnt[i];
+        const int64_t qrow = (int64_t)r * B + i;
+        for (int j = lane; j < c; j += 32) {
+            qid[i * QS + j] = J.q_ids[(size_t)qrow * J.q_cap + j];
+            qpr[i * QS + j] = J.q_probs[(size_t)qrow * J.q_cap + j];
+        }
+    }
+    __syncwarp();
+
+    int32_t* toks = J.out_tokens + (size_t)r * (B + 1);
+    int32_t acc = B, ntok = B + 1;
+    bool stopped = false;
+    const uint32_t req = J.first_request + (uint32_t)r;
+    for (int i = 0; i < B && !stopped; ++i) {
+        const int pc = pcnt[i];
+        if (pc == 0) {  // a non-finite target row was reached
+            acc = i;
+            ntok = i;
+            stopped = true;
+            break;
+        }
+        const int32_t* pi = pid + i * kc;
+        const float* pp = ppr + i * kc;
+        const int32_t* qi = qid + i * QS;
+        const float* qp = qpr + i * QS;
+        const int32_t x = dft[i];
+        const bool xin = x >= 0 && (int64_t)x < J.vocab;
+        const double a = xin ? warp_lookup(qi, qp, qcnt[i], x, lane) : 0.0;
+        const double px = xin ? warp_lookup(pi, pp, pc, x, lane) : 0.0;
+        bool accept = false;
+        if (a > 0.0) {
+            const double u = uniform53(J.seed, req, (uint32_t)i, kDrawAccept, J.cycle);
+            accept = (u * a < px);
+        } else {
+            flags |= kFlagDraftNotInSupport;
+        }
+        if (accept) {
+            if (lane == 0) otok[i] = x;
+            continue;
+        }
+        // residual max(0, p_i - q_i) over supp p_i, ascending ids
+        double ra = 0.0, rb = 0.0, pa = 0.0, pb = 0.0;
+        if (lane < pc) {
+            pa = (double)pp[lane];
+            const double d = pa - smem_lookup(qi, qp, qcnt[i], pi[lane]);
+            ra = d > 0.0 ? d : 0.0;
+        }
+        if (lane + 32 < pc) {
+            pb = (double)pp[lane + 32];
+            const double d = pb - smem_lookup(qi, qp, qcnt[i], pi[lane + 32]);
+            rb = d > 0.0 ? d : 0.0;
+        }
+        const double u = uniform53(J.seed, req, (uint32_t)i, kDrawResidual, J.cycle);
+        int pick = warp_inv_cdf(ra, rb, u, lane);
+        if (pick < 0) {  // the residual is empty: draw from p_i
+            flags |= kFlagResidualEmpty;
+            pick = warp_inv_cdf(pa, pb, u, lane);
+        }
+        if (lane == 0) otok[i] = pick >= 0 ? pi[pick] : -1;
+        acc = i;
+        ntok = i + 1;
+        stopped = true;
+    }
+    if (!stopped) {
+        const int pc = pcnt[B];
+        if (pc == 0) {
+            ntok = B;
+        } else {
+            const float* pp = ppr + B * kc;
+            const double wa = lane < pc ? (double)pp[lane] : 0.0, wb = lane + 32 < pc ? (double)pp[lane + 32] : 0.0;
+            const double u = uniform53(J.seed, req, (uint32_t)B, kDrawTarget, J.cycle);
+            const int pick = warp_inv_cdf(wa, wb, u, lane);
+            if (lane == 0) otok[B] = pick >= 0 ? pid[B * kc + pick] : -1;
+        }
+    }
+    __syncwarp();
+    for (int t = lane; t <= B; t += 32) toks[t] = otok[t];
+    if (lane == 0) {
+        J.out_accept_len[r] = acc;
+        J.out_num_tokens[r] = ntok;
+        J.out_req_flags[r] = flags;
+    }
+    return true;
+}
+
+__device__ __noinline__ bool tree_tail_fast(const RowJob& J, int32_t r, unsigned char* sm, int lane) {
+    const int32_t B = J.B, V = J.V;
+    const int kc = J.k;
+    if (kc > 64) return false;
+    int32_t n = J.num_nodes[r];
+    n = n < 1 ? 1 : (n > V ? V : n);
+    const size_t need = (size_t)n * kc * 8 + (size_t)n * 12 + (size_t)(B + 1) * 8;
+    if (need > (size_t)J.tail_bytes) return false;
+    int32_t* nid = reinterpret_cast<int32_t*>(sm);        // [n][kc]
+    float* npr = reinterpret_cast<float*>(nid + n * kc);  // [n][kc]
+    int32_t* ncnt = reinterpret_cast<int32_t*>(npr + n * kc);  // [n]
+    int32_t* tk = ncnt + n;                               // [n]
+    int32_t* pa = tk + n;                                 // [n]
+    int32_t* otok = pa + n;                               // [B+1] emitted tokens
+    int32_t* opath = otok + (B + 1);                      // [B+1] nodes that drew them
+    const int64_t base = (int64_t)r * V;
+    uint32_t flags = 0;
+    for (int j = lane; j < n; j += 32) {
+        ncnt[j] = __ldcg(J.c_count + base + j);
+        flags |= __ldcg(J.c_flags + base + j);
+        tk[j] = J.node_token[(size_t)r * V + j];
+        pa[j] = J.node_parent[(size_t)r * V + j];
+    }
+    for (int q = lane; q <= B; q += 32) {
+        otok[q] = -1;
+        opath[q] = -1;
+    }
+    flags = __reduce_or_sync(kFull, flags);
+    __syncwarp();
+    for (int j = 0; j < n; ++j) {
+        const int c = ncnt[j];
+        for (int e = lane; e < c; e += 32) {
+            nid[j * kc + e] = __ldcg(J.c_ids + (size_t)(base + j) * kc + e);
+            npr[j * kc + e] = __ldcg(J.c_probs + (size_t)(base + j) * kc + e);
+        }
+    }
+    __syncwarp();
+    int32_t* toks = J.out_tokens + (size_t)r * (B + 1);
+    int32_t* path = J.out_path_nodes + (size_t)r * (B + 1);
+    const uint32_t req = J.first_request + (uint32_t)r;
+    int32_t j = 0, t = 0, acc = 0, ntok = 0;
+    for (;;) {
+        const int pc = ncnt[j];
+        if (pc == 0) {
+            if (lane == 0) opath[t] = j;
+            ntok = t;
+            acc = t;
+            break;
+        }
+        const float* pp = npr + j * kc;
+        const double wa = lane < pc ? (double)pp[lane] : 0.0, wb = lane + 32 < pc ? (double)pp[lane + 32] : 0.0;
+        const double u = uniform53(J.seed, req, (uint32_t)j, kDrawTarget, J.cycle);
+        const int pick = warp_inv_cdf(wa, wb, u, lane);
+        const int32_t y = pick >= 0 ? nid[j * kc + pick] : -1;
+        if (lane == 0) {
+            otok[t] = y;
+            opath[t] = j;
+        }
+        ++t;
+        ntok = t;
+        acc = t - 1;
+        int32_t next = -1;  // the lowest-index child of j carrying y
+        for (int c0 = 1; c0 < n && next < 0; c0 += 32) {
+            const int c = c0 + lane;
+            const bool hit = c < n && pa[c] == j && tk[c] == y;
+            const unsigned bal = __ballot_sync(kFull, hit);
+            if (bal) next = c0 + __ffs(bal) - 1;
+        }
+        if (next < 0 || t > B) break;
+        j = next;
+    }
+    __syncwarp();
+    for (int q = lane; q <= B; q += 32) {
+        toks[q] = otok[q];
+        path[q] = opath[q];
+    }
+    if (lane == 0) {
+        J.out_accept_len[r] = acc;
+        J.out_num_tokens[r] = ntok;
+        J.out_req_flags[r] = flags;
+    }
+    return true;
+}
+
+template <int MODE>
+__device__ __forceinline__ void request_tail(const RowJob& J, int32_t req, double* wd, unsigned char* tail_smem,
+                                             int lane) {
+    if (MODE == kModeLinear) {
+        if (!linear_tail_fast(J, req, tail_smem, lane)) linear_tail(J, req, wd, lane);
+    } else {
+        if (!tree_tail_fast(J, req, tail_smem, lane)) tree_tail(J, req, wd, lane);
+    }
+}
+
+
+// ---------------------------------------------------------------------------
+// Finishing a row (all threads of the CTA).
+// ---------------------------------------------------------------------------
+struct FinishShared {
+    double S, W;
+    int kept, last, n;
+};
+
+// Exact top k of the unique keys uni[0..U): each key's rank is the number of
+// larger keys; ranks below k land in sel[rank], so sel comes out sorted
+// (descending).  All threads call it.
+__device__ __forceinline__ void cta_rank_topk(const uint64_t* uni, int U, int k, uint64_t* sel) {
+    for (int i = threadIdx.x; i < U; i += kThreads) {
+        const uint64_t key = uni[i];
+        int rank = 0;
+        int j = 0;
+        for (; j + 8 <= U; j += 8) {  // independent loads ahead of the compares
+            ulonglong2 p[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) p[q] = *reinterpret_cast<const ulonglong2*>(uni + j + 2 * q);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) rank += (p[q].x > key) + (p[q].y > key);
+        }
+        for (; j < U; ++j) rank += (uni[j] > key);
+        if (rank < k) sel[rank] = key;
+    }
+}
+
 template <int MODE>
 __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n, uint32_t rowbad,
-                                const uint64_t* sel, double* wd, FinishShared& fs, int lane) {
+                                const uint64_t* sel, double* wd, unsigned char* tail_smem, FinishShared& fs, int lane) {
     const bool bad = rowbad != 0u || n == 0;
     int kept = 0;
     uint64_t oa = ~0ull, ob = ~0ull;  // (id, prob) pairs, ascending id after the sort
@@ -982,12 +1241,7 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
             }
         }
         last = __shfl_sync(kFull, last, 0);
-        if (last) {
-            if (MODE == kModeLinear)
-                linear_tail(J, req, wd, lane);
-            else
-                tree_tail(J, req, wd, lane);
-        }
+        if (last) request_tail<MODE>(J, req, wd, tail_smem, lane);
     }
 }
 
@@ -995,7 +1249,8 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
 // the row (filter: output; verifiers: workspace + request tail).
 template <int MODE>
 __device__ void finish_row(const RowJob& J, int64_t row, int32_t req, int n, uint32_t rowbad, const uint64_t* sel,
-                           uint64_t* outk, double* wd, double* pd, FinishShared& fs, int warp, int lane) {
+                           uint64_t* outk, double* wd, double* pd, unsigned char* tail_smem, FinishShared& fs, int warp,
+                           int lane) {
     const int tid = threadIdx.x;
     const bool bad = rowbad != 0u || n == 0;
     int kept = 0;
@@ -1130,12 +1385,7 @@ __device__ void finish_row(const RowJob& J, int64_t row, int32_t req, int n, uin
             }
         }
         __syncthreads();
-        if (fs.last && warp == 0) {
-            if (MODE == kModeLinear)
-                linear_tail(J, req, wd, lane);
-            else
-                tree_tail(J, req, wd, lane);
-        }
+        if (fs.last && warp == 0) request_tail<MODE>(J, req, wd, tail_smem, lane);
     }
 }
 
@@ -1185,7 +1435,7 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const RowJob J) {
                 }
             }
             __syncthreads();
-            if (fs.last && warp == 0) tree_tail(J, req, wd, lane);
+            if (fs.last && warp == 0) request_tail<kModeTree>(J, req, wd, smem + J.tail_off, lane);
             return;
         }
     }
@@ -1294,9 +1544,9 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const RowJob J) {
     }
 
     if (J.k <= 64) {
-        if (warp == 0) finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, fs, lane);
+        if (warp == 0) finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, smem + J.tail_off, fs, lane);
     } else {
-        finish_row<MODE>(J, row, req, n, rowbad, sel, outk, wd, pd, fs, warp, lane);
+        finish_row<MODE>(J, row, req, n, rowbad, sel, outk, wd, pd, smem + J.tail_off, fs, warp, lane);
     }
 }
 
@@ -1536,11 +1786,17 @@ template <typename T, int MODE>
 static size_t row_smem_bytes(RowJob& J) {
     const size_t stream = (size_t)kStages * kStageBytes + 32 + (size_t)kWarps * J.cap_w * 8;
     const size_t finish = (size_t)J.merge_cap * 8 + (size_t)J.k * 32;
-    if (finish <= (size_t)kStages * kStageBytes) {
+    const size_t ring = (size_t)kStages * kStageBytes;
+    // the request tails use the rest of the ring
+    if (finish <= ring) {
         J.fin_off = 0;
+        J.tail_off = (int32_t)((finish + 127) / 128 * 128);
+        J.tail_bytes = J.tail_off < (int32_t)ring ? (int32_t)ring - J.tail_off : 0;
         return stream;
     }
     J.fin_off = (int32_t)((stream + 127) / 128 * 128);
+    J.tail_off = 0;
+    J.tail_bytes = (int32_t)ring;
     return (size_t)J.fin_off + finish;
 }
 

@@ -77,6 +77,9 @@ LINEAR_CASES = [
              seed=8),
     Workload("lin bf16 full vocab few requests", "linear", R=2, B=3, vocab=151936, dtype="bf16", sigma=1.0,
              noise=0.7, peak=8.0, seed=9),
+    # more than 32 draft positions (token slots beyond one warp)
+    Workload("lin f32 B=40", "linear", R=3, B=40, vocab=600, dtype="f32", sigma=1.0, noise=0.05, top_k=10, seed=10),
+    Workload("lin bf16 B=40 top-k 50", "linear", R=3, B=40, vocab=600, dtype="bf16", sigma=1.0, noise=0.05, seed=13),
 ]
 
 
@@ -133,6 +136,9 @@ TREE_CASES = [
              temperature=0.0, seed=24),
     Workload("tree max shape", "tree", R=2, B=16, K=16, V=128, vocab=2000, dtype="bf16", sigma=1.0, noise=0.7,
              peak=3.0, seed=25),
+    # a chain longer than 32 nodes (token slots beyond one warp)
+    Workload("tree deep chain", "tree", R=2, B=40, K=1, V=48, vocab=600, dtype="f32", sigma=1.0, noise=0.02,
+             top_k=10, seed=26),
 ]
 
 
