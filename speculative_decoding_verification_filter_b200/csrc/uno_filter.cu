@@ -47,6 +47,7 @@ struct RowJob {
     int32_t merge_cap;                // entries of the merge area
     int32_t fin_off;                  // shared-memory offset of the finishing area (0: the ring)
     int32_t tail_off, tail_bytes;     // shared-memory scratch of the request tails
+    int32_t nst, fin_stride;          // pipelined kernel: ring stages, bytes per finishing warp
     // filter outputs
     int32_t* out_ids;
     float* out_probs;
@@ -120,6 +121,18 @@ struct Elem<__nv_bfloat16> {
         const uint32_t w = (e < 2) ? r.x : (e < 4) ? r.y : (e < 6) ? r.z : r.w;
         return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
     }
+    // bit e set when element e is finite and >= t; *bad when some element is NaN or +inf
+    __device__ static uint32_t elem_mask(const uint4& r, float t, uint32_t& bad) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int e = 0; e < kPerUnit; ++e) {
+            const float v = get(r, e);
+            const bool nonfinite = (v != v) || v == __int_as_float(0x7f800000);
+            bad |= nonfinite ? 1u : 0u;
+            m |= (!nonfinite && v >= t && v != -__int_as_float(0x7f800000)) ? (1u << e) : 0u;
+        }
+        return m;
+    }
     __device__ static float load_scalar(const unsigned char* p) {
         const uint16_t h = *reinterpret_cast<const uint16_t*>(p);
         return __uint_as_float((uint32_t)h << 16);
@@ -132,6 +145,14 @@ struct Elem<__nv_bfloat16> {
     __device__ static Top top_init() {
         const __nv_bfloat16 ninf = __ushort_as_bfloat16((unsigned short)0xff80u);
         return __halves2bfloat162(ninf, ninf);
+    }
+    // running maximum of a unit's elements (NaN skipped)
+    __device__ static void max_update(Top& m1, const uint4& r) {
+        m1 = __hmax2(__hmax2(m1, __hmax2(w2(r.x), w2(r.y))), __hmax2(w2(r.z), w2(r.w)));
+    }
+    __device__ static uint32_t lane_max_ord(Top m1) {
+        const float f = fmaxf(__low2float(m1), __high2float(m1));
+        return (f > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(f, 0.0f)) : 0u;
     }
     __device__ static void top2_update(Top& m1, Top& m2, const uint4* c) {
 #pragma unroll
@@ -218,10 +239,28 @@ struct Elem<float> {
         const uint32_t w = (e == 0) ? r.x : (e == 1) ? r.y : (e == 2) ? r.z : r.w;
         return __uint_as_float(w);
     }
+    __device__ static uint32_t elem_mask(const uint4& r, float t, uint32_t& bad) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int e = 0; e < kPerUnit; ++e) {
+            const float v = get(r, e);
+            const bool nonfinite = (v != v) || v == __int_as_float(0x7f800000);
+            bad |= nonfinite ? 1u : 0u;
+            m |= (!nonfinite && v >= t && v != -__int_as_float(0x7f800000)) ? (1u << e) : 0u;
+        }
+        return m;
+    }
     __device__ static float load_scalar(const unsigned char* p) { return *reinterpret_cast<const float*>(p); }
     __device__ static uint4 neg_inf_unit() { return make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u); }
     typedef float Top;
     __device__ static Top top_init() { return -__int_as_float(0x7f800000); }
+    __device__ static void max_update(Top& m1, const uint4& r) {
+        m1 = fmaxf(fmaxf(m1, fmaxf(__uint_as_float(r.x), __uint_as_float(r.y))),
+                   fmaxf(__uint_as_float(r.z), __uint_as_float(r.w)));
+    }
+    __device__ static uint32_t lane_max_ord(Top m1) {
+        return (m1 > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(m1, 0.0f)) : 0u;
+    }
     __device__ static void top2_update(Top& m1, Top& m2, const uint4* c) {
 #pragma unroll
         for (int u = 0; u < kUnits; ++u) {
@@ -411,9 +450,9 @@ template <typename T>
 __device__ __forceinline__ bool ring_take(const Ring& R, int q, int warp, int lane, uint4* c) {
     uint64_t* bar = R.full + (q % kStages);
     const uint32_t par = (uint32_t)((q / kStages) & 1);
-    bool got = mbar_try_wait(bar, par);
-    if (!got) got = mbar_wait_bounded(bar, par);
-    const bool ok = __all_sync(kFull, got);
+    uint32_t got = 0;  // lane 0 polls; the warp learns the outcome
+    if (lane == 0) got = (mbar_try_wait(bar, par) || mbar_wait_bounded(bar, par)) ? 1u : 0u;
+    const bool ok = __shfl_sync(kFull, got, 0) != 0;
     const int u0 = R.ub + ring_stage_index(R, q) * kStageUnits + warp * kWarpUnits + lane;
     const uint4* sp = reinterpret_cast<const uint4*>(R.stages + (q % kStages) * kStageBytes) + warp * kWarpUnits + lane;
 #pragma unroll
@@ -429,10 +468,7 @@ __device__ __forceinline__ void ring_release(const Ring& R, int q, int lane) {
         int* d = R.done + (q % kStages);
         if (atomicAdd(d, 1) == kWarps - 1) {
             atomicExch(d, 0);
-            if (q + kStages < R.total) {
-                fence_proxy_async();
-                ring_issue(R, q + kStages);
-            }
+            if (q + kStages < R.total) ring_issue(R, q + kStages);
         }
     }
 }
@@ -915,19 +951,22 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     flags = __reduce_or_sync(kFull, flags);
     if (__any_sync(kFull, qbig)) return false;
     __syncwarp();
-    for (int i = 0; i <= B; ++i) {
-        const int c = pcnt[i];
-        for (int j = lane; j < c; j += 32) {
-            pid[i * kc + j] = __ldcg(J.c_ids + (size_t)(base + i) * kc + j);
-            ppr[i * kc + j] = __ldcg(J.c_probs + (size_t)(base + i) * kc + j);
+    // every row at once: the loads are independent, so they overlap
+#pragma unroll 4
+    for (int idx = lane; idx < (B + 1) * kc; idx += 32) {
+        const int i = idx / kc, j = idx - i * kc;
+        if (j < pcnt[i]) {
+            pid[idx] = __ldcg(J.c_ids + (size_t)(base + i) * kc + j);
+            ppr[idx] = __ldcg(J.c_probs + (size_t)(base + i) * kc + j);
         }
     }
-    for (int i = 0; i < B; ++i) {
-        const int c = qcnt[i];
-        const int64_t qrow = (int64_t)r * B + i;
-        for (int j = lane; j < c; j += 32) {
-            qid[i * QS + j] = J.q_ids[(size_t)qrow * J.q_cap + j];
-            qpr[i * QS + j] = J.q_probs[(size_t)qrow * J.q_cap + j];
+    const int64_t qbase = (int64_t)r * B;
+#pragma unroll 4
+    for (int idx = lane; idx < B * QS; idx += 32) {
+        const int i = idx / QS, j = idx % QS;
+        if (j < qcnt[i]) {
+            qid[idx] = J.q_ids[(size_t)(qbase + i) * J.q_cap + j];
+            qpr[idx] = J.q_probs[(size_t)(qbase + i) * J.q_cap + j];
         }
     }
     __syncwarp();
@@ -1037,11 +1076,12 @@ __device__ __noinline__ bool tree_tail_fast(const RowJob& J, int32_t r, unsigned
     }
     flags = __reduce_or_sync(kFull, flags);
     __syncwarp();
-    for (int j = 0; j < n; ++j) {
-        const int c = ncnt[j];
-        for (int e = lane; e < c; e += 32) {
-            nid[j * kc + e] = __ldcg(J.c_ids + (size_t)(base + j) * kc + e);
-            npr[j * kc + e] = __ldcg(J.c_probs + (size_t)(base + j) * kc + e);
+#pragma unroll 4
+    for (int idx = lane; idx < n * kc; idx += 32) {
+        const int j = idx / kc, e = idx - j * kc;
+        if (e < ncnt[j]) {
+            nid[idx] = __ldcg(J.c_ids + (size_t)(base + j) * kc + e);
+            npr[idx] = __ldcg(J.c_probs + (size_t)(base + j) * kc + e);
         }
     }
     __syncwarp();
@@ -1100,6 +1140,26 @@ __device__ __forceinline__ void request_tail(const RowJob& J, int32_t req, doubl
     } else {
         if (!tree_tail_fast(J, req, tail_smem, lane)) tree_tail(J, req, wd, lane);
     }
+}
+
+// One warp: count a finished row of request req; the warp that counts the
+// request's last row runs the request's tail.
+template <int MODE>
+__device__ __forceinline__ void request_arrive(const RowJob& J, int32_t req, double* wd, unsigned char* tail_smem,
+                                               int lane) {
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+        __threadfence();
+        const uint32_t t = atomicAdd(J.req_ticket + req, 1u);
+        last = (t == (uint32_t)(J.rpr - 1));
+        if (last) {
+            atomicExch(J.req_ticket + req, 0u);
+            __threadfence();
+        }
+    }
+    last = __shfl_sync(kFull, last, 0);
+    if (last) request_tail<MODE>(J, req, wd, tail_smem, lane);
 }
 
 
@@ -1229,19 +1289,7 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
             J.c_count[row] = kept;
             J.c_flags[row] = rflags;
         }
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-            __threadfence();
-            const uint32_t t = atomicAdd(J.req_ticket + req, 1u);
-            last = (t == (uint32_t)(J.rpr - 1));
-            if (last) {
-                atomicExch(J.req_ticket + req, 0u);
-                __threadfence();
-            }
-        }
-        last = __shfl_sync(kFull, last, 0);
-        if (last) request_tail<MODE>(J, req, wd, tail_smem, lane);
+        request_arrive<MODE>(J, req, wd, tail_smem, lane);
     }
 }
 
@@ -1551,6 +1599,680 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const RowJob J) {
 }
 
 // ---------------------------------------------------------------------------
+// The pipelined row kernel (k <= 64, no dense row): one persistent CTA per
+// SM works through a static list of items (row segments: item = row * S +
+// segment, CTA b takes items b, b + grid, ...).
+//
+//   warp 0      producer: lane 0 keeps a ring of `nst` 16 KB stages filled
+//               with bulk copies (TMA, no multicast), running across item
+//               boundaries, each stage tracked by a `full` mbarrier and
+//               given back through an `empty` mbarrier;
+//   warps 1..8  consumers: per item, a threshold seed from the lane maxima
+//               of the first stages (read twice from shared memory), then
+//               the threshold filter of every stage into per-warp candidate
+//               buffers of the item's slot;
+//   warps 9..12 finishers: finisher f takes the items whose ordinal in the
+//               CTA's list is f mod 4 from slot f -- exact top-k of the
+//               slot's candidates with a warp bitonic merge, then the
+//               softmax / top-p / output / request-tail work of the row.
+//
+// The streaming never waits for a row's serial work: while a finisher works
+// on one row the producer and consumers are already on the next ones.  Every
+// wait is bounded; a wait that gives up sets the CTA's abort word, every
+// role stops at its next check, and rows that were not finished are written
+// with UNO_FLAG_TIMEOUT.
+// ---------------------------------------------------------------------------
+constexpr int kPipeConsumers = 8;
+constexpr int kPipeFinishers = 4;
+constexpr int kPipeSlots = kPipeFinishers;
+constexpr int kPipeWarps = 1 + kPipeConsumers + kPipeFinishers;
+constexpr int kPipeThreads = 32 * kPipeWarps;
+constexpr int kPipeMaxK = 64;
+// A pipelined stage is 16 KB (1024 units).  In the select pass consumer warp
+// st % 8 owns stage st of an item whole: lane l takes units l, l + 32, ...,
+// (conflict-free shared loads).  In the seed pass every
+// consumer warp reads a slice of each seed stage: warp c units [c*128,
+// (c+1)*128), four per lane.
+constexpr int kPStageBytes = 16384;
+constexpr int kPStageUnits = kPStageBytes / 16;                 // 1024
+constexpr int kPLaneUnits = kPStageUnits / 32;                  // 32 per lane per stage
+constexpr int kPSliceUnits = kPStageUnits / kPipeConsumers;     // 128 (seed pass)
+constexpr int kPBootStages = 8;                                 // stages of the threshold seed
+constexpr int kPipeMinStages = 10, kPipeMaxStages = 12;
+static_assert(kPipeMinStages > kPBootStages, "a stage beyond the seed stages is in flight");
+// Suspend hint of the off-path waits (ns): the waiting thread sleeps until
+// the phase completes or the hint runs out, instead of polling.
+constexpr uint32_t kNapNs = 2000;
+
+struct __align__(16) PipeShared {
+    uint64_t full[kPipeMaxStages];          // stage bytes arrived
+    uint64_t empty[kPipeMaxStages];         // the stage's owner warp is done with it
+    uint32_t fill[kPipeMaxStages];          // ring element each buffer holds or is receiving
+    uint64_t slot_full[kPipeSlots];         // every consumer warp is done with the slot's item
+    uint64_t slot_empty[kPipeSlots];        // the finisher is done with the slot's buffers
+    unsigned long long tau[2];              // CTA threshold of the current item (by item parity)
+    uint32_t boot[2][kPipeConsumers * 32];  // lane maxima of the seed stages (by item parity)
+    uint32_t seed[2];                       // the seed threshold's high word (by item parity)
+    int wcnt[kPipeConsumers];               // candidate counts (compaction bookkeeping)
+    int cnt[kPipeSlots][kPipeConsumers];    // candidates per consumer warp of the slot's item
+    uint32_t bad[kPipeSlots];               // NaN / +inf (bit 0) or gave-up (bit 1) of the slot's item
+    int abort;
+};
+
+template <int MODE>
+__device__ __forceinline__ bool item_active(const RowJob& J, int64_t row) {
+    if (MODE != kModeTree) return true;
+    int32_t nn = J.num_nodes[row / J.rpr];
+    nn = nn < 1 ? 1 : (nn > J.V ? J.V : nn);
+    return (int32_t)(row % J.V) < nn;
+}
+
+// 16-byte units [ub, ue) of a row segment and its stage count.
+struct SegGeom {
+    RowGeom g;
+    const unsigned char* ubase;  // unit 0 of the row (16-byte aligned)
+    int ub, ue, nstage;
+};
+
+template <typename T>
+__device__ __forceinline__ SegGeom seg_geom(const RowJob& J, int64_t row, int seg) {
+    SegGeom s;
+    s.g = row_geom<T>(J, row);
+    s.ubase = s.g.base + (size_t)s.g.head * Elem<T>::kBytes;
+    const int64_t per = (s.g.nunit + J.S - 1) / J.S;
+    const int64_t vb = per * seg < s.g.nunit ? per * seg : s.g.nunit;
+    const int64_t ve = vb + per < s.g.nunit ? vb + per : s.g.nunit;
+    s.ub = (int)vb;
+    s.ue = (int)ve;
+    s.nstage = (int)((ve - vb + kPStageUnits - 1) / kPStageUnits);
+    return s;
+}
+
+__device__ __forceinline__ bool pipe_aborted(const PipeShared& P) {
+    return *reinterpret_cast<const volatile int*>(&P.abort) != 0;
+}
+
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait that also gives up once the CTA has aborted.  The first probe
+// returns at once; later ones sleep in the barrier until the phase completes
+// (or the hint runs out), so waiting threads leave the issue slots and the
+// shared-memory pipe to the others.  Every thread that calls it polls; call
+// it with the whole warp converged.
+__device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, const PipeShared& P) {
+    if (mbar_try_wait(bar, parity)) return true;
+    for (uint32_t it = 0; it < (kMaxWaitTries >> 4); ++it) {
+        if (mbar_try_wait_hint(bar, parity, kNapNs)) return true;
+        if (pipe_aborted(P)) return false;
+    }
+    return false;
+}
+
+__device__ __forceinline__ bool pipe_wait_warp(uint64_t* bar, uint32_t parity, const PipeShared& P) {
+    return __all_sync(kFull, pipe_wait(bar, parity, P));
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_shared(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_shared(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+// Whole warp: wait until ring element qq has landed in its buffer.  A buffer
+// may still hold an older element that another warp has not released (the
+// stages of an item go to different warps), and a parity wait cannot tell
+// that phase from qq's, so the buffer's fill tag must name qq first; the
+// producer stores the tag (release) before it arms the barrier for qq.
+__device__ __forceinline__ bool pipe_wait_stage(PipeShared& P, uint32_t qq, uint32_t nst) {
+    const uint32_t b = qq % nst;
+    bool ok = ld_acquire_shared(&P.fill[b]) == qq;
+    for (uint32_t it = 0; !ok && it < kMaxWaitTries; ++it) {
+        __nanosleep(64);
+        ok = ld_acquire_shared(&P.fill[b]) == qq;
+        if (!ok && (it & 15u) == 15u && pipe_aborted(P)) break;
+    }
+    if (!__all_sync(kFull, ok)) return false;
+    return pipe_wait_warp(&P.full[b], (qq / nst) & 1u, P);
+}
+
+// Consumer barrier over warps 1..8 (named barrier 1) returning the OR of v.
+__device__ __forceinline__ bool consumers_sync_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.or.pred p, 1, %2, q;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "n"(kPipeConsumers * 32)
+        : "memory");
+    return r != 0;
+}
+
+// Plain consumer barrier (named barrier 1).
+__device__ __forceinline__ void consumers_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kPipeConsumers * 32) : "memory");
+}
+
+// Producer (one thread).
+template <typename T, int MODE>
+__device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring) {
+    const int64_t nitems = J.rows * J.S;
+    const uint32_t nst = (uint32_t)J.nst;
+    uint32_t q = 0;
+    bool ok = true;
+    for (int64_t it = blockIdx.x; ok && it < nitems; it += gridDim.x) {
+        const int64_t row = it / J.S;
+        if (!item_active<MODE>(J, row)) continue;
+        const SegGeom s = seg_geom<T>(J, row, (int)(it % J.S));
+        for (int st = 0; st < s.nstage; ++st) {
+            const uint32_t b = q % nst;
+            if (q >= nst && !pipe_wait(&P.empty[b], ((q / nst) - 1u) & 1u, P)) {
+                ok = false;
+                break;
+            }
+            if (pipe_aborted(P)) {
+                ok = false;
+                break;
+            }
+            const int u0 = s.ub + st * kPStageUnits;
+            const int nu = (s.ue - u0) < kPStageUnits ? (s.ue - u0) : kPStageUnits;
+            st_release_shared(&P.fill[b], q);  // the buffer now belongs to element q
+            mbar_expect_tx(&P.full[b], (uint32_t)nu * 16u);
+            bulk_g2s(ring + (size_t)b * kPStageBytes, s.ubase + (size_t)u0 * 16, (uint32_t)nu * 16u, &P.full[b]);
+            ++q;
+        }
+    }
+    if (!ok) atomicExch(&P.abort, 1);
+    // the copies still in flight land before the CTA may exit (bounded)
+    for (uint32_t d = q > nst ? q - nst : 0u; d < q; ++d) (void)mbar_wait_bounded(&P.full[d % nst], (d / nst) & 1u);
+}
+
+// Hand a stage back to the producer.  The warp's shared loads of it have
+// completed (their values decided the warp's branches), so a plain arrival
+// orders them before the producer's next copy into the stage.
+__device__ __forceinline__ void pipe_release(PipeShared& P, uint32_t b, int lane) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&P.empty[b]);
+}
+
+// A valid threshold from the 256 lane maxima (0 = no element): the largest x
+// with a zero low half such that at least k of them are >= x.  Distinct lanes
+// hold distinct elements, so at least k elements of the segment are >= x.
+// Two bits per step: the counts of three trial values travel packed in one
+// warp reduction (10 bits each; a count is at most 256).
+__device__ __forceinline__ uint32_t seed_threshold(const uint32_t* bv, int k, int lane) {
+    const uint4 x = reinterpret_cast<const uint4*>(bv)[2 * lane];
+    const uint4 y = reinterpret_cast<const uint4*>(bv)[2 * lane + 1];
+    const uint32_t v[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+    uint32_t p = 0;  // high bits of the answer found so far
+#pragma unroll
+    for (int sh = 14; sh >= 0; sh -= 2) {
+        const uint32_t t1 = (p | (1u << sh)) << 16, t2 = (p | (2u << sh)) << 16, t3 = (p | (3u << sh)) << 16;
+        uint32_t c = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            c += (v[j] >= t1 ? 1u : 0u) + (v[j] >= t2 ? (1u << 10) : 0u) + (v[j] >= t3 ? (1u << 20) : 0u);
+        c = __reduce_add_sync(kFull, c);
+        const uint32_t kk = (uint32_t)k;
+        const uint32_t d = ((c >> 20) >= kk) ? 3u : (((c >> 10) & 1023u) >= kk) ? 2u : ((c & 1023u) >= kk) ? 1u : 0u;
+        p |= d << sh;
+    }
+    return p << 16;
+}
+
+// One consumer warp's candidates of one stage: every element of the lane's
+// eight units that is >= the threshold (or NaN) is re-read from the stage
+// and appended; one element per lane per round, positions by ballot.  The
+// warp state travels by value (it stays in registers in the caller).
+struct AppendState {
+    int cnt;
+    uint64_t tau;
+    uint32_t bad;
+};
+
+template <typename T>
+__device__ __noinline__ AppendState pipe_append(uint64_t* buf, int* wcnt, AppendState st, uint64_t m,
+                                                const unsigned char* wstage, uint32_t id0, int hw, int k,
+                                                unsigned long long* s_tau, int lane) {
+    constexpr int KPU = Elem<T>::kPerUnit;
+    const unsigned lt = lanemask_lt();
+    while (__any_sync(kFull, m != 0ull)) {
+        uint64_t key = 0ull;
+        bool has = false;
+        if (m != 0ull) {
+            const int j = __ffsll((long long)m) - 1;
+            m &= m - 1ull;
+            const int u = j / KPU, e = j % KPU;
+            const float v = Elem<T>::load_scalar(wstage + (size_t)(u * 32) * 16 + (size_t)e * Elem<T>::kBytes);
+            if (v != v || v == __int_as_float(0x7f800000)) {
+                st.bad |= 1u;
+            } else if (v != -__int_as_float(0x7f800000)) {
+                key = make_key(v, id0 + (uint32_t)(u * 32 * KPU + e));
+                has = key > st.tau;
+            }
+        }
+        const unsigned bal = __ballot_sync(kFull, has);
+        if (has) buf[st.cnt + __popc(bal & lt)] = key;
+        st.cnt += __popc(bal);
+        if (st.cnt > hw) {
+            __syncwarp();
+            const Compacted cp = warp_compact(buf, wcnt, st.cnt, st.tau, k, s_tau, lane);
+            st.cnt = cp.cnt;
+            st.tau = cp.tau;
+        }
+    }
+    __syncwarp();
+    return st;
+}
+
+// The candidates of one stage (ub = the lane's units, of its 32, whose
+// maximum may reach the threshold): each round every lane with a unit
+// left re-reads it from the stage, masks its finite elements >= the
+// threshold, and writes them at positions from bit-sliced ballots of the
+// per-lane counts.  A round that would overflow the buffer goes one element
+// per lane at a time with compaction in between (pipe_append).
+template <typename T>
+__device__ __forceinline__ AppendState pipe_units(uint64_t* buf, int* wcnt, AppendState st, uint32_t ub,
+                                               const uint4* sp, uint32_t id0, int hw, int cap_w, int k,
+                                               unsigned long long* s_tau, int lane) {
+    constexpr int KPU = Elem<T>::kPerUnit;
+    const unsigned lt = lanemask_lt();
+    while (__any_sync(kFull, ub != 0u)) {
+        const float tf = tau_value(st.tau);
+        uint32_t em = 0;
+        uint4 r = make_uint4(0u, 0u, 0u, 0u);
+        int u = 0;
+        if (ub != 0u) {
+            u = __ffs(ub) - 1;
+            ub &= ub - 1u;
+            r = sp[u * 32];
+            em = Elem<T>::elem_mask(r, tf, st.bad);
+        }
+        const uint32_t c = (uint32_t)__popc(em);  // <= 8
+        const unsigned b0 = __ballot_sync(kFull, c & 1u), b1 = __ballot_sync(kFull, c & 2u);
+        const unsigned b2 = __ballot_sync(kFull, c & 4u), b3 = __ballot_sync(kFull, c & 8u);
+        const int tot = __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2) + 8 * __popc(b3);
+        if (tot == 0) continue;
+        if (st.cnt + tot > cap_w) {
+            st = pipe_append<T>(buf, wcnt, st, (uint64_t)em, reinterpret_cast<const unsigned char*>(sp + u * 32),
+                                id0 + (uint32_t)(u * 32 * KPU), hw, k, s_tau, lane);
+            continue;
+        }
+        int pos = st.cnt + __popc(b0 & lt) + 2 * __popc(b1 & lt) + 4 * __popc(b2 & lt) + 8 * __popc(b3 & lt);
+        const uint32_t idu = id0 + (uint32_t)(u * 32 * KPU);
+        while (em != 0u) {
+            const int e = __ffs(em) - 1;
+            em &= em - 1u;
+            buf[pos++] = make_key(Elem<T>::get(r, e), idu + (uint32_t)e);
+        }
+        st.cnt += tot;
+        if (st.cnt > hw) {
+            __syncwarp();
+            const Compacted cp = warp_compact(buf, wcnt, st.cnt, st.tau, k, s_tau, lane);
+            st.cnt = cp.cnt;
+            st.tau = cp.tau;
+        }
+    }
+    __syncwarp();
+    return st;
+}
+
+// Consumer warp c (0 .. kPipeConsumers-1).
+template <typename T, int MODE>
+__device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char* ring, uint64_t* slots, int c,
+                             int lane) {
+    typedef typename Elem<T>::Tau Tau;
+    constexpr int KPU = Elem<T>::kPerUnit;
+    const int64_t nitems = J.rows * J.S;
+    const uint32_t nst = (uint32_t)J.nst;
+    const int k = J.k, hw = J.hw, cap_w = J.cap_w, S = J.S;
+    uint32_t q = 0;              // ring element of the item's first stage
+    uint32_t a = 0;              // active items so far
+    uint32_t used = 0, par = 0;  // per slot: used before; parity of its current use
+    bool fail = false;
+    int64_t i = 0;
+    for (int64_t it = blockIdx.x; it < nitems; it += gridDim.x, ++i) {
+        const int64_t row = it / S;
+        const int seg = (int)(it % S);
+        if (!item_active<MODE>(J, row)) continue;
+        const int slot = (int)(i % kPipeSlots);
+        const uint32_t sb = 1u << slot;
+        // the finisher is done with this slot's previous item
+        if ((used & sb) && !pipe_wait_warp(&P.slot_empty[slot], (par & sb) ? 0u : 1u, P)) fail = true;
+        const SegGeom s = seg_geom<T>(J, row, seg);
+        const int nA = s.nstage < kPBootStages ? s.nstage : kPBootStages;
+
+        // pass 1: lane maxima of this warp's slice of the first nA stages
+        typename Elem<T>::Top m1 = Elem<T>::top_init();
+        for (int st = 0; st < nA && !fail; ++st) {
+            const uint32_t qq = q + st;
+            const uint32_t b = qq % nst;
+            if (!pipe_wait_stage(P, qq, nst)) {
+                fail = true;
+                break;
+            }
+            const int u0 = s.ub + st * kPStageUnits + c * kPSliceUnits + lane;
+            const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)b * kPStageBytes) + c * kPSliceUnits + lane;
+#pragma unroll
+            for (int u = 0; u < kPSliceUnits / 32; ++u)
+                if (u0 + u * 32 < s.ue) Elem<T>::max_update(m1, sp[u * 32]);
+        }
+        P.boot[a & 1][c * 32 + lane] = fail ? 0u : Elem<T>::lane_max_ord(m1);
+        // every consumer warp takes the same exit decision here
+        if (consumers_sync_or(fail || pipe_aborted(P))) {
+            if (lane == 0) atomicExch(&P.abort, 1);
+            return;
+        }
+        unsigned long long* s_tau = &P.tau[a & 1];
+
+        WarpState ws;
+        ws.buf = slots + ((size_t)slot * kPipeConsumers + c) * cap_w;
+        ws.wcnt = &P.wcnt[c];
+        ws.cnt = 0;
+        ws.bad = 0u;
+        if (c == 0) {
+            // the threshold seed, for every consumer warp
+            const uint32_t t0 = seed_threshold(P.boot[a & 1], k, lane);
+            if (lane == 0) {
+                P.seed[a & 1] = t0;
+                P.tau[(a + 1) & 1] = 0ull;  // nobody reads the previous item's threshold now
+            }
+        } else if (c == 1 && seg == 0) {
+            // row head / tail scalars (fewer than 16): every finite one
+            const int64_t ntail = J.vocab - s.g.tail_begin;
+            const int64_t nsc = s.g.head + ntail;
+            uint64_t key = 0ull;
+            bool has = false;
+            if (lane < nsc) {
+                const int64_t id = (lane < s.g.head) ? (int64_t)lane : s.g.tail_begin + (lane - s.g.head);
+                const float v = Elem<T>::load_scalar(s.g.base + (size_t)id * Elem<T>::kBytes);
+                if (v != v || v == __int_as_float(0x7f800000)) {
+                    ws.bad |= 1u;
+                } else if (v != -__int_as_float(0x7f800000)) {
+                    key = make_key(v, (uint32_t)id);
+                    has = true;
+                }
+            }
+            const unsigned bal = __ballot_sync(kFull, has);
+            if (has) ws.buf[__popc(bal & lanemask_lt())] = key;
+            ws.cnt = __popc(bal);
+        }
+        consumers_sync();
+        ws.tau = (uint64_t)P.seed[a & 1] << 32;
+
+        // pass 2: select, this warp's stages of the item
+        const uint32_t id_base = (uint32_t)s.g.head;
+        Tau tau_v = Elem<T>::make_tau(tau_value(ws.tau));
+        for (int st = c; st < s.nstage && !fail; st += kPipeConsumers) {
+            const uint32_t qq = q + st;
+            const uint32_t b = qq % nst;
+            if (!pipe_wait_stage(P, qq, nst)) {
+                fail = true;
+                break;
+            }
+            const int us = s.ub + st * kPStageUnits + lane;  // the lane's first unit in the row
+            const uint4* lsp = reinterpret_cast<const uint4*>(ring + (size_t)b * kPStageBytes) + lane;
+            uint32_t ub = 0;  // bit j: the lane's unit j (unit us + 32 j) may hold a candidate
+            if (s.ue - (s.ub + st * kPStageUnits) >= kPStageUnits) {
+#pragma unroll
+                for (int u = 0; u < kPLaneUnits; ++u) ub |= Elem<T>::maybe(lsp[u * 32], tau_v) ? (1u << u) : 0u;
+            } else {  // the segment's last stage: only its units (the rest holds older data)
+                const int left = s.ue - us;
+#pragma unroll
+                for (int u = 0; u < kPLaneUnits; ++u)
+                    if (32 * u < left) ub |= Elem<T>::maybe(lsp[u * 32], tau_v) ? (1u << u) : 0u;
+            }
+            if (__any_sync(kFull, ub != 0u)) {
+                const AppendState r = pipe_units<T>(ws.buf, ws.wcnt, AppendState{ws.cnt, ws.tau, ws.bad}, ub, lsp,
+                                                    id_base + (uint32_t)us * KPU, hw, cap_w, k, s_tau, lane);
+                ws.cnt = r.cnt;
+                ws.tau = r.tau;
+                ws.bad = r.bad;
+            }
+            pipe_release(P, b, lane);
+            // adopt a better threshold found by another warp
+            const unsigned long long stv = *reinterpret_cast<volatile unsigned long long*>(s_tau);
+            if (stv > ws.tau) ws.tau = stv;
+            tau_v = Elem<T>::make_tau(tau_value(ws.tau));
+        }
+        {
+            const unsigned long long stv = *reinterpret_cast<volatile unsigned long long*>(s_tau);
+            if (stv > ws.tau) ws.tau = stv;
+            ws.cnt = warp_keep_ge(ws.buf, ws.cnt, ws.tau, lane);
+        }
+        const uint32_t wb = __reduce_or_sync(kFull, ws.bad | (fail ? 2u : 0u));
+        if (lane == 0) {
+            P.cnt[slot][c] = ws.cnt;
+            if (wb) atomicOr(&P.bad[slot], wb);
+            mbar_arrive(&P.slot_full[slot]);
+        }
+        if (fail && lane == 0) atomicExch(&P.abort, 1);
+        q += (uint32_t)s.nstage;
+        ++a;
+        par ^= sb;
+        used |= sb;
+    }
+}
+
+// Ascending bitonic merge of a bitonic sequence of 64 keys (element e = lane
+// in a, e = lane + 32 in b).
+__device__ __forceinline__ void warp_merge64(uint64_t& a, uint64_t& b, int lane) {
+    {
+        const uint64_t lo = a < b ? a : b, hi = a < b ? b : a;
+        a = lo;
+        b = hi;
+    }
+#pragma unroll
+    for (int stride = 16; stride > 0; stride >>= 1) {
+        const uint64_t pa = __shfl_xor_sync(kFull, a, stride), pb = __shfl_xor_sync(kFull, b, stride);
+        const bool lower = (lane & stride) == 0;
+        a = lower ? (a < pa ? a : pa) : (a < pa ? pa : a);
+        b = lower ? (b < pb ? b : pb) : (b < pb ? pb : b);
+    }
+}
+
+// The best min(k, U) of U distinct keys get(0 .. U-1) (k <= 64), written to
+// sel[] in descending order; one warp.  Chunks of 64 are sorted and merged
+// into a running best 64 (the 64 smallest complements).
+template <class Get>
+__device__ __forceinline__ int warp_topk64(int U, int k, const Get& get, uint64_t* sel, int lane) {
+    uint64_t ra = ~0ull, rb = ~0ull;
+    for (int base = 0; base < U; base += 64) {
+        uint64_t xa = base + lane < U ? ~get(base + lane) : ~0ull;
+        uint64_t xb = base + 32 + lane < U ? ~get(base + 32 + lane) : ~0ull;
+        warp_sort64(xa, xb, lane);
+        if (base == 0) {
+            ra = xa;
+            rb = xb;
+        } else {
+            // element e pairs with chunk element 63 - e
+            const uint64_t ca = __shfl_xor_sync(kFull, xb, 31), cb = __shfl_xor_sync(kFull, xa, 31);
+            ra = ra < ca ? ra : ca;
+            rb = rb < cb ? rb : cb;
+            warp_merge64(ra, rb, lane);
+        }
+    }
+    const int n = U < k ? U : k;
+    if (lane < n) sel[lane] = ~ra;
+    if (lane + 32 < n) sel[lane + 32] = ~rb;
+    __syncwarp();
+    return n;
+}
+
+// The last finishing warp of a split row: the best min(k, U) keys of the U
+// keys its segments published, into sel[] (descending); rowbad gets the OR
+// of the segments' flags.  Segment t's keys occupy indices [excl_t,
+// excl_t + count_t) of the merged order (lane t holds excl_t; S <= 16).
+__device__ __noinline__ int merge_partials(const RowJob& J, int64_t row, uint64_t* sel, uint32_t& rowbad, int lane) {
+    const size_t p0 = (size_t)row * J.S;
+    const int c_l = lane < J.S ? __ldcg(J.part_count + p0 + lane) : 0;
+    rowbad = __reduce_or_sync(kFull, lane < J.S ? __ldcg(J.part_flags + p0 + lane) : 0u);
+    int incl = c_l;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += t;
+    }
+    const int U = __shfl_sync(kFull, incl, 31);
+    const int excl = incl - c_l;
+    const int kk = J.k;
+    const unsigned long long* pbase = reinterpret_cast<const unsigned long long*>(J.part_keys + p0 * kk);
+    uint64_t ra = ~0ull, rb = ~0ull;
+    for (int base = 0; base < U; base += 64) {
+        const int ga = base + lane, gb = base + 32 + lane;
+        int sa = 0, sg = 0;
+        for (int t = 1; t < J.S; ++t) {
+            const int e = __shfl_sync(kFull, excl, t);
+            sa = (e <= ga) ? t : sa;
+            sg = (e <= gb) ? t : sg;
+        }
+        const int ea = __shfl_sync(kFull, excl, sa), eb = __shfl_sync(kFull, excl, sg);
+        uint64_t xa = ga < U ? ~(uint64_t)__ldcg(pbase + (size_t)sa * kk + (ga - ea)) : ~0ull;
+        uint64_t xb = gb < U ? ~(uint64_t)__ldcg(pbase + (size_t)sg * kk + (gb - eb)) : ~0ull;
+        warp_sort64(xa, xb, lane);
+        if (base == 0) {
+            ra = xa;
+            rb = xb;
+        } else {
+            const uint64_t ca = __shfl_xor_sync(kFull, xb, 31), cb = __shfl_xor_sync(kFull, xa, 31);
+            ra = ra < ca ? ra : ca;
+            rb = rb < cb ? rb : cb;
+            warp_merge64(ra, rb, lane);
+        }
+    }
+    const int n = U < kk ? U : kk;
+    if (lane < n) sel[lane] = ~ra;
+    if (lane + 32 < n) sel[lane + 32] = ~rb;
+    __syncwarp();
+    return n;
+}
+
+// Finishing warp f.
+template <typename T, int MODE>
+__device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slots, unsigned char* scratch, int f,
+                            int lane) {
+    uint64_t* sel = reinterpret_cast<uint64_t*>(scratch);            // [kPipeMaxK]
+    double* wd = reinterpret_cast<double*>(sel + kPipeMaxK);         // [kPipeMaxK]
+    unsigned char* tail = reinterpret_cast<unsigned char*>(wd + kPipeMaxK);
+    FinishShared unused_fs;
+    const int64_t nitems = J.rows * J.S;
+    const int slot = f;
+    const uint64_t* sbuf = slots + (size_t)slot * kPipeConsumers * J.cap_w;
+    uint32_t use = 0;
+    for (int64_t it = blockIdx.x + (int64_t)f * gridDim.x; it < nitems; it += (int64_t)kPipeFinishers * gridDim.x) {
+        const int64_t row = it / J.S;
+        const int seg = (int)(it % J.S);
+        const int32_t req = (int32_t)(row / J.rpr);
+        if (!item_active<MODE>(J, row)) {
+            if (MODE != kModeFilter && seg == 0) request_arrive<MODE>(J, req, wd, tail, lane);
+            continue;
+        }
+        uint32_t rowbad = 2u;
+        int n = 0;
+        const bool ok = pipe_wait_warp(&P.slot_full[slot], use & 1u, P);
+        ++use;
+        if (ok) {
+            int cw[kPipeConsumers];
+            int U = 0;
+#pragma unroll
+            for (int w = 0; w < kPipeConsumers; ++w) {
+                cw[w] = P.cnt[slot][w];
+                U += cw[w];
+            }
+            rowbad = P.bad[slot];
+            const int cap_w = J.cap_w;
+            auto get = [&](int g) -> uint64_t {
+                int w = 0, off = g;
+#pragma unroll
+                for (int t = 0; t < kPipeConsumers - 1; ++t) {
+                    if (w == t && off >= cw[t]) {
+                        off -= cw[t];
+                        w = t + 1;
+                    }
+                }
+                return sbuf[(size_t)w * cap_w + off];
+            };
+            n = warp_topk64(U, J.k, get, sel, lane);
+            __syncwarp();
+            if (lane == 0) {
+                P.bad[slot] = 0u;
+                mbar_arrive(&P.slot_empty[slot]);
+            }
+        } else if (lane == 0) {
+            atomicExch(&P.abort, 1);
+        }
+        if (J.S > 1) {
+            // publish this segment's best; the last segment of the row merges
+            const size_t pslot = (size_t)row * J.S + seg;
+            uint64_t* pk = J.part_keys + pslot * J.k;
+            if (lane < n) pk[lane] = sel[lane];
+            if (lane + 32 < n) pk[lane + 32] = sel[lane + 32];
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) {
+                J.part_count[pslot] = n;
+                J.part_flags[pslot] = rowbad;
+                __threadfence();
+                const uint32_t t = atomicAdd(J.row_ticket + row, 1u);
+                last = (t == (uint32_t)(J.S - 1));
+                if (last) {
+                    atomicExch(J.row_ticket + row, 0u);
+                    __threadfence();
+                }
+            }
+            last = __shfl_sync(kFull, last, 0);
+            if (!last) continue;
+            n = merge_partials(J, row, sel, rowbad, lane);
+        }
+        finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, tail, unused_fs, lane);
+    }
+}
+
+template <typename T, int MODE>
+__global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const RowJob J) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ PipeShared P;
+    unsigned char* ring = smem;                                                           // [nst][kPStageBytes]
+    uint64_t* slots = reinterpret_cast<uint64_t*>(smem + (size_t)J.nst * kPStageBytes);  // [slots][consumers][cap_w]
+    unsigned char* fin = reinterpret_cast<unsigned char*>(slots + (size_t)kPipeSlots * kPipeConsumers * J.cap_w);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < J.nst; ++s) {
+            mbar_init(&P.full[s], 1);
+            mbar_init(&P.empty[s], 1);
+            P.fill[s] = 0xffffffffu;  // no element yet
+        }
+        for (int s = 0; s < kPipeSlots; ++s) {
+            mbar_init(&P.slot_full[s], kPipeConsumers);
+            mbar_init(&P.slot_empty[s], 1);
+            P.bad[s] = 0u;
+        }
+        P.tau[0] = 0ull;
+        P.tau[1] = 0ull;
+        P.abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        if (lane == 0) pipe_produce<T, MODE>(J, P, ring);
+    } else if (warp <= kPipeConsumers) {
+        pipe_consume<T, MODE>(J, P, ring, slots, warp - 1, lane);
+    } else {
+        const int f = warp - 1 - kPipeConsumers;
+        pipe_finish<T, MODE>(J, P, slots, fin + (size_t)f * J.fin_stride, f, lane);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Tree expansion: one warp per request.
 // ---------------------------------------------------------------------------
 struct TreeJob {
@@ -1800,8 +2522,71 @@ static size_t row_smem_bytes(RowJob& J) {
     return (size_t)J.fin_off + finish;
 }
 
+// The pipelined kernel: segments per row, ring depth and shared memory.
+// Returns UNO_ERR_UNSUPPORTED (nothing launched) when it does not fit.
+template <typename T, int MODE>
+static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
+    J.hw = J.k + 16 > 64 ? J.k + 16 : 64;
+    J.cap_w = J.hw + 64;  // a round of unit appends that fits, else one element per lane per round
+    const int G = sm_count();
+    // segments per row, only when rows are fewer than the SMs: spread the
+    // items over the SMs, each segment at least one full stage, a price per
+    // extra segment (its seed and the merge)
+    int smax = J.rows <= kRowCounterWords ? split_bound(J.rows) : 1;
+    const int64_t by_work = J.vocab / Elem<T>::kPerUnit / kPStageUnits;
+    if (smax > by_work) smax = by_work < 1 ? 1 : (int)by_work;
+    int S = 1;
+    if (J.rows < G) {
+        double best = 1e300;
+        for (int s = 1; s <= smax; ++s) {
+            const int64_t rounds = (J.rows * s + G - 1) / G;
+            const double cost = (double)rounds / s + 0.03 * (s - 1);
+            if (cost < best - 1e-9) {
+                best = cost;
+                S = s;
+            }
+        }
+    }
+    J.S = S;
+    // shared memory: ring | candidate slots | per finisher: sel, wd, tail
+    const size_t slot_bytes = (size_t)kPipeSlots * kPipeConsumers * J.cap_w * 8;
+    size_t tail = 0;
+    if (MODE == kModeLinear)
+        tail = (size_t)(J.B + 1) * J.k * 8 + (size_t)J.B * 64 * 8 + (size_t)(4 * J.B + 2) * 4;
+    else if (MODE == kModeTree)
+        tail = (size_t)J.V * J.k * 8 + (size_t)J.V * 12 + (size_t)(J.B + 1) * 8;
+    const size_t dyn_max = 227 * 1024 - sizeof(PipeShared);
+    auto stride_of = [](size_t tb) { return align_up((size_t)2 * kPipeMaxK * 8 + tb, 128); };
+    auto stages_of = [&](size_t tb) -> int64_t {
+        const size_t fixed = slot_bytes + (size_t)kPipeFinishers * stride_of(tb);
+        return fixed >= dyn_max ? 0 : (int64_t)((dyn_max - fixed) / kPStageBytes);
+    };
+    // request rows in shared memory unless that leaves too shallow a ring
+    // (the tails then read them from global memory)
+    if (tail > 0 && stages_of(tail) < kPipeMinStages) tail = 0;
+    int64_t nst = stages_of(tail);
+    if (nst > kPipeMaxStages) nst = kPipeMaxStages;
+    if (nst < kPipeMinStages) return UNO_ERR_UNSUPPORTED;
+    J.nst = (int32_t)nst;
+    J.tail_bytes = (int32_t)tail;
+    J.fin_stride = (int32_t)stride_of(tail);
+    const size_t dyn = (size_t)nst * kPStageBytes + slot_bytes + (size_t)kPipeFinishers * J.fin_stride;
+    auto kern = pipe_kernel<T, MODE>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
+        return UNO_ERR_CUDA;
+    const int64_t items = J.rows * S;
+    const int64_t grid = items < G ? items : G;
+    if (grid <= 0) return UNO_OK;
+    kern<<<(unsigned)grid, kPipeThreads, dyn, stream>>>(J);
+    return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
+}
+
 template <typename T, int MODE>
 static uno_status launch_rows(RowJob J, cudaStream_t stream) {
+    if (J.k <= kPipeMaxK && J.out_dense == nullptr) {
+        const uno_status st = launch_pipe<T, MODE>(J, stream);
+        if (st != UNO_ERR_UNSUPPORTED) return st;
+    }
     // warp buffer: high-water mark, plus room for one piece of appends from
     // every lane; it also holds the threshold seed (2 keys per thread)
     J.hw = J.k + 16 > 64 ? J.k + 16 : 64;
