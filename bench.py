@@ -391,7 +391,9 @@ def run_ours(args, w):
                      "filter_ms": fq_ms, "verify_ms": fp_ms},
         "e2e": {"value": w.R * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": 2 * K,
+        # uno_filter_softmax launches one kernel; uno_linear_verify two for top-k <= 64 (rows, then
+        # request tails), one otherwise
+        "gpu_launches": K * (1 + (2 if min(w.top_k, w.vocab) <= 64 else 1)),
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -48,6 +48,7 @@ struct RowJob {
     int32_t fin_off;                  // shared-memory offset of the finishing area (0: the ring)
     int32_t tail_off, tail_bytes;     // shared-memory scratch of the request tails
     int32_t nst, fin_stride;          // pipelined kernel: ring stages, bytes per finishing warp
+    int32_t defer_tails;              // verifiers: the request tails run in tail_kernel afterwards
     // filter outputs
     int32_t* out_ids;
     float* out_probs;
@@ -918,11 +919,89 @@ __device__ __forceinline__ double smem_lookup(const int32_t* ids, const float* p
     return 0.0;
 }
 
+// One warp copies rows [0, nrows) x [0, width) of (ids, probs) from global
+// memory (row stride gs) into shared arrays (row stride ss).  Loads are
+// staged in registers, eight per lane, so that they are all in flight
+// together (a shared store between them could alias a later load and
+// serialise the round trips).  Entries past a row's count are copied too and
+// never read.  CG: through L2 only (rows written by this kernel).
+template <bool CG>
+__device__ __forceinline__ void warp_copy_rows(const int32_t* gid, const float* gpr, int64_t gs, int nrows, int width,
+                                               int32_t* sid, float* spr, int ss, int lane) {
+    constexpr int RB = 8;
+    const int total = nrows * width;
+    for (int b0 = 0; b0 < total; b0 += 32 * RB) {
+        int32_t vi[RB];
+        float vp[RB];
+#pragma unroll
+        for (int t = 0; t < RB; ++t) {
+            const int idx = b0 + t * 32 + lane;
+            if (idx < total) {
+                const int i = idx / width, j = idx - i * width;
+                const size_t g = (size_t)i * (size_t)gs + (size_t)j;
+                vi[t] = CG ? __ldcg(gid + g) : __ldg(gid + g);
+                vp[t] = CG ? __ldcg(gpr + g) : __ldg(gpr + g);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < RB; ++t) {
+            const int idx = b0 + t * 32 + lane;
+            if (idx < total) {
+                const int i = idx / width, j = idx - i * width;
+                sid[i * ss + j] = vi[t];
+                spr[i * ss + j] = vp[t];
+            }
+        }
+    }
+}
+
+// Two row sets at once (p: np entries, q: nq entries), in one stream of
+// loads: every load of a batch is issued before any store.
+__device__ __forceinline__ void warp_copy_two(const int32_t* gpi, const float* gpp, int64_t pgs, int pw, int np,
+                                              int32_t* spi, float* spp, int pss, const int32_t* gqi, const float* gqp,
+                                              int64_t qgs, int qw, int nq, int32_t* sqi, float* sqp, int qss,
+                                              int lane) {
+    constexpr int RB = 16;
+    const int total = np > nq ? np : nq;
+    for (int b0 = 0; b0 < total; b0 += 32 * RB) {
+        int32_t ai[RB], bi[RB];
+        float ap[RB], bp[RB];
+#pragma unroll
+        for (int t = 0; t < RB; ++t) {
+            const int idx = b0 + t * 32 + lane;
+            if (idx < np) {
+                const int i = idx / pw, j = idx - i * pw;
+                ai[t] = __ldcg(gpi + (size_t)i * (size_t)pgs + j);
+                ap[t] = __ldcg(gpp + (size_t)i * (size_t)pgs + j);
+            }
+            if (idx < nq) {
+                const int i = idx / qw, j = idx - i * qw;
+                bi[t] = __ldg(gqi + (size_t)i * (size_t)qgs + j);
+                bp[t] = __ldg(gqp + (size_t)i * (size_t)qgs + j);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < RB; ++t) {
+            const int idx = b0 + t * 32 + lane;
+            if (idx < np) {
+                const int i = idx / pw, j = idx - i * pw;
+                spi[i * pss + j] = ai[t];
+                spp[i * pss + j] = ap[t];
+            }
+            if (idx < nq) {
+                const int i = idx / qw, j = idx - i * qw;
+                sqi[i * qss + j] = bi[t];
+                sqp[i * qss + j] = bp[t];
+            }
+        }
+    }
+}
+
 __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsigned char* sm, int lane) {
     const int32_t B = J.B;
     const int kc = J.k;
     constexpr int QS = 64;  // q entries kept per row
-    if (kc > 64) return false;
+    if (kc > 64 || B > 31) return false;
     const size_t need = (size_t)(B + 1) * kc * 8 + (size_t)B * QS * 8 + (size_t)(4 * B + 2) * 4;
     if (need > (size_t)J.tail_bytes) return false;
     int32_t* pid = reinterpret_cast<int32_t*>(sm);           // [B+1][kc]
@@ -934,47 +1013,48 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     int32_t* dft = qcnt + B;                                    // [B]
     int32_t* otok = dft + B;                                    // [B+1] emitted tokens
     const int64_t base = (int64_t)r * (B + 1);
-    uint32_t flags = 0;
-    bool qbig = false;
-    for (int i = lane; i <= B; i += 32) {
-        pcnt[i] = __ldcg(J.c_count + base + i);
-        flags |= __ldcg(J.c_flags + base + i);
+    const uint32_t req = J.first_request + (uint32_t)r;
+    // Every global load of the tail goes out at once: under a saturated
+    // memory system each round trip costs microseconds.  Counts, flags and
+    // drafts first (registers), then the rows (staged), then the stores.
+    int pc_l = 0, qc_l = 0, d_l = 0;
+    uint32_t f_l = 0;
+    if (lane <= B) {
+        pc_l = __ldcg(J.c_count + base + lane);
+        f_l = __ldcg(J.c_flags + base + lane);
     }
-    for (int i = lane; i < B; i += 32) {
-        int qc = J.q_count[(int64_t)r * B + i];
-        qc = qc < 0 ? 0 : (qc > J.q_cap ? J.q_cap : qc);
-        qbig |= qc > QS;
-        qcnt[i] = qc;
-        dft[i] = J.draft_ids[(size_t)r * B + i];
+    if (lane < B) {
+        qc_l = J.q_count[(int64_t)r * B + lane];
+        d_l = J.draft_ids[(size_t)r * B + lane];
     }
-    for (int i = lane; i <= B; i += 32) otok[i] = -1;
-    flags = __reduce_or_sync(kFull, flags);
-    if (__any_sync(kFull, qbig)) return false;
-    __syncwarp();
-    // every row at once: the loads are independent, so they overlap
-#pragma unroll 4
-    for (int idx = lane; idx < (B + 1) * kc; idx += 32) {
-        const int i = idx / kc, j = idx - i * kc;
-        if (j < pcnt[i]) {
-            pid[idx] = __ldcg(J.c_ids + (size_t)(base + i) * kc + j);
-            ppr[idx] = __ldcg(J.c_probs + (size_t)(base + i) * kc + j);
-        }
+    const int qw = J.q_cap < QS ? J.q_cap : QS;
+    warp_copy_two(J.c_ids + (size_t)base * kc, J.c_probs + (size_t)base * kc, kc, kc, (B + 1) * kc, pid, ppr, kc,
+                  J.q_ids + (size_t)r * B * J.q_cap, J.q_probs + (size_t)r * B * J.q_cap, J.q_cap, qw, B * qw, qid, qpr,
+                  QS, lane);
+    // the decisions' uniforms, one position per lane
+    double ua = 0.0, ur = 0.0;
+    if (lane < B) {
+        ua = uniform53(J.seed, req, (uint32_t)lane, kDrawAccept, J.cycle);
+        ur = uniform53(J.seed, req, (uint32_t)lane, kDrawResidual, J.cycle);
+    } else if (lane == B) {
+        ur = uniform53(J.seed, req, (uint32_t)B, kDrawTarget, J.cycle);
     }
-    const int64_t qbase = (int64_t)r * B;
-#pragma unroll 4
-    for (int idx = lane; idx < B * QS; idx += 32) {
-        const int i = idx / QS, j = idx % QS;
-        if (j < qcnt[i]) {
-            qid[idx] = J.q_ids[(size_t)(qbase + i) * J.q_cap + j];
-            qpr[idx] = J.q_probs[(size_t)(qbase + i) * J.q_cap + j];
-        }
+    qc_l = qc_l < 0 ? 0 : (qc_l > J.q_cap ? J.q_cap : qc_l);
+    if (__any_sync(kFull, lane < B && qc_l > QS)) return false;
+    uint32_t flags = __reduce_or_sync(kFull, f_l);
+    if (lane <= B) {
+        pcnt[lane] = pc_l;
+        otok[lane] = -1;
+    }
+    if (lane < B) {
+        qcnt[lane] = qc_l;
+        dft[lane] = d_l;
     }
     __syncwarp();
 
     int32_t* toks = J.out_tokens + (size_t)r * (B + 1);
     int32_t acc = B, ntok = B + 1;
     bool stopped = false;
-    const uint32_t req = J.first_request + (uint32_t)r;
     for (int i = 0; i < B && !stopped; ++i) {
         const int pc = pcnt[i];
         if (pc == 0) {  // a non-finite target row was reached
@@ -993,7 +1073,7 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
         const double px = xin ? warp_lookup(pi, pp, pc, x, lane) : 0.0;
         bool accept = false;
         if (a > 0.0) {
-            const double u = uniform53(J.seed, req, (uint32_t)i, kDrawAccept, J.cycle);
+            const double u = __shfl_sync(kFull, ua, i);
             accept = (u * a < px);
         } else {
             flags |= kFlagDraftNotInSupport;
@@ -1014,7 +1094,7 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
             const double d = pb - smem_lookup(qi, qp, qcnt[i], pi[lane + 32]);
             rb = d > 0.0 ? d : 0.0;
         }
-        const double u = uniform53(J.seed, req, (uint32_t)i, kDrawResidual, J.cycle);
+        const double u = __shfl_sync(kFull, ur, i);
         int pick = warp_inv_cdf(ra, rb, u, lane);
         if (pick < 0) {  // the residual is empty: draw from p_i
             flags |= kFlagResidualEmpty;
@@ -1032,7 +1112,7 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
         } else {
             const float* pp = ppr + B * kc;
             const double wa = lane < pc ? (double)pp[lane] : 0.0, wb = lane + 32 < pc ? (double)pp[lane + 32] : 0.0;
-            const double u = uniform53(J.seed, req, (uint32_t)B, kDrawTarget, J.cycle);
+            const double u = __shfl_sync(kFull, ur, B);
             const int pick = warp_inv_cdf(wa, wb, u, lane);
             if (lane == 0) otok[B] = pick >= 0 ? pid[B * kc + pick] : -1;
         }
@@ -1076,14 +1156,7 @@ __device__ __noinline__ bool tree_tail_fast(const RowJob& J, int32_t r, unsigned
     }
     flags = __reduce_or_sync(kFull, flags);
     __syncwarp();
-#pragma unroll 4
-    for (int idx = lane; idx < n * kc; idx += 32) {
-        const int j = idx / kc, e = idx - j * kc;
-        if (e < ncnt[j]) {
-            nid[idx] = __ldcg(J.c_ids + (size_t)(base + j) * kc + e);
-            npr[idx] = __ldcg(J.c_probs + (size_t)(base + j) * kc + e);
-        }
-    }
+    warp_copy_rows<true>(J.c_ids + (size_t)base * kc, J.c_probs + (size_t)base * kc, kc, n, kc, nid, npr, kc, lane);
     __syncwarp();
     int32_t* toks = J.out_tokens + (size_t)r * (B + 1);
     int32_t* path = J.out_path_nodes + (size_t)r * (B + 1);
@@ -1289,7 +1362,7 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
             J.c_count[row] = kept;
             J.c_flags[row] = rflags;
         }
-        request_arrive<MODE>(J, req, wd, tail_smem, lane);
+        if (!J.defer_tails) request_arrive<MODE>(J, req, wd, tail_smem, lane);
     }
 }
 
@@ -1605,14 +1678,15 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const RowJob J) {
 //
 //   warp 0      producer: lane 0 keeps a ring of `nst` 16 KB stages filled
 //               with bulk copies (TMA, no multicast), running across item
-//               boundaries, each stage tracked by a `full` mbarrier and
-//               given back through an `empty` mbarrier;
+//               boundaries, each stage tracked by a `full` mbarrier, a fill
+//               tag and an `empty` mbarrier;
 //   warps 1..8  consumers: per item, a threshold seed from the lane maxima
-//               of the first stages (read twice from shared memory), then
-//               the threshold filter of every stage into per-warp candidate
-//               buffers of the item's slot;
-//   warps 9..12 finishers: finisher f takes the items whose ordinal in the
-//               CTA's list is f mod 4 from slot f -- exact top-k of the
+//               of the first eight stages (every warp reads a slice of
+//               each), then each warp filters the stages it owns (stage st
+//               of the item goes to warp st % 8) into its candidate buffer
+//               of the item's slot;
+//   warps 9..10 finishers: finisher f takes the items whose ordinal in the
+//               CTA's list is f mod 2 from slot f -- exact top-k of the
 //               slot's candidates with a warp bitonic merge, then the
 //               softmax / top-p / output / request-tail work of the row.
 //
@@ -1623,7 +1697,7 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const RowJob J) {
 // with UNO_FLAG_TIMEOUT.
 // ---------------------------------------------------------------------------
 constexpr int kPipeConsumers = 8;
-constexpr int kPipeFinishers = 4;
+constexpr int kPipeFinishers = 2;
 constexpr int kPipeSlots = kPipeFinishers;
 constexpr int kPipeWarps = 1 + kPipeConsumers + kPipeFinishers;
 constexpr int kPipeThreads = 32 * kPipeWarps;
@@ -2172,10 +2246,7 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
         const int64_t row = it / J.S;
         const int seg = (int)(it % J.S);
         const int32_t req = (int32_t)(row / J.rpr);
-        if (!item_active<MODE>(J, row)) {
-            if (MODE != kModeFilter && seg == 0) request_arrive<MODE>(J, req, wd, tail, lane);
-            continue;
-        }
+        if (!item_active<MODE>(J, row)) continue;  // nothing to filter (the tails run afterwards)
         uint32_t rowbad = 2u;
         int n = 0;
         const bool ok = pipe_wait_warp(&P.slot_full[slot], use & 1u, P);
@@ -2270,6 +2341,24 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const RowJob J) {
         const int f = warp - 1 - kPipeConsumers;
         pipe_finish<T, MODE>(J, P, slots, fin + (size_t)f * J.fin_stride, f, lane);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Request tails after the pipelined kernel: one warp per request, with its
+// own shared-memory scratch.  Run on their own, the tails' reads of the
+// compact rows hit L2 without queueing behind streaming copies.
+// ---------------------------------------------------------------------------
+constexpr int kTailWarps = 4;
+
+template <int MODE>
+__global__ void __launch_bounds__(32 * kTailWarps) tail_kernel(const RowJob J, int64_t nreq) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * kTailWarps + warp;
+    if (r >= nreq) return;
+    unsigned char* mine = smem + (size_t)warp * J.fin_stride;
+    double* wd = reinterpret_cast<double*>(mine);  // [k] (the global-memory path)
+    request_tail<MODE>(J, (int32_t)r, wd, mine + (size_t)kPipeMaxK * 8, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -2561,15 +2650,13 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
         const size_t fixed = slot_bytes + (size_t)kPipeFinishers * stride_of(tb);
         return fixed >= dyn_max ? 0 : (int64_t)((dyn_max - fixed) / kPStageBytes);
     };
-    // request rows in shared memory unless that leaves too shallow a ring
-    // (the tails then read them from global memory)
-    if (tail > 0 && stages_of(tail) < kPipeMinStages) tail = 0;
-    int64_t nst = stages_of(tail);
+    int64_t nst = stages_of(0);  // the request tails run in their own kernel
     if (nst > kPipeMaxStages) nst = kPipeMaxStages;
     if (nst < kPipeMinStages) return UNO_ERR_UNSUPPORTED;
     J.nst = (int32_t)nst;
-    J.tail_bytes = (int32_t)tail;
-    J.fin_stride = (int32_t)stride_of(tail);
+    J.tail_bytes = 0;
+    J.fin_stride = (int32_t)stride_of(0);
+    J.defer_tails = 1;
     const size_t dyn = (size_t)nst * kPStageBytes + slot_bytes + (size_t)kPipeFinishers * J.fin_stride;
     auto kern = pipe_kernel<T, MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
@@ -2578,6 +2665,19 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     const int64_t grid = items < G ? items : G;
     if (grid <= 0) return UNO_OK;
     kern<<<(unsigned)grid, kPipeThreads, dyn, stream>>>(J);
+    if (cudaGetLastError() != cudaSuccess) return UNO_ERR_CUDA;
+    if (MODE == kModeFilter) return UNO_OK;
+    // the request tails: shared-memory rows when they fit in 48 KB a warp
+    RowJob TJ = J;
+    TJ.tail_bytes = tail <= 48 * 1024 ? (int32_t)tail : 0;
+    TJ.fin_stride = (int32_t)align_up((size_t)kPipeMaxK * 8 + (size_t)TJ.tail_bytes, 128);
+    const int64_t nreq = J.rows / J.rpr;
+    const size_t tsm = (size_t)kTailWarps * TJ.fin_stride;
+    auto tkern = tail_kernel<MODE>;
+    if (tsm > 48 * 1024 &&
+        cudaFuncSetAttribute(tkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm) != cudaSuccess)
+        return UNO_ERR_CUDA;
+    tkern<<<(unsigned)((nreq + kTailWarps - 1) / kTailWarps), 32 * kTailWarps, tsm, stream>>>(TJ, nreq);
     return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
 }
 
