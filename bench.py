@@ -60,12 +60,20 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
-def init_dist(world):
+def init_dist(world, backend="nccl"):
     import torch.distributed as dist
     if world > 1 and not dist.is_initialized():
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return dist
+
+
+def shard(rank, per_rank):
+    """This rank's requests: per_rank consecutive global indices.  The global
+    index is also the request word of the random-number counter, so a rank's
+    draws equal those of the same requests in one big batch."""
+    first = rank * per_rank
+    return first, range(first, first + per_rank)
 
 
 def max_over_ranks(values, world, device):
@@ -258,8 +266,7 @@ def run_ours(args, w):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     lib = b.load_library()
-    first = rank * w.R
-    reqs = range(first, first + w.R)
+    first, reqs = shard(rank, w.R)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
 
     def dev(a):

@@ -67,8 +67,9 @@ struct RowJob {
     uint64_t* part_keys;   // [rows*S][k]
     int32_t* part_count;   // [rows*S]
     uint32_t* part_flags;  // [rows*S]
-    int32_t* c_ids;        // [rows][k]   compact target rows (verifiers)
-    float* c_probs;        // [rows][k]
+    int32_t* c_ids;        // [rows][ks]  compact target rows (verifiers)
+    float* c_probs;        // [rows][ks]
+    int32_t ks;            // their row stride: k rounded up to a multiple of 4 (16-byte rows)
     int32_t* c_count;      // [rows]
     uint32_t* c_flags;     // [rows]
     // linear verification
@@ -678,7 +679,6 @@ __device__ __forceinline__ double lookup_sorted(const int32_t* ids, const float*
 __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd, int lane) {
     const int32_t B = J.B;
     const int64_t base = (int64_t)r * (B + 1);
-    const int kc = J.k;
     uint32_t flags = 0;
     for (int i = lane; i <= B; i += 32) flags |= __ldcg(J.c_flags + base + i);
     flags = __reduce_or_sync(kFull, flags);
@@ -689,8 +689,8 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
     bool stopped = false;
     for (int i = 0; i < B && !stopped; ++i) {
         const int pc = __ldcg(J.c_count + base + i);
-        const int32_t* pid = J.c_ids + (size_t)(base + i) * kc;
-        const float* ppr = J.c_probs + (size_t)(base + i) * kc;
+        const int32_t* pid = J.c_ids + (size_t)(base + i) * J.ks;
+        const float* ppr = J.c_probs + (size_t)(base + i) * J.ks;
         if (pc == 0) {
             acc = i;
             ntok = i;
@@ -746,8 +746,8 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
         if (pc == 0) {
             ntok = B;
         } else if (lane == 0) {
-            const int32_t* pid = J.c_ids + (size_t)(base + B) * kc;
-            const float* ppr = J.c_probs + (size_t)(base + B) * kc;
+            const int32_t* pid = J.c_ids + (size_t)(base + B) * J.ks;
+            const float* ppr = J.c_probs + (size_t)(base + B) * J.ks;
             for (int j = 0; j < pc; ++j) wd[j] = (double)__ldcg(ppr + j);
             const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)B, kDrawTarget, J.cycle);
             const int pick = inv_cdf_serial(wd, pc, u);
@@ -764,7 +764,6 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
 __device__ __noinline__ void tree_tail(const RowJob& J, int32_t r, double* wd, int lane) {
     const int32_t B = J.B, V = J.V;
     const int64_t base = (int64_t)r * V;
-    const int kc = J.k;
     int32_t n = J.num_nodes[r];
     n = n < 1 ? 1 : (n > V ? V : n);
     const int32_t* tk = J.node_token + (size_t)r * V;
@@ -790,8 +789,8 @@ __device__ __noinline__ void tree_tail(const RowJob& J, int32_t r, double* wd, i
         }
         int32_t y = -1;
         if (lane == 0) {
-            const int32_t* pid = J.c_ids + (size_t)(base + j) * kc;
-            const float* ppr = J.c_probs + (size_t)(base + j) * kc;
+            const int32_t* pid = J.c_ids + (size_t)(base + j) * J.ks;
+            const float* ppr = J.c_probs + (size_t)(base + j) * J.ks;
             for (int q = 0; q < pc; ++q) wd[q] = (double)__ldcg(ppr + q);
             const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)j, kDrawTarget, J.cycle);
             const int pick = inv_cdf_serial(wd, pc, u);
@@ -955,68 +954,72 @@ __device__ __forceinline__ void warp_copy_rows(const int32_t* gid, const float* 
     }
 }
 
-// Two row sets at once (p: np entries, q: nq entries), in one stream of
-// loads: every load of a batch is issued before any store.
-__device__ __forceinline__ void warp_copy_two(const int32_t* gpi, const float* gpp, int64_t pgs, int pw, int np,
-                                              int32_t* spi, float* spp, int pss, const int32_t* gqi, const float* gqp,
-                                              int64_t qgs, int qw, int nq, int32_t* sqi, float* sqp, int qss,
-                                              int lane) {
-    constexpr int RB = 16;
-    const int total = np > nq ? np : nq;
-    for (int b0 = 0; b0 < total; b0 += 32 * RB) {
-        int32_t ai[RB], bi[RB];
-        float ap[RB], bp[RB];
-#pragma unroll
-        for (int t = 0; t < RB; ++t) {
-            const int idx = b0 + t * 32 + lane;
-            if (idx < np) {
-                const int i = idx / pw, j = idx - i * pw;
-                ai[t] = __ldcg(gpi + (size_t)i * (size_t)pgs + j);
-                ap[t] = __ldcg(gpp + (size_t)i * (size_t)pgs + j);
-            }
-            if (idx < nq) {
-                const int i = idx / qw, j = idx - i * qw;
-                bi[t] = __ldg(gqi + (size_t)i * (size_t)qgs + j);
-                bp[t] = __ldg(gqp + (size_t)i * (size_t)qgs + j);
-            }
-        }
-#pragma unroll
-        for (int t = 0; t < RB; ++t) {
-            const int idx = b0 + t * 32 + lane;
-            if (idx < np) {
-                const int i = idx / pw, j = idx - i * pw;
-                spi[i * pss + j] = ai[t];
-                spp[i * pss + j] = ap[t];
-            }
-            if (idx < nq) {
-                const int i = idx / qw, j = idx - i * qw;
-                sqi[i * qss + j] = bi[t];
-                sqp[i * qss + j] = bp[t];
-            }
-        }
+__device__ __forceinline__ void mbar_inval(uint64_t* bar) {
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Whole warp: bounded wait for a tail's bulk copies (phase 0 of bar).  Every
+// lane waits on the barrier itself, so that every lane sees the copied data.
+// On expiry a second bounded wait lets copies in flight land first.
+__device__ __forceinline__ bool tail_copies_wait(uint64_t* bar, int lane) {
+    bool got = mbar_try_wait(bar, 0) || mbar_wait_bounded(bar, 0);
+    const bool ok = __all_sync(kFull, got);
+    if (!ok && !got) (void)mbar_wait_bounded(bar, 0);
+    __syncwarp();
+    if (ok && lane == 0) mbar_inval(bar);
+    return ok;
+}
+
+// A request's outputs when its tail could not get its rows in time.
+__device__ __forceinline__ void tail_timeout(const RowJob& J, int32_t r, int lane) {
+    int32_t* toks = J.out_tokens + (size_t)r * (J.B + 1);
+    for (int t = lane; t <= J.B; t += 32) toks[t] = -1;
+    if (J.out_path_nodes != nullptr)
+        for (int t = lane; t <= J.B; t += 32) J.out_path_nodes[(size_t)r * (J.B + 1) + t] = -1;
+    if (lane == 0) {
+        J.out_accept_len[r] = 0;
+        J.out_num_tokens[r] = 0;
+        J.out_req_flags[r] = kFlagTimeout;
     }
 }
 
 __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsigned char* sm, int lane) {
     const int32_t B = J.B;
-    const int kc = J.k;
+    const int kc = J.k, ks = J.ks;
     constexpr int QS = 64;  // q entries kept per row
     if (kc > 64 || B > 31) return false;
-    const size_t need = (size_t)(B + 1) * kc * 8 + (size_t)B * QS * 8 + (size_t)(4 * B + 2) * 4;
+    const size_t need = 16 + (size_t)(B + 1) * ks * 8 + (size_t)B * QS * 8 + (size_t)(4 * B + 2) * 4;
     if (need > (size_t)J.tail_bytes) return false;
-    int32_t* pid = reinterpret_cast<int32_t*>(sm);           // [B+1][kc]
-    float* ppr = reinterpret_cast<float*>(pid + (B + 1) * kc);  // [B+1][kc]
-    int32_t* qid = reinterpret_cast<int32_t*>(ppr + (B + 1) * kc);  // [B][QS]
-    float* qpr = reinterpret_cast<float*>(qid + B * QS);        // [B][QS]
-    int32_t* pcnt = reinterpret_cast<int32_t*>(qpr + B * QS);  // [B+1]
-    int32_t* qcnt = pcnt + (B + 1);                             // [B]
-    int32_t* dft = qcnt + B;                                    // [B]
-    int32_t* otok = dft + B;                                    // [B+1] emitted tokens
+    // q rows come in one bulk copy when the caller's layout allows it
+    const bool qbulk = (reinterpret_cast<uintptr_t>(J.q_ids) & 15u) == 0 &&
+                       (reinterpret_cast<uintptr_t>(J.q_probs) & 15u) == 0 && (J.q_cap & 3) == 0 && J.q_cap <= QS;
+    const int qs = qbulk ? J.q_cap : QS;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm);                         // the copies' mbarrier
+    int32_t* pid = reinterpret_cast<int32_t*>(sm + 16);                      // [B+1][ks]
+    float* ppr = reinterpret_cast<float*>(pid + (B + 1) * ks);               // [B+1][ks]
+    int32_t* qid = reinterpret_cast<int32_t*>(ppr + (B + 1) * ks);           // [B][qs]
+    float* qpr = reinterpret_cast<float*>(qid + B * qs);                     // [B][qs]
+    int32_t* pcnt = reinterpret_cast<int32_t*>(qpr + B * qs);                // [B+1]
+    int32_t* qcnt = pcnt + (B + 1);                                          // [B]
+    int32_t* dft = qcnt + B;                                                 // [B]
+    int32_t* otok = dft + B;                                                 // [B+1] emitted tokens
     const int64_t base = (int64_t)r * (B + 1);
     const uint32_t req = J.first_request + (uint32_t)r;
-    // Every global load of the tail goes out at once: under a saturated
-    // memory system each round trip costs microseconds.  Counts, flags and
-    // drafts first (registers), then the rows (staged), then the stores.
+    // The request's compact target rows (and q rows) arrive by bulk copies
+    // (TMA) on one mbarrier: one round trip, whatever the memory system's
+    // queueing; counts, flags and drafts load alongside.
+    if (lane == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        const uint32_t pb = (uint32_t)((B + 1) * ks * 4), qb = qbulk ? (uint32_t)(B * qs * 4) : 0u;
+        mbar_expect_tx(bar, 2 * pb + 2 * qb);
+        bulk_g2s(pid, J.c_ids + (size_t)base * ks, pb, bar);
+        bulk_g2s(ppr, J.c_probs + (size_t)base * ks, pb, bar);
+        if (qbulk) {
+            bulk_g2s(qid, J.q_ids + (size_t)r * B * J.q_cap, qb, bar);
+            bulk_g2s(qpr, J.q_probs + (size_t)r * B * J.q_cap, qb, bar);
+        }
+    }
     int pc_l = 0, qc_l = 0, d_l = 0;
     uint32_t f_l = 0;
     if (lane <= B) {
@@ -1027,10 +1030,11 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
         qc_l = J.q_count[(int64_t)r * B + lane];
         d_l = J.draft_ids[(size_t)r * B + lane];
     }
-    const int qw = J.q_cap < QS ? J.q_cap : QS;
-    warp_copy_two(J.c_ids + (size_t)base * kc, J.c_probs + (size_t)base * kc, kc, kc, (B + 1) * kc, pid, ppr, kc,
-                  J.q_ids + (size_t)r * B * J.q_cap, J.q_probs + (size_t)r * B * J.q_cap, J.q_cap, qw, B * qw, qid, qpr,
-                  QS, lane);
+    if (!qbulk) {
+        const int qw = J.q_cap < QS ? J.q_cap : QS;
+        warp_copy_rows<false>(J.q_ids + (size_t)r * B * J.q_cap, J.q_probs + (size_t)r * B * J.q_cap, J.q_cap, B, qw,
+                              qid, qpr, QS, lane);
+    }
     // the decisions' uniforms, one position per lane
     double ua = 0.0, ur = 0.0;
     if (lane < B) {
@@ -1038,6 +1042,11 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
         ur = uniform53(J.seed, req, (uint32_t)lane, kDrawResidual, J.cycle);
     } else if (lane == B) {
         ur = uniform53(J.seed, req, (uint32_t)B, kDrawTarget, J.cycle);
+    }
+    const bool copied = tail_copies_wait(bar, lane);
+    if (!copied) {
+        tail_timeout(J, r, lane);
+        return true;
     }
     qc_l = qc_l < 0 ? 0 : (qc_l > J.q_cap ? J.q_cap : qc_l);
     if (__any_sync(kFull, lane < B && qc_l > QS)) return false;
@@ -1053,68 +1062,70 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     __syncwarp();
 
     int32_t* toks = J.out_tokens + (size_t)r * (B + 1);
-    int32_t acc = B, ntok = B + 1;
-    bool stopped = false;
-    for (int i = 0; i < B && !stopped; ++i) {
-        const int pc = pcnt[i];
-        if (pc == 0) {  // a non-finite target row was reached
-            acc = i;
-            ntok = i;
-            stopped = true;
-            break;
-        }
-        const int32_t* pi = pid + i * kc;
-        const float* pp = ppr + i * kc;
-        const int32_t* qi = qid + i * QS;
-        const float* qp = qpr + i * QS;
-        const int32_t x = dft[i];
-        const bool xin = x >= 0 && (int64_t)x < J.vocab;
-        const double a = xin ? warp_lookup(qi, qp, qcnt[i], x, lane) : 0.0;
-        const double px = xin ? warp_lookup(pi, pp, pc, x, lane) : 0.0;
-        bool accept = false;
-        if (a > 0.0) {
-            const double u = __shfl_sync(kFull, ua, i);
-            accept = (u * a < px);
+    // Every position's accept test at once (lane i: position i).  The walk
+    // stops at the first position whose target row is empty or whose draft
+    // is rejected; the positions before it are accepted, so deciding them
+    // all in parallel and taking the first stop gives the sequential result.
+    bool stop_i = false, empty_i = false, notin_i = false;
+    int32_t x_i = -1;
+    if (lane < B) {
+        const int pc = pcnt[lane];
+        x_i = dft[lane];
+        if (pc == 0) {
+            stop_i = empty_i = true;  // a non-finite target row
         } else {
-            flags |= kFlagDraftNotInSupport;
+            const bool xin = x_i >= 0 && (int64_t)x_i < J.vocab;
+            const double a = xin ? smem_lookup(qid + lane * qs, qpr + lane * qs, qcnt[lane], x_i) : 0.0;
+            const double px = xin ? smem_lookup(pid + lane * ks, ppr + lane * ks, pc, x_i) : 0.0;
+            notin_i = !(a > 0.0);
+            stop_i = notin_i || !(ua * a < px);
         }
-        if (accept) {
-            if (lane == 0) otok[i] = x;
-            continue;
-        }
-        // residual max(0, p_i - q_i) over supp p_i, ascending ids
-        double ra = 0.0, rb = 0.0, pa = 0.0, pb = 0.0;
-        if (lane < pc) {
-            pa = (double)pp[lane];
-            const double d = pa - smem_lookup(qi, qp, qcnt[i], pi[lane]);
-            ra = d > 0.0 ? d : 0.0;
-        }
-        if (lane + 32 < pc) {
-            pb = (double)pp[lane + 32];
-            const double d = pb - smem_lookup(qi, qp, qcnt[i], pi[lane + 32]);
-            rb = d > 0.0 ? d : 0.0;
-        }
-        const double u = __shfl_sync(kFull, ur, i);
-        int pick = warp_inv_cdf(ra, rb, u, lane);
-        if (pick < 0) {  // the residual is empty: draw from p_i
-            flags |= kFlagResidualEmpty;
-            pick = warp_inv_cdf(pa, pb, u, lane);
-        }
-        if (lane == 0) otok[i] = pick >= 0 ? pi[pick] : -1;
-        acc = i;
-        ntok = i + 1;
-        stopped = true;
     }
-    if (!stopped) {
+    const unsigned stops = __ballot_sync(kFull, stop_i);
+    const int istop = stops ? __ffs(stops) - 1 : B;  // first stopping position (B: none)
+    if (lane < istop) otok[lane] = x_i;             // accepted drafts
+    int32_t acc = B, ntok = B + 1;
+    if (istop < B) {
+        const bool empty = __shfl_sync(kFull, empty_i, istop);
+        acc = istop;
+        ntok = empty ? istop : istop + 1;
+        if (!empty) {
+            if (__shfl_sync(kFull, notin_i, istop)) flags |= kFlagDraftNotInSupport;
+            // residual max(0, p_i - q_i) over supp p_i, ascending ids
+            const int i = istop, pc = pcnt[i];
+            const int32_t* pi = pid + i * ks;
+            const float* pp = ppr + i * ks;
+            const int32_t* qi = qid + i * qs;
+            const float* qp = qpr + i * qs;
+            double ra = 0.0, rb = 0.0, pa = 0.0, pb = 0.0;
+            if (lane < pc) {
+                pa = (double)pp[lane];
+                const double d = pa - smem_lookup(qi, qp, qcnt[i], pi[lane]);
+                ra = d > 0.0 ? d : 0.0;
+            }
+            if (lane + 32 < pc) {
+                pb = (double)pp[lane + 32];
+                const double d = pb - smem_lookup(qi, qp, qcnt[i], pi[lane + 32]);
+                rb = d > 0.0 ? d : 0.0;
+            }
+            const double u = __shfl_sync(kFull, ur, i);
+            int pick = warp_inv_cdf(ra, rb, u, lane);
+            if (pick < 0) {  // the residual is empty: draw from p_i
+                flags |= kFlagResidualEmpty;
+                pick = warp_inv_cdf(pa, pb, u, lane);
+            }
+            if (lane == 0) otok[i] = pick >= 0 ? pi[pick] : -1;
+        }
+    } else {
         const int pc = pcnt[B];
         if (pc == 0) {
             ntok = B;
         } else {
-            const float* pp = ppr + B * kc;
+            const float* pp = ppr + B * ks;
             const double wa = lane < pc ? (double)pp[lane] : 0.0, wb = lane + 32 < pc ? (double)pp[lane + 32] : 0.0;
             const double u = __shfl_sync(kFull, ur, B);
             const int pick = warp_inv_cdf(wa, wb, u, lane);
-            if (lane == 0) otok[B] = pick >= 0 ? pid[B * kc + pick] : -1;
+            if (lane == 0) otok[B] = pick >= 0 ? pid[B * ks + pick] : -1;
         }
     }
     __syncwarp();
@@ -1129,20 +1140,30 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
 
 __device__ __noinline__ bool tree_tail_fast(const RowJob& J, int32_t r, unsigned char* sm, int lane) {
     const int32_t B = J.B, V = J.V;
-    const int kc = J.k;
+    const int kc = J.k, ks = J.ks;
     if (kc > 64) return false;
     int32_t n = J.num_nodes[r];
     n = n < 1 ? 1 : (n > V ? V : n);
-    const size_t need = (size_t)n * kc * 8 + (size_t)n * 12 + (size_t)(B + 1) * 8;
+    const size_t need = 16 + (size_t)n * ks * 8 + (size_t)n * 12 + (size_t)(B + 1) * 8;
     if (need > (size_t)J.tail_bytes) return false;
-    int32_t* nid = reinterpret_cast<int32_t*>(sm);        // [n][kc]
-    float* npr = reinterpret_cast<float*>(nid + n * kc);  // [n][kc]
-    int32_t* ncnt = reinterpret_cast<int32_t*>(npr + n * kc);  // [n]
-    int32_t* tk = ncnt + n;                               // [n]
-    int32_t* pa = tk + n;                                 // [n]
-    int32_t* otok = pa + n;                               // [B+1] emitted tokens
-    int32_t* opath = otok + (B + 1);                      // [B+1] nodes that drew them
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm);           // the copies' mbarrier
+    int32_t* nid = reinterpret_cast<int32_t*>(sm + 16);        // [n][ks]
+    float* npr = reinterpret_cast<float*>(nid + n * ks);       // [n][ks]
+    int32_t* ncnt = reinterpret_cast<int32_t*>(npr + n * ks);  // [n]
+    int32_t* tk = ncnt + n;                                    // [n]
+    int32_t* pa = tk + n;                                      // [n]
+    int32_t* otok = pa + n;                                    // [B+1] emitted tokens
+    int32_t* opath = otok + (B + 1);                           // [B+1] nodes that drew them
     const int64_t base = (int64_t)r * V;
+    // the nodes' compact target rows by bulk copies (one round trip)
+    if (lane == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        const uint32_t nb = (uint32_t)(n * ks * 4);
+        mbar_expect_tx(bar, 2 * nb);
+        bulk_g2s(nid, J.c_ids + (size_t)base * ks, nb, bar);
+        bulk_g2s(npr, J.c_probs + (size_t)base * ks, nb, bar);
+    }
     uint32_t flags = 0;
     for (int j = lane; j < n; j += 32) {
         ncnt[j] = __ldcg(J.c_count + base + j);
@@ -1155,9 +1176,10 @@ __device__ __noinline__ bool tree_tail_fast(const RowJob& J, int32_t r, unsigned
         opath[q] = -1;
     }
     flags = __reduce_or_sync(kFull, flags);
-    __syncwarp();
-    warp_copy_rows<true>(J.c_ids + (size_t)base * kc, J.c_probs + (size_t)base * kc, kc, n, kc, nid, npr, kc, lane);
-    __syncwarp();
+    if (!tail_copies_wait(bar, lane)) {
+        tail_timeout(J, r, lane);
+        return true;
+    }
     int32_t* toks = J.out_tokens + (size_t)r * (B + 1);
     int32_t* path = J.out_path_nodes + (size_t)r * (B + 1);
     const uint32_t req = J.first_request + (uint32_t)r;
@@ -1170,11 +1192,11 @@ __device__ __noinline__ bool tree_tail_fast(const RowJob& J, int32_t r, unsigned
             acc = t;
             break;
         }
-        const float* pp = npr + j * kc;
+        const float* pp = npr + j * ks;
         const double wa = lane < pc ? (double)pp[lane] : 0.0, wb = lane + 32 < pc ? (double)pp[lane + 32] : 0.0;
         const double u = uniform53(J.seed, req, (uint32_t)j, kDrawTarget, J.cycle);
         const int pick = warp_inv_cdf(wa, wb, u, lane);
-        const int32_t y = pick >= 0 ? nid[j * kc + pick] : -1;
+        const int32_t y = pick >= 0 ? nid[j * ks + pick] : -1;
         if (lane == 0) {
             otok[t] = y;
             opath[t] = j;
@@ -1348,8 +1370,8 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
             if (J.has_rng) J.out_sample[row] = tok;
         }
     } else {
-        int32_t* ids = J.c_ids + (size_t)row * J.k;
-        float* pr = J.c_probs + (size_t)row * J.k;
+        int32_t* ids = J.c_ids + (size_t)row * J.ks;
+        float* pr = J.c_probs + (size_t)row * J.ks;
         if (lane < kept) {
             ids[lane] = (int32_t)(oa >> 32);
             pr[lane] = __uint_as_float((uint32_t)oa);
@@ -1485,8 +1507,8 @@ __device__ void finish_row(const RowJob& J, int64_t row, int32_t req, int n, uin
             }
         }
     } else {
-        int32_t* ids = J.c_ids + (size_t)row * J.k;
-        float* pr = J.c_probs + (size_t)row * J.k;
+        int32_t* ids = J.c_ids + (size_t)row * J.ks;
+        float* pr = J.c_probs + (size_t)row * J.ks;
         for (int j = tid; j < kept; j += kThreads) {
             ids[j] = (int32_t)(outk[j] >> 32);
             pr[j] = __uint_as_float((uint32_t)outk[j]);
@@ -2573,9 +2595,10 @@ static WsLayout ws_layout(int64_t rows, int32_t k, bool compact) {
     off = align_up(off + nslot * 4, 256);
     L.c_ids = off;
     const size_t crow = compact ? (size_t)rows : 0;
-    off = align_up(off + crow * (size_t)k * 4, 256);
+    const size_t ks = (size_t)((k + 3) & ~3);
+    off = align_up(off + crow * ks * 4, 256);
     L.c_probs = off;
-    off = align_up(off + crow * (size_t)k * 4, 256);
+    off = align_up(off + crow * ks * 4, 256);
     L.c_count = off;
     off = align_up(off + crow * 4, 256);
     L.c_flags = off;
@@ -2641,9 +2664,9 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     const size_t slot_bytes = (size_t)kPipeSlots * kPipeConsumers * J.cap_w * 8;
     size_t tail = 0;
     if (MODE == kModeLinear)
-        tail = (size_t)(J.B + 1) * J.k * 8 + (size_t)J.B * 64 * 8 + (size_t)(4 * J.B + 2) * 4;
+        tail = 16 + (size_t)(J.B + 1) * J.ks * 8 + (size_t)J.B * 64 * 8 + (size_t)(4 * J.B + 2) * 4;
     else if (MODE == kModeTree)
-        tail = (size_t)J.V * J.k * 8 + (size_t)J.V * 12 + (size_t)(J.B + 1) * 8;
+        tail = 16 + (size_t)J.V * J.ks * 8 + (size_t)J.V * 12 + (size_t)(J.B + 1) * 8;
     const size_t dyn_max = 227 * 1024 - sizeof(PipeShared);
     auto stride_of = [](size_t tb) { return align_up((size_t)2 * kPipeMaxK * 8 + tb, 128); };
     auto stages_of = [&](size_t tb) -> int64_t {
@@ -2733,6 +2756,7 @@ static void bind_workspace(RowJob& J, void* ws, const WsLayout& L) {
     J.part_count = reinterpret_cast<int32_t*>(b + L.part_count);
     J.part_flags = reinterpret_cast<uint32_t*>(b + L.part_flags);
     J.c_ids = reinterpret_cast<int32_t*>(b + L.c_ids);
+    J.ks = (J.k + 3) & ~3;
     J.c_probs = reinterpret_cast<float*>(b + L.c_probs);
     J.c_count = reinterpret_cast<int32_t*>(b + L.c_count);
     J.c_flags = reinterpret_cast<uint32_t*>(b + L.c_flags);
