@@ -172,8 +172,8 @@ def kernel_source_hash():
 
 
 def committed_traffic():
-    """DRAM bytes per launch of the verify kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
+    """DRAM bytes (read + write) per launch of the filter kernel from the
+    committed ncu summary, if it was taken on the current kernel source."""
     p = ROOT / "profiles" / "traffic.json"
     try:
         d = json.loads(p.read_text())
@@ -181,7 +181,7 @@ def committed_traffic():
         return None
     if d.get("kernel_source_sha") != kernel_source_hash():
         return None
-    return d.get("verify_dram_bytes_per_launch")
+    return d.get("filter_dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------
@@ -383,7 +383,9 @@ def run_ours(args, w):
     peak, peak_kind = hbm_peak()
     verify_bytes = npr * V * w.elem_bytes
     filter_bytes = nq * V * w.elem_bytes
-    achieved = verify_bytes / (fp_ms / 1e3) / 1e9
+    # the dominant kernel: the filter call's single row-kernel launch, timed
+    # alone by the events around its graph replay
+    achieved = filter_bytes / (fq_ms / 1e3) / 1e9
     step_gbs = (verify_bytes + filter_bytes) / (ms_step / 1e3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -391,10 +393,11 @@ def run_ours(args, w):
         "dtype": w.dtype, "data": "synthetic", "config": workload_config(w, world),
         "logits_gbs_per_gpu": step_gbs,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": committed_traffic(), "kernel": "row_kernel<bf16, linear> (uno_linear_verify)",
+                     "traffic": committed_traffic(),
+                     "kernel": "pipe_kernel<bf16, filter> (uno_filter_softmax, 512 rows)",
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                      else "fallback", "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
-                     "filter_kernel_gbs": filter_bytes / (fq_ms / 1e3) / 1e9,
+                     "verify_call_gbs": verify_bytes / (fp_ms / 1e3) / 1e9,
                      "filter_ms": fq_ms, "verify_ms": fp_ms},
         "e2e": {"value": w.R * world / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},

@@ -1536,7 +1536,7 @@ __device__ void finish_row(const RowJob& J, int64_t row, int32_t req, int n, uin
 // The row kernel.
 // ---------------------------------------------------------------------------
 template <typename T, int MODE>
-__global__ void __launch_bounds__(kThreads, 4) row_kernel(const RowJob J) {
+__global__ void __launch_bounds__(kThreads, 4) row_kernel(const __grid_constant__ RowJob J) {
     extern __shared__ __align__(128) unsigned char smem[];
     // streaming: ring stages | barriers | counters | warp buffers
     unsigned char* stages = smem;                                                   // [kStages][kStageBytes]
@@ -2331,7 +2331,7 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
 }
 
 template <typename T, int MODE>
-__global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const RowJob J) {
+__global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_constant__ RowJob J) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ PipeShared P;
     unsigned char* ring = smem;                                                           // [nst][kPStageBytes]
@@ -2373,7 +2373,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const RowJob J) {
 constexpr int kTailWarps = 4;
 
 template <int MODE>
-__global__ void __launch_bounds__(32 * kTailWarps) tail_kernel(const RowJob J, int64_t nreq) {
+__global__ void __launch_bounds__(32 * kTailWarps) tail_kernel(const __grid_constant__ RowJob J, int64_t nreq) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * kTailWarps + warp;
@@ -2398,7 +2398,7 @@ struct TreeJob {
     int32_t* num_nodes;
 };
 
-__global__ void __launch_bounds__(32) tree_expand_kernel(const TreeJob J) {
+__global__ void __launch_bounds__(32) tree_expand_kernel(const __grid_constant__ TreeJob J) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int B = J.B, K = J.K, V = J.V;
     uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem);            // [sort_cap]
