@@ -1725,10 +1725,10 @@ constexpr int kPipeWarps = 1 + kPipeConsumers + kPipeFinishers;
 constexpr int kPipeThreads = 32 * kPipeWarps;
 constexpr int kPipeMaxK = 64;
 // A pipelined stage is 16 KB (1024 units).  In the select pass consumer warp
-// st % 8 owns stage st of an item whole: lane l takes units l, l + 32, ...,
-// (conflict-free shared loads).  In the seed pass every
-// consumer warp reads a slice of each seed stage: warp c units [c*128,
-// (c+1)*128), four per lane.
+// st % kPipeConsumers owns stage st of an item whole: lane l takes units l,
+// l + 32, ... (conflict-free shared loads).  In the seed pass every consumer
+// warp reads a slice of each seed stage: warp c units [c*S, (c+1)*S) with
+// S = kPSliceUnits, S / 32 per lane.
 constexpr int kPStageBytes = 16384;
 constexpr int kPStageUnits = kPStageBytes / 16;                 // 1024
 constexpr int kPLaneUnits = kPStageUnits / 32;                  // 32 per lane per stage
@@ -1747,7 +1747,7 @@ struct __align__(16) PipeShared {
     uint64_t slot_full[kPipeSlots];         // every consumer warp is done with the slot's item
     uint64_t slot_empty[kPipeSlots];        // the finisher is done with the slot's buffers
     unsigned long long tau[2];              // CTA threshold of the current item (by item parity)
-    uint32_t boot[2][kPipeConsumers * 32];  // lane maxima of the seed stages (by item parity)
+    __align__(16) uint32_t boot[2][kPipeConsumers * 32];  // lane maxima of the seed stages (read as uint4)
     uint32_t seed[2];                       // the seed threshold's high word (by item parity)
     int wcnt[kPipeConsumers];               // candidate counts (compaction bookkeeping)
     int cnt[kPipeSlots][kPipeConsumers];    // candidates per consumer warp of the slot's item
@@ -1842,7 +1842,7 @@ __device__ __forceinline__ bool pipe_wait_stage(PipeShared& P, uint32_t qq, uint
     return pipe_wait_warp(&P.full[b], (qq / nst) & 1u, P);
 }
 
-// Consumer barrier over warps 1..8 (named barrier 1) returning the OR of v.
+// Consumer barrier over the filter warps (named barrier 1) returning the OR of v.
 __device__ __forceinline__ bool consumers_sync_or(bool v) {
     uint32_t r;
     asm volatile(
@@ -1900,22 +1900,30 @@ __device__ __forceinline__ void pipe_release(PipeShared& P, uint32_t b, int lane
     if (lane == 0) mbar_arrive(&P.empty[b]);
 }
 
-// A valid threshold from the 256 lane maxima (0 = no element): the largest x
-// with a zero low half such that at least k of them are >= x.  Distinct lanes
-// hold distinct elements, so at least k elements of the segment are >= x.
-// Two bits per step: the counts of three trial values travel packed in one
-// warp reduction (10 bits each; a count is at most 256).
+// A valid threshold from the lane maxima of every filter warp (0 = no
+// element): the largest x with a zero low half such that at least k of them
+// are >= x.  Distinct lanes hold distinct elements, so at least k elements of
+// the segment are >= x.  Two bits per step: the counts of three trial values
+// travel packed in one warp reduction (10 bits each; a count is at most 512).
+constexpr int kSeedPerLane = kPipeConsumers;  // lane maxima per lane of the searching warp
+static_assert(kSeedPerLane % 4 == 0 && kSeedPerLane * 32 < 1024, "packed 10-bit counts");
 __device__ __forceinline__ uint32_t seed_threshold(const uint32_t* bv, int k, int lane) {
-    const uint4 x = reinterpret_cast<const uint4*>(bv)[2 * lane];
-    const uint4 y = reinterpret_cast<const uint4*>(bv)[2 * lane + 1];
-    const uint32_t v[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+    uint32_t v[kSeedPerLane];
+#pragma unroll
+    for (int j = 0; j < kSeedPerLane; j += 4) {
+        const uint4 x = reinterpret_cast<const uint4*>(bv + lane * kSeedPerLane)[j / 4];
+        v[j] = x.x;
+        v[j + 1] = x.y;
+        v[j + 2] = x.z;
+        v[j + 3] = x.w;
+    }
     uint32_t p = 0;  // high bits of the answer found so far
 #pragma unroll
     for (int sh = 14; sh >= 0; sh -= 2) {
         const uint32_t t1 = (p | (1u << sh)) << 16, t2 = (p | (2u << sh)) << 16, t3 = (p | (3u << sh)) << 16;
         uint32_t c = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < kSeedPerLane; ++j)
             c += (v[j] >= t1 ? 1u : 0u) + (v[j] >= t2 ? (1u << 10) : 0u) + (v[j] >= t3 ? (1u << 20) : 0u);
         c = __reduce_add_sync(kFull, c);
         const uint32_t kk = (uint32_t)k;
