@@ -983,42 +983,77 @@ __device__ __forceinline__ void tail_timeout(const RowJob& J, int32_t r, int lan
     }
 }
 
+// Bytes of the 16-byte-aligned middle of the byte range [src, src + n).
+__device__ __forceinline__ uint32_t range_bulk_bytes(const unsigned char* src, uint32_t n) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(src), a1 = a0 + n;
+    const uintptr_t m0 = (a0 + 15u) & ~(uintptr_t)15u, m1 = a1 & ~(uintptr_t)15u;
+    return m1 > m0 ? (uint32_t)(m1 - m0) : 0u;
+}
+
+// Bring the 4-byte-aligned byte range [src, src + n) of global memory into
+// shared memory at dst (the same address modulo 16: dst is a 16-aligned
+// region plus src % 16): lane 0 bulk-copies the 16-byte-aligned middle on
+// bar (lane 0 has already added range_bulk_bytes to the barrier's expected
+// count), lanes 1..6 copy the at most three words at each edge.  Nothing
+// outside the range is read.
+__device__ __forceinline__ void copy_range_async(unsigned char* dst, const unsigned char* src, uint32_t n,
+                                                 uint64_t* bar, int lane) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(src), a1 = a0 + n;
+    const uintptr_t m0 = (a0 + 15u) & ~(uintptr_t)15u, m1 = a1 & ~(uintptr_t)15u;
+    if (m1 > m0 && lane == 0) bulk_g2s(dst + (m0 - a0), reinterpret_cast<const void*>(m0), (uint32_t)(m1 - m0), bar);
+    // edge words: [a0, min(m0, a1)) and [max(m1, m0), a1)
+    const uintptr_t h1 = m0 < a1 ? m0 : a1, t0 = m1 > m0 ? m1 : (m0 < a1 ? m0 : a1);
+    const int nh = (int)((h1 - a0) / 4), nt = (int)((a1 - t0) / 4);
+    if (lane >= 1 && lane <= nh) {
+        const uintptr_t a = a0 + 4u * (uintptr_t)(lane - 1);
+        *reinterpret_cast<uint32_t*>(dst + (a - a0)) = *reinterpret_cast<const uint32_t*>(a);
+    } else if (lane >= 4 && lane < 4 + nt) {
+        const uintptr_t a = t0 + 4u * (uintptr_t)(lane - 4);
+        *reinterpret_cast<uint32_t*>(dst + (a - a0)) = *reinterpret_cast<const uint32_t*>(a);
+    }
+}
+
 __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsigned char* sm, int lane) {
     const int32_t B = J.B;
     const int kc = J.k, ks = J.ks;
     constexpr int QS = 64;  // q entries kept per row
     if (kc > 64 || B > 31) return false;
-    const size_t need = 16 + (size_t)(B + 1) * ks * 8 + (size_t)B * QS * 8 + (size_t)(4 * B + 2) * 4;
+    const size_t need = 16 + (size_t)(B + 1) * ks * 8 + 2 * ((size_t)B * QS * 4 + 16) + (size_t)(4 * B + 2) * 4;
     if (need > (size_t)J.tail_bytes) return false;
-    // q rows come in one bulk copy when the caller's layout allows it
-    const bool qbulk = (reinterpret_cast<uintptr_t>(J.q_ids) & 15u) == 0 &&
-                       (reinterpret_cast<uintptr_t>(J.q_probs) & 15u) == 0 && (J.q_cap & 3) == 0 && J.q_cap <= QS;
-    const int qs = qbulk ? J.q_cap : QS;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(sm);                         // the copies' mbarrier
-    int32_t* pid = reinterpret_cast<int32_t*>(sm + 16);                      // [B+1][ks]
-    float* ppr = reinterpret_cast<float*>(pid + (B + 1) * ks);               // [B+1][ks]
-    int32_t* qid = reinterpret_cast<int32_t*>(ppr + (B + 1) * ks);           // [B][qs]
-    float* qpr = reinterpret_cast<float*>(qid + B * qs);                     // [B][qs]
-    int32_t* pcnt = reinterpret_cast<int32_t*>(qpr + B * qs);                // [B+1]
-    int32_t* qcnt = pcnt + (B + 1);                                          // [B]
-    int32_t* dft = qcnt + B;                                                 // [B]
-    int32_t* otok = dft + B;                                                 // [B+1] emitted tokens
+    // the draft rows as one byte range per array (stride q_cap) when short
+    const bool qflat = J.q_cap <= QS;
+    const int qs = qflat ? J.q_cap : QS;
+    const uint32_t qn = (uint32_t)B * (uint32_t)J.q_cap * 4u;
+    const unsigned char* qsi = reinterpret_cast<const unsigned char*>(J.q_ids + (size_t)r * B * J.q_cap);
+    const unsigned char* qsp = reinterpret_cast<const unsigned char*>(J.q_probs + (size_t)r * B * J.q_cap);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm);                              // the copies' mbarrier
+    int32_t* pid = reinterpret_cast<int32_t*>(sm + 16);                           // [B+1][ks]
+    float* ppr = reinterpret_cast<float*>(pid + (B + 1) * ks);                    // [B+1][ks]
+    unsigned char* qreg_i = reinterpret_cast<unsigned char*>(ppr + (B + 1) * ks);  // 16-aligned regions
+    unsigned char* qreg_p = qreg_i + ((size_t)B * QS * 4 + 16);
+    int32_t* qid = reinterpret_cast<int32_t*>(qflat ? qreg_i + (reinterpret_cast<uintptr_t>(qsi) & 15u) : qreg_i);  // [B][qs]
+    float* qpr = reinterpret_cast<float*>(qflat ? qreg_p + (reinterpret_cast<uintptr_t>(qsp) & 15u) : qreg_p);     // [B][qs]
+    int32_t* pcnt = reinterpret_cast<int32_t*>(qreg_p + ((size_t)B * QS * 4 + 16));  // [B+1]
+    int32_t* qcnt = pcnt + (B + 1);                                                  // [B]
+    int32_t* dft = qcnt + B;                                                         // [B]
+    int32_t* otok = dft + B;                                                         // [B+1] emitted tokens
     const int64_t base = (int64_t)r * (B + 1);
     const uint32_t req = J.first_request + (uint32_t)r;
-    // The request's compact target rows (and q rows) arrive by bulk copies
+    // The request's compact target rows and draft rows arrive by bulk copies
     // (TMA) on one mbarrier: one round trip, whatever the memory system's
     // queueing; counts, flags and drafts load alongside.
     if (lane == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
-        const uint32_t pb = (uint32_t)((B + 1) * ks * 4), qb = qbulk ? (uint32_t)(B * qs * 4) : 0u;
-        mbar_expect_tx(bar, 2 * pb + 2 * qb);
+        const uint32_t pb = (uint32_t)((B + 1) * ks * 4);
+        const uint32_t qb = qflat ? range_bulk_bytes(qsi, qn) + range_bulk_bytes(qsp, qn) : 0u;
+        mbar_expect_tx(bar, 2 * pb + qb);  // before any copy is issued
         bulk_g2s(pid, J.c_ids + (size_t)base * ks, pb, bar);
         bulk_g2s(ppr, J.c_probs + (size_t)base * ks, pb, bar);
-        if (qbulk) {
-            bulk_g2s(qid, J.q_ids + (size_t)r * B * J.q_cap, qb, bar);
-            bulk_g2s(qpr, J.q_probs + (size_t)r * B * J.q_cap, qb, bar);
-        }
+    }
+    if (qflat) {
+        copy_range_async(reinterpret_cast<unsigned char*>(qid), qsi, qn, bar, lane);
+        copy_range_async(reinterpret_cast<unsigned char*>(qpr), qsp, qn, bar, lane);
     }
     int pc_l = 0, qc_l = 0, d_l = 0;
     uint32_t f_l = 0;
@@ -1030,11 +1065,9 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
         qc_l = J.q_count[(int64_t)r * B + lane];
         d_l = J.draft_ids[(size_t)r * B + lane];
     }
-    if (!qbulk) {
-        const int qw = J.q_cap < QS ? J.q_cap : QS;
-        warp_copy_rows<false>(J.q_ids + (size_t)r * B * J.q_cap, J.q_probs + (size_t)r * B * J.q_cap, J.q_cap, B, qw,
+    if (!qflat)
+        warp_copy_rows<false>(J.q_ids + (size_t)r * B * J.q_cap, J.q_probs + (size_t)r * B * J.q_cap, J.q_cap, B, QS,
                               qid, qpr, QS, lane);
-    }
     // the decisions' uniforms, one position per lane
     double ua = 0.0, ur = 0.0;
     if (lane < B) {
@@ -2383,12 +2416,19 @@ constexpr int kTailWarps = 4;
 template <int MODE>
 __global__ void __launch_bounds__(32 * kTailWarps) tail_kernel(const __grid_constant__ RowJob J, int64_t nreq) {
     extern __shared__ __align__(128) unsigned char smem[];
+    // The job in shared memory: the tails read many of its fields once each,
+    // and one parallel copy beats a chain of cold parameter-cache misses.
+    __shared__ __align__(16) RowJob sJ;
+    static_assert(sizeof(RowJob) % 4 == 0, "copied by words");
+    for (int i = threadIdx.x; i < (int)(sizeof(RowJob) / 4); i += blockDim.x)
+        reinterpret_cast<uint32_t*>(&sJ)[i] = reinterpret_cast<const uint32_t*>(&J)[i];
+    __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * kTailWarps + warp;
     if (r >= nreq) return;
-    unsigned char* mine = smem + (size_t)warp * J.fin_stride;
+    unsigned char* mine = smem + (size_t)warp * sJ.fin_stride;
     double* wd = reinterpret_cast<double*>(mine);  // [k] (the global-memory path)
-    request_tail<MODE>(J, (int32_t)r, wd, mine + (size_t)kPipeMaxK * 8, lane);
+    request_tail<MODE>(sJ, (int32_t)r, wd, mine + (size_t)kPipeMaxK * 8, lane);
 }
 
 // ---------------------------------------------------------------------------
@@ -2672,7 +2712,7 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     const size_t slot_bytes = (size_t)kPipeSlots * kPipeConsumers * J.cap_w * 8;
     size_t tail = 0;
     if (MODE == kModeLinear)
-        tail = 16 + (size_t)(J.B + 1) * J.ks * 8 + (size_t)J.B * 64 * 8 + (size_t)(4 * J.B + 2) * 4;
+        tail = 16 + (size_t)(J.B + 1) * J.ks * 8 + 2 * ((size_t)J.B * 64 * 4 + 16) + (size_t)(4 * J.B + 2) * 4;
     else if (MODE == kModeTree)
         tail = 16 + (size_t)J.V * J.ks * 8 + (size_t)J.V * 12 + (size_t)(J.B + 1) * 8;
     const size_t dyn_max = 227 * 1024 - sizeof(PipeShared);
