@@ -116,9 +116,6 @@ struct Elem<__nv_bfloat16> {
     }
     // true when some element of the unit may be >= tau, or is NaN
     __device__ static bool maybe(const uint4& r, Tau tau) { return !__hblt2(umax(r), tau); }
-    __device__ static bool chunk_maybe(const uint4* c, Tau tau) {
-        return !__hblt2(__hmax2_nan(__hmax2_nan(umax(c[0]), umax(c[1])), __hmax2_nan(umax(c[2]), umax(c[3]))), tau);
-    }
     __device__ static float get(const uint4& r, int e) {
         const uint32_t w = (e < 2) ? r.x : (e < 4) ? r.y : (e < 6) ? r.z : r.w;
         return __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
@@ -169,13 +166,6 @@ struct Elem<__nv_bfloat16> {
             }
         }
     }
-    // ordered bits of the second largest tracked element, 0 when there is none
-    __device__ static uint32_t second_ord(Top m1, Top m2) {
-        const float a1 = __low2float(m1), b1 = __high2float(m1), a2 = __low2float(m2), b2 = __high2float(m2);
-        const float second = fmaxf(fminf(a1, b1), fmaxf(a2, b2));
-        if (!(second > -__int_as_float(0x7f800000))) return 0u;
-        return ord_of_float(__fadd_rn(second, 0.0f));
-    }
     // ordered bits of the lane's two largest tracked elements (0 = none)
     __device__ static void lane_top2_ord(Top m1, Top m2, uint32_t& t1, uint32_t& t2) {
         const float a1 = __low2float(m1), b1 = __high2float(m1), a2 = __low2float(m2), b2 = __high2float(m2);
@@ -186,22 +176,6 @@ struct Elem<__nv_bfloat16> {
     }
     // bit u*8+e set when element e of unit u is >= tau (rounded down) or NaN
     __device__ static unsigned cand_mask4(const uint4* c, Tau tau) {
-        unsigned m = 0;
-#pragma unroll
-        for (int u = 0; u < kUnits; ++u) {
-            if (maybe(c[u], tau)) {
-                const uint32_t w[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const unsigned g = __hgeu2_mask(w2(w[q]), tau);
-                    m |= ((g & 1u) | ((g >> 15) & 2u)) << (u * 8 + 2 * q);
-                }
-            }
-        }
-        return m;
-    }
-    // bit u*8+e set when element e of unit u is >= tau (rounded down) or NaN
-    __device__ static unsigned cand_mask(const uint4* c, Tau tau) {
         unsigned m = 0;
 #pragma unroll
         for (int u = 0; u < kUnits; ++u) {
@@ -234,9 +208,6 @@ struct Elem<float> {
                        max_nan(__uint_as_float(r.z), __uint_as_float(r.w)));
     }
     __device__ static bool maybe(const uint4& r, Tau tau) { return !(umax(r) < tau); }
-    __device__ static bool chunk_maybe(const uint4* c, Tau tau) {
-        return !(max_nan(max_nan(umax(c[0]), umax(c[1])), max_nan(umax(c[2]), umax(c[3]))) < tau);
-    }
     __device__ static float get(const uint4& r, int e) {
         const uint32_t w = (e == 0) ? r.x : (e == 1) ? r.y : (e == 2) ? r.z : r.w;
         return __uint_as_float(w);
@@ -276,11 +247,6 @@ struct Elem<float> {
             }
         }
     }
-    __device__ static uint32_t second_ord(Top m1, Top m2) {
-        (void)m1;
-        if (!(m2 > -__int_as_float(0x7f800000))) return 0u;
-        return ord_of_float(__fadd_rn(m2, 0.0f));
-    }
     __device__ static void lane_top2_ord(Top m1, Top m2, uint32_t& t1, uint32_t& t2) {
         t1 = (m1 > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(m1, 0.0f)) : 0u;
         t2 = (m2 > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(m2, 0.0f)) : 0u;
@@ -297,27 +263,8 @@ struct Elem<float> {
         }
         return m;
     }
-    // bit u*4+e set when element e of unit u is >= tau or NaN
-    __device__ static unsigned cand_mask(const uint4* c, Tau tau) {
-        unsigned m = 0;
-#pragma unroll
-        for (int u = 0; u < kUnits; ++u) {
-            const float x[4] = {__uint_as_float(c[u].x), __uint_as_float(c[u].y), __uint_as_float(c[u].z),
-                                __uint_as_float(c[u].w)};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) m |= (!(x[q] < tau) ? 1u : 0u) << (u * 4 + q);
-        }
-        return m;
-    }
 };
 
-// 32-byte streaming load (bypasses L1, 256-byte L2 prefetch hint).  The
-// address is 32-byte aligned.
-__device__ __forceinline__ void ld_stream32(const void* p, uint4& lo, uint4& hi) {
-    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                 : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
-                 : "l"(p));
-}
 
 // Per-warp streaming state.  Candidates are appended by single lanes with a
 // shared-memory counter (*wcnt); cnt is the warp-uniform copy of it.
@@ -350,25 +297,6 @@ __device__ __noinline__ Compacted warp_compact(uint64_t* buf, int* wcnt, int cnt
     if (lane == 0) *wcnt = cnt;
     __syncwarp();
     return Compacted{cnt, tau};
-}
-
-// One lane's slow path for one 16-byte unit: append every finite element
-// whose key beats the threshold (ids id0 ..); flag NaN / +inf.
-template <typename T>
-__device__ __forceinline__ void append_lane_unit(const uint4& r, uint32_t id0, float tau_f, uint64_t tau,
-                                                 uint64_t* buf, int* wcnt, uint32_t& bad) {
-#pragma unroll
-    for (int e = 0; e < Elem<T>::kPerUnit; ++e) {
-        const float v = Elem<T>::get(r, e);
-        if (!(v < tau_f)) {  // v >= threshold value, or NaN
-            if (v != v || v == __int_as_float(0x7f800000)) {
-                bad = 1u;
-            } else if (v != -__int_as_float(0x7f800000)) {
-                const uint64_t key = make_key(v, id0 + (uint32_t)e);
-                if (key > tau) buf[atomicAdd(wcnt, 1)] = key;
-            }
-        }
-    }
 }
 
 // Geometry of a row: `head` scalar elements up to the first 16-byte boundary,
@@ -888,19 +816,6 @@ __device__ __forceinline__ int warp_inv_cdf(double wa, double wb, double u, int 
 // tails above) when the rows do not fit.
 // ---------------------------------------------------------------------------
 
-// Probability of token x in a compact row held in shared memory (0 if absent).
-__device__ __forceinline__ double warp_lookup(const int32_t* ids, const float* pr, int n, int32_t x, int lane) {
-    float v = 0.0f;
-    bool hit = false;
-    for (int j = lane; j < n; j += 32)
-        if (ids[j] == x) {
-            v = pr[j];
-            hit = true;
-        }
-    const unsigned bal = __ballot_sync(kFull, hit);
-    if (!bal) return 0.0;
-    return (double)__shfl_sync(kFull, v, __ffs(bal) - 1);
-}
 
 // Probability of token x in a compact row with ascending ids (one lane,
 // binary search in shared memory).

@@ -158,3 +158,35 @@ def test_tree_nonfinite_node_rows():
     g, r, rt = run_tree(w, rng=(5, 0), target_edit=edit)
     assert np_of(g["flags"])[0] & oracle.FLAG_NONFINITE_ROW
     assert np_of(g["num_tokens"])[0] == 0
+
+
+@pytest.mark.parametrize("layout", ["wide rows", "offset start"])
+def test_linear_draft_row_layouts(layout):
+    """The draft rows as the verifier receives them: a row stride above 64 entries
+    (cap 100 for top-k 50), or arrays that start 4 bytes past a 16-byte boundary.
+    Both must give the same verification as the oracle."""
+    w = Workload("lin bf16 layouts", "linear", R=12, B=6, vocab=4099, dtype="bf16", sigma=1.0, noise=0.7, peak=6.0,
+                 seed=21)
+    rng = (77, 2)
+    sp = dict(temperature=w.temperature, top_k=w.top_k, top_p=w.top_p)
+    q_np, p_np = linear_draft(w), linear_target(w)
+    ev = Events()
+    cap = 100 if layout == "wide rows" else w.top_k
+    gq = uno_filter_softmax(to_device(q_np, w.dtype), rows_per_request=w.B, rng=rng, cap=cap, **sp)
+    rq = oracle.filter_softmax(q_np, w.dtype, w.temperature, w.top_k, w.top_p, rows_per_request=w.B, rng=rng)
+    compare_filter(gq, rq, ev, sample=True)
+    q_ids, q_probs = gq["ids"], gq["probs"]
+    if layout == "offset start":
+        n = q_ids.numel()
+        flat_i = torch.empty(n + 1, dtype=q_ids.dtype, device=q_ids.device)
+        flat_p = torch.empty(n + 1, dtype=q_probs.dtype, device=q_probs.device)
+        flat_i[1:].copy_(q_ids.reshape(-1))
+        flat_p[1:].copy_(q_probs.reshape(-1))
+        q_ids, q_probs = flat_i[1:].view(q_ids.shape), flat_p[1:].view(q_probs.shape)
+        assert q_ids.data_ptr() % 16 == 4
+    g = uno_linear_verify(to_device(p_np, w.dtype), gq["sample"].reshape(w.R, w.B), q_ids, q_probs, gq["count"],
+                          R=w.R, B=w.B, rng=rng, **sp)
+    r = oracle.linear_verify(p_np, w.dtype, w.R, w.B, w.temperature, w.top_k, w.top_p,
+                             rq["sample"].reshape(w.R, w.B), rq["ids"], rq["probs"], rq["count"], rng=rng)
+    compare_requests(g, r, ev, LINEAR_KEYS)
+    ev.check()
