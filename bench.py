@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", type=int, default=WORKLOAD_INDEX, help="index into inputs.WORKLOADS (linear only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-tree", action="store_true", help="skip the tree-path timings")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget of the cpu_baseline")
     return ap.parse_args()
 
@@ -252,6 +253,59 @@ def workload_config(w, world):
 
 
 # ---------------------------------------------------------------------------
+# the tree path (reported beside the headline metric)
+# ---------------------------------------------------------------------------
+TREE_WORKLOAD_INDEX = 3
+
+
+def tree_leg(device, first, reps=30):
+    """Time the tree cycle on the tree 8/16/8 workload (64 requests): filter of
+    the R*B draft rows, top-K extraction + best-first expansion, and target-only
+    verification of the R*V node rows.  Inputs resident in HBM; CUDA events
+    around each call on the current stream."""
+    import torch
+    from speculative_decoding_verification_filter_b200 import (uno_filter_softmax, uno_tree_topk_expand,
+                                                              uno_tree_verify)
+    from speculative_decoding_verification_filter_b200.inputs import WORKLOADS, tree_draft, tree_target
+    w = WORKLOADS[TREE_WORKLOAD_INDEX]
+    reqs = range(first, first + w.R)
+    sp = dict(temperature=w.temperature, top_k=w.top_k, top_p=w.top_p)
+
+    def dev(a):
+        return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+
+    q = dev(tree_draft(w, reqs))
+    fo = uno_filter_softmax(q, rows_per_request=w.B, **sp)
+    to = uno_tree_topk_expand(fo["ids"], fo["probs"], fo["count"], R=w.R, B=w.B, K=w.K, V=w.V)
+    p = dev(tree_target(w, to["node_depth"].cpu().numpy(), to["num_nodes"].cpu().numpy(), reqs))
+    rng = (w.seed, 0, first)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+        for i in range(reps):
+            ev[2 * i].record()
+            fn()
+            ev[2 * i + 1].record()
+        torch.cuda.synchronize(device)
+        return statistics.fmean(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(reps))
+
+    f_ms = timed(lambda: uno_filter_softmax(q, rows_per_request=w.B, **sp))
+    e_ms = timed(lambda: uno_tree_topk_expand(fo["ids"], fo["probs"], fo["count"], R=w.R, B=w.B, K=w.K, V=w.V))
+    v_ms = timed(lambda: uno_tree_verify(p, to["node_token"], to["node_parent"], to["num_nodes"], R=w.R, B=w.B,
+                                         V=w.V, rng=rng, **sp))
+    active = int(to["num_nodes"].sum().item())
+    row_bytes = w.vocab * w.elem_bytes
+    return {"workload": f"{w.name}: R={w.R}, B={w.B}, K={w.K}, V={w.V}, vocab {w.vocab}, {w.dtype}",
+            "filter_ms": f_ms, "expand_ms": e_ms, "verify_ms": v_ms,
+            "filter_gbs": w.R * w.B * row_bytes / (f_ms / 1e3) / 1e9,
+            "verify_active_rows": active, "verify_gbs": active * row_bytes / (v_ms / 1e3) / 1e9,
+            "note": ("per-call CUDA-event times through the Python API, so a call whose GPU work is shorter than "
+                     "its host-side launch (expand) reports the launch; verify reads only the active node rows")}
+
+
+# ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 def run_ours(args, w):
@@ -406,6 +460,8 @@ def run_ours(args, w):
         "gpu_launches": K * (1 + (2 if min(w.top_k, w.vocab) <= 64 else 1)),
         "clocks": clocks,
     }
+    if not args.no_tree:
+        line["tree"] = tree_leg(device, rank * 64)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if rank == 0:
