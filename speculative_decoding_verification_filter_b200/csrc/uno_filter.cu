@@ -2377,80 +2377,30 @@ __global__ void __launch_bounds__(32) tree_expand_kernel(const __grid_constant__
     const int lane = threadIdx.x;
     const int r = blockIdx.x;
 
-    // 1. top-K of each marginal by (prob desc, id asc).  Rows of at most 64
-    // entries: every row's two keys per lane load first (all loads in flight
-    // together), then a register bitonic sort per row.  Wider rows: a
-    // shared-memory sort.
-    constexpr int kRegRows = 8;  // marginals whose keys are staged in registers at a time
-    if (J.q_cap <= 64) {
-        for (int d0 = 0; d0 < B; d0 += kRegRows) {
-            uint64_t ka[kRegRows], kb[kRegRows];
-            int cnt[kRegRows];
-#pragma unroll
-            for (int j = 0; j < kRegRows; ++j) {
-                const int d = d0 + j;
-                ka[j] = kb[j] = 0ull;
-                cnt[j] = 0;
-                if (d < B) {
-                    const int64_t row = (int64_t)r * B + d;
-                    int c = J.q_count[row];
-                    c = c < 0 ? 0 : (c > J.q_cap ? J.q_cap : c);
-                    cnt[j] = c;
-                    const float* pr = J.q_probs + (size_t)row * J.q_cap;
-                    const int32_t* ids = J.q_ids + (size_t)row * J.q_cap;
-                    if (lane < c)
-                        ka[j] = ((uint64_t)ord_of_float(__fadd_rn(pr[lane], 0.0f)) << 32) | (uint64_t)(~(uint32_t)ids[lane]);
-                    if (lane + 32 < c)
-                        kb[j] = ((uint64_t)ord_of_float(__fadd_rn(pr[lane + 32], 0.0f)) << 32) |
-                                (uint64_t)(~(uint32_t)ids[lane + 32]);
-                }
+    // 1. top-K of each marginal by (prob desc, id asc)
+    for (int d = 0; d < B; ++d) {
+        const int64_t row = (int64_t)r * B + d;
+        int c = J.q_count[row];
+        c = c < 0 ? 0 : (c > J.q_cap ? J.q_cap : c);
+        const int np2 = next_pow2(c < 1 ? 1 : c);
+        for (int i = lane; i < np2; i += 32) {
+            uint64_t key = 0ull;
+            if (i < c) {
+                const float p = __fadd_rn(J.q_probs[(size_t)row * J.q_cap + i], 0.0f);
+                const int32_t id = J.q_ids[(size_t)row * J.q_cap + i];
+                key = ((uint64_t)ord_of_float(p) << 32) | (uint64_t)(~(uint32_t)id);
             }
-#pragma unroll
-            for (int j = 0; j < kRegRows; ++j) {
-                const int d = d0 + j;
-                if (d >= B) break;
-                // ascending sort of the complements = descending keys (missing
-                // entries, key 0, sort last)
-                uint64_t xa = ~ka[j], xb = ~kb[j];
-                warp_sort64(xa, xb, lane);
-                const int nk = cnt[j] < K ? cnt[j] : K;
-                if (lane < nk) {
-                    cand_id[d * K + lane] = key_id(~xa);
-                    cand_p[d * K + lane] = float_of_ord((uint32_t)(~xa >> 32));
-                }
-                if (lane + 32 < nk) {
-                    cand_id[d * K + lane + 32] = key_id(~xb);
-                    cand_p[d * K + lane + 32] = float_of_ord((uint32_t)(~xb >> 32));
-                }
-                if (lane == 0) ncand[d] = nk;
-            }
+            sortbuf[i] = key;
         }
         __syncwarp();
-    } else {
-        for (int d = 0; d < B; ++d) {
-            const int64_t row = (int64_t)r * B + d;
-            int c = J.q_count[row];
-            c = c < 0 ? 0 : (c > J.q_cap ? J.q_cap : c);
-            const int np2 = next_pow2(c < 1 ? 1 : c);
-            for (int i = lane; i < np2; i += 32) {
-                uint64_t key = 0ull;
-                if (i < c) {
-                    const float p = __fadd_rn(J.q_probs[(size_t)row * J.q_cap + i], 0.0f);
-                    const int32_t id = J.q_ids[(size_t)row * J.q_cap + i];
-                    key = ((uint64_t)ord_of_float(p) << 32) | (uint64_t)(~(uint32_t)id);
-                }
-                sortbuf[i] = key;
-            }
-            __syncwarp();
-            warp_bitonic_sort(sortbuf, np2, true, lane);
-            const int nk = c < K ? c : K;
-            for (int i = lane; i < nk; i += 32) {
-                cand_id[d * K + i] = key_id(sortbuf[i]);
-                cand_p[d * K + i] = float_of_ord((uint32_t)(sortbuf[i] >> 32));
-            }
-            if (lane == 0) ncand[d] = nk;
-            __syncwarp();
+        warp_bitonic_sort(sortbuf, np2, true, lane);
+        const int nk = c < K ? c : K;
+        for (int i = lane; i < nk; i += 32) {
+            cand_id[d * K + i] = key_id(sortbuf[i]);
+            cand_p[d * K + i] = float_of_ord((uint32_t)(sortbuf[i] >> 32));
         }
+        if (lane == 0) ncand[d] = nk;
+        __syncwarp();
     }
 
     int32_t* tok = J.node_token + (size_t)r * V;
