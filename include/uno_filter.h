@@ -224,11 +224,13 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
  * Arguments, results and errors are those of uno_linear_verify, minus the
  * workspace.  Sizes whose uno_linear_verify_workspace_bytes exceeds
  * UNO_NOALLOC_SCRATCH_BYTES return UNO_ERR_UNSUPPORTED before anything is
- * enqueued: the 8 MiB hold R*(B+1) * min(top_k, vocab) up to about 880,000
- * (512 requests with B = 16 at top_k 50 fit; at top_k 200 they do not).  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  The call itself allocates nothing: it enqueues
- * cudaMemsetAsync of the counters it uses, then the kernel.  Every call
+ * enqueued: the 8 MiB hold R*(B+1) * k4 up to about 880,000, k4 being
+ * min(top_k, vocab) rounded up to a multiple of 4 (512 requests with B = 16
+ * at top_k 50 fit; at top_k 200 they do not).  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  The call
+ * itself allocates nothing: it enqueues cudaMemsetAsync of the counters it
+ * uses, then its kernels.  Every call
  * shares the one array, so calls that overlap on the GPU (other streams,
  * other host threads) race; serialise them.
  * ---------------------------------------------------------------------- */
