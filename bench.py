@@ -226,7 +226,8 @@ def run_reference(args, w):
     t_req = oracle_requests(w, [0])
     budget = 150.0
     steps = max(1, min(args.steps, int(budget / max(t_req, 1e-3))))
-    warm = min(args.warmup, 1)
+    # at least three warm-up steps, at most about 30 s of them
+    warm = max(3, min(args.warmup, int(30.0 / max(t_req, 1e-3))))
     oracle_requests(w, [1 % w.R] * warm)
     secs = oracle_requests(w, [(2 + i) % w.R for i in range(steps)])
     value = steps / secs

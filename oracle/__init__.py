@@ -28,6 +28,20 @@ What pins each function (the tests under ``tests/test_oracle_*.py``):
 * ``tree_verify``: emitted sequence distributed as the target-only process
   (chi-square), mean accept length equals the sum over tree nodes of the
   target path probability, one-hot targets equal greedy decoding.
+* the joint filter order (``order="joint"``, top-p read from the softmax of
+  the whole row): a worked example derived by hand (weights 4 : 2 : 1 : 1),
+  the closed form of a geometric row, its definition written with
+  ``scipy.special.softmax`` over the whole row, the nesting of its support
+  over the top-k-first one, reduction to the top-k-first order when
+  top_p = 1 or top_k >= vocab, and linear verification under it distributed
+  as the joint-filtered target process (chi-square).
+* per-request sampling parameters (arrays of temperature, top_k, top_p):
+  every call equals the same requests run one at a time.
+* ``linear_cycle`` (the two-pass layout: base-weights first token, B - 1
+  proposals, B + 1 output slots): it emits exactly what ``linear_verify``
+  emits when the first draft row is also the first target row; its counters
+  satisfy num_correct_drafts = accept_len - 2 and sum to the generated-token
+  count; its output is distributed as the target-only process (chi-square).
 
 Parity unpinned: the boundary-event margin below which a GPU/oracle decision
 difference is excused (``BOUNDARY_EPS``) is a stated tolerance, not a value the
@@ -87,6 +101,18 @@ def _bind(lib):
     lib.uno_ref_tree_verify.argtypes = [P, ctypes.c_int, i32, i32, i32, i64, f32, i32, f32, P, P, P,
                                         u64, u32, u32, P, P, P, P, P, P]
     lib.uno_ref_tree_verify.restype = ctypes.c_int
+    lib.uno_ref_filter_softmax_params.argtypes = [P, ctypes.c_int, i64, i64, i64, i32, P, P, P, ctypes.c_int,
+                                                  i32, P, P, P, P, ctypes.c_int, u64, u32, u32, P, P, P]
+    lib.uno_ref_filter_softmax_params.restype = ctypes.c_int
+    lib.uno_ref_linear_verify_params.argtypes = [P, ctypes.c_int, i32, i32, i64, P, P, P, ctypes.c_int, P, P, P,
+                                                 P, i32, u64, u32, u32, P, P, P, P, P]
+    lib.uno_ref_linear_verify_params.restype = ctypes.c_int
+    lib.uno_ref_tree_verify_params.argtypes = [P, ctypes.c_int, i32, i32, i32, i64, P, P, P, ctypes.c_int, P, P,
+                                               P, u64, u32, u32, P, P, P, P, P, P]
+    lib.uno_ref_tree_verify_params.restype = ctypes.c_int
+    lib.uno_ref_linear_cycle.argtypes = [P, P, ctypes.c_int, i32, i32, i64, P, P, P, ctypes.c_int, u64, u32, u32,
+                                         P, P, P, P, P]
+    lib.uno_ref_linear_cycle.restype = ctypes.c_int
     return lib
 
 
@@ -143,6 +169,34 @@ class OracleError(RuntimeError):
     pass
 
 
+# Filter orders: "topk_first" renormalises the top-k set before the top-p
+# cut; "joint" takes the top-p cut on the full-vocabulary softmax.
+ORDERS = {"topk_first": 0, "joint": 1}
+
+
+def _order_code(order):
+    if order not in ORDERS:
+        raise ValueError("order must be one of %s" % sorted(ORDERS))
+    return ORDERS[order]
+
+
+def _param_arrays(temperature, top_k, top_p, nreq):
+    """One temperature, top_k and top_p per request (scalars broadcast)."""
+    T = np.ascontiguousarray(np.broadcast_to(np.asarray(temperature, dtype=np.float32), (nreq,)))
+    K = np.ascontiguousarray(np.broadcast_to(np.asarray(top_k, dtype=np.int32), (nreq,)))
+    P = np.ascontiguousarray(np.broadcast_to(np.asarray(top_p, dtype=np.float32), (nreq,)))
+    return T, K, P
+
+
+def _per_request(temperature, top_k, top_p, order, nreq):
+    """None when the call is the scalar top-k-first form; otherwise the
+    three per-request arrays and the order code."""
+    code = _order_code(order)
+    if order == "topk_first" and all(np.ndim(v) == 0 for v in (temperature, top_k, top_p)):
+        return None
+    return _param_arrays(temperature, top_k, top_p, nreq) + (code,)
+
+
 def _check(rc, what):
     if rc != 0:
         raise OracleError(f"{what}: oracle status {rc}")
@@ -163,14 +217,17 @@ def uniform(seed, request, position, draw, cycle=0):
 
 
 def filter_softmax(logits, dtype, temperature, top_k, top_p, *, rows_per_request=1, cap=None,
-                   rng=None, dense=False):
+                   rng=None, dense=False, order="topk_first"):
     """Filter each row of ``logits`` ([rows, vocab]); returns a dict with
     ids [rows, cap], probs [rows, cap], count, flags, margin, and, on request,
-    sample (rng = (seed, cycle)) and dense [rows, vocab]."""
+    sample (rng = (seed, cycle)) and dense [rows, vocab].  temperature, top_k
+    and top_p are scalars or one value per request."""
     a, code = _logits(logits, dtype)
     rows, vocab = a.shape
+    nreq = -(-rows // rows_per_request)
+    per = _per_request(temperature, top_k, top_p, order, nreq)
     if cap is None:
-        cap = min(top_k, vocab)
+        cap = max(1, min(int(np.max(top_k)), vocab))
     ids = np.empty((rows, cap), dtype=np.int32)
     probs = np.empty((rows, cap), dtype=np.float32)
     count = np.empty(rows, dtype=np.int32)
@@ -179,11 +236,15 @@ def filter_softmax(logits, dtype, temperature, top_k, top_p, *, rows_per_request
     dn = np.empty((rows, vocab), dtype=np.float32) if dense else None
     sample = np.empty(rows, dtype=np.int32) if rng is not None else None
     seed, cycle, first = _rng(rng)
-    rc = _load().uno_ref_filter_softmax(_ptr(a), code, rows, vocab, vocab, rows_per_request,
-                                        float(temperature), int(top_k), float(top_p), cap,
-                                        _ptr(ids), _ptr(probs), _ptr(count), _ptr(dn),
-                                        1 if rng is not None else 0, seed, cycle, first,
-                                        _ptr(sample), _ptr(flags), _ptr(margin))
+    tail = (cap, _ptr(ids), _ptr(probs), _ptr(count), _ptr(dn), 1 if rng is not None else 0, seed, cycle,
+            first, _ptr(sample), _ptr(flags), _ptr(margin))
+    if per is None:
+        rc = _load().uno_ref_filter_softmax(_ptr(a), code, rows, vocab, vocab, rows_per_request,
+                                            float(temperature), int(top_k), float(top_p), *tail)
+    else:
+        T, K, P, oc = per
+        rc = _load().uno_ref_filter_softmax_params(_ptr(a), code, rows, vocab, vocab, rows_per_request,
+                                                   _ptr(T), _ptr(K), _ptr(P), oc, *tail)
     _check(rc, "filter_softmax")
     out = dict(ids=ids, probs=probs, count=count, flags=flags, margin=margin)
     if dense:
@@ -194,8 +255,9 @@ def filter_softmax(logits, dtype, temperature, top_k, top_p, *, rows_per_request
 
 
 def linear_verify(target_logits, dtype, R, B, temperature, top_k, top_p, draft_ids, q_ids, q_probs,
-                  q_count, rng):
+                  q_count, rng, order="topk_first"):
     """Linear rejection sampling; target_logits [R*(B+1), vocab]."""
+    per = _per_request(temperature, top_k, top_p, order, R)
     a, code = _logits(target_logits, dtype)
     vocab = a.shape[-1]
     assert a.size == R * (B + 1) * vocab
@@ -210,10 +272,15 @@ def linear_verify(target_logits, dtype, R, B, temperature, top_k, top_p, draft_i
     flags = np.empty(R, dtype=np.uint32)
     margin = np.empty(R, dtype=np.float64)
     seed, cycle, first = _rng(rng)
-    rc = _load().uno_ref_linear_verify(_ptr(a), code, R, B, vocab, float(temperature), int(top_k),
-                                       float(top_p), _ptr(d), _ptr(qi), _ptr(qp), _ptr(qc), q_cap,
-                                       seed, cycle, first, _ptr(toks), _ptr(acc), _ptr(ntok),
-                                       _ptr(flags), _ptr(margin))
+    tail = (_ptr(d), _ptr(qi), _ptr(qp), _ptr(qc), q_cap, seed, cycle, first, _ptr(toks), _ptr(acc),
+            _ptr(ntok), _ptr(flags), _ptr(margin))
+    if per is None:
+        rc = _load().uno_ref_linear_verify(_ptr(a), code, R, B, vocab, float(temperature), int(top_k),
+                                           float(top_p), *tail)
+    else:
+        T, K, P, oc = per
+        rc = _load().uno_ref_linear_verify_params(_ptr(a), code, R, B, vocab, _ptr(T), _ptr(K), _ptr(P), oc,
+                                                  *tail)
     _check(rc, "linear_verify")
     return dict(tokens=toks, accept_len=acc, num_tokens=ntok, flags=flags, margin=margin)
 
@@ -235,8 +302,9 @@ def tree_topk_expand(q_ids, q_probs, q_count, R, B, K, V):
 
 
 def tree_verify(target_logits, dtype, R, B, V, temperature, top_k, top_p, node_token, node_parent,
-                num_nodes, rng):
+                num_nodes, rng, order="topk_first"):
     """Target-only tree verification; target_logits [R*V, vocab]."""
+    per = _per_request(temperature, top_k, top_p, order, R)
     a, code = _logits(target_logits, dtype)
     vocab = a.shape[-1]
     assert a.size == R * V * vocab
@@ -250,10 +318,40 @@ def tree_verify(target_logits, dtype, R, B, V, temperature, top_k, top_p, node_t
     flags = np.empty(R, dtype=np.uint32)
     margin = np.empty(R, dtype=np.float64)
     seed, cycle, first = _rng(rng)
-    rc = _load().uno_ref_tree_verify(_ptr(a), code, R, B, V, vocab, float(temperature), int(top_k),
-                                     float(top_p), _ptr(tk), _ptr(pa), _ptr(nn), seed, cycle, first,
-                                     _ptr(toks), _ptr(acc), _ptr(ntok), _ptr(path), _ptr(flags),
-                                     _ptr(margin))
+    tail = (_ptr(tk), _ptr(pa), _ptr(nn), seed, cycle, first, _ptr(toks), _ptr(acc), _ptr(ntok), _ptr(path),
+            _ptr(flags), _ptr(margin))
+    if per is None:
+        rc = _load().uno_ref_tree_verify(_ptr(a), code, R, B, V, vocab, float(temperature), int(top_k),
+                                         float(top_p), *tail)
+    else:
+        T, K, P, oc = per
+        rc = _load().uno_ref_tree_verify_params(_ptr(a), code, R, B, V, vocab, _ptr(T), _ptr(K), _ptr(P), oc,
+                                                *tail)
     _check(rc, "tree_verify")
     return dict(tokens=toks, accept_len=acc, num_tokens=ntok, path_nodes=path, flags=flags,
                 margin=margin)
+
+
+def linear_cycle(draft_logits, target_logits, dtype, R, B, temperature, top_k, top_p, rng,
+                 order="topk_first"):
+    """One linear cycle in the two-pass layout: draft_logits and target_logits
+    [R*B, vocab] each (draft row 0 of a request is the base-weights row);
+    returns tokens [R, B+1], accept_len (tokens emitted), num_correct_drafts,
+    flags and margin."""
+    d, code = _logits(draft_logits, dtype)
+    t, code_t = _logits(target_logits, dtype)
+    vocab = d.shape[-1]
+    assert code == code_t and d.size == R * B * vocab and t.size == R * B * vocab
+    oc = _order_code(order)
+    T, K, P = _param_arrays(temperature, top_k, top_p, R)
+    toks = np.empty((R, B + 1), dtype=np.int32)
+    acc = np.empty(R, dtype=np.int32)
+    ncd = np.empty(R, dtype=np.int32)
+    flags = np.empty(R, dtype=np.uint32)
+    margin = np.empty(R, dtype=np.float64)
+    seed, cycle, first = _rng(rng)
+    rc = _load().uno_ref_linear_cycle(_ptr(d), _ptr(t), code, R, B, vocab, _ptr(T), _ptr(K), _ptr(P), oc,
+                                      seed, cycle, first, _ptr(toks), _ptr(acc), _ptr(ncd), _ptr(flags),
+                                      _ptr(margin))
+    _check(rc, "linear_cycle")
+    return dict(tokens=toks, accept_len=acc, num_correct_drafts=ncd, flags=flags, margin=margin)

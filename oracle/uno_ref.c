@@ -44,6 +44,12 @@ enum { DRAW_PROPOSAL = 0, DRAW_ACCEPT = 1, DRAW_RESIDUAL = 2, DRAW_TARGET = 3 };
 #define FLAG_DRAFT_NOT_IN_SUPPORT 2u /* draft token has q = 0: rejected w.p. 1 */
 #define FLAG_RESIDUAL_EMPTY 4u       /* max(0, p - q) summed to 0: sampled p */
 
+/* Filter order.  TOPK_FIRST: the top-p cut is taken on the top-k set
+ * renormalised (the speculative-decoding convention UNO follows).  JOINT: the
+ * top-p cut is taken on the full-vocabulary softmax (the order of the regular
+ * autoregressive sampler the review asks UNO to align with). */
+enum { ORDER_TOPK_FIRST = 0, ORDER_JOINT = 1 };
+
 /* Return codes. */
 enum { REF_OK = 0, REF_ERR_INVALID_ARG = 1, REF_ERR_UNSUPPORTED = 2, REF_ERR_NOMEM = 5 };
 
@@ -133,8 +139,12 @@ static double min_d(double a, double b) { return a < b ? a : b; }
  * [UNO PR, review thread on the filter order]: UNO keeps the top-k tokens,
  * renormalises over them, and applies the top-p cut to that renormalised
  * distribution (the speculative-decoding convention), so the full-vocabulary
- * softmax is never formed.  [eval guide, run_math_eval 全参数详解]: top_k > 0,
- * top_p in (0, 1], temperature >= 0.
+ * softmax is never formed.  The same thread names the regular sampler's
+ * "joint" order, where the top-p cut is computed from the full softmax; with
+ * order = ORDER_JOINT step 4 divides by the sum over every finite token
+ * instead (top-k still bounds the kept set, and the kept weights are still
+ * renormalised among themselves in step 6).  [eval guide, run_math_eval
+ * 全参数详解]: top_k > 0, top_p in (0, 1], temperature >= 0.
  *
  * Steps, in order:
  *  1. a NaN or +inf logit, or a row with no finite logit, makes the row
@@ -143,7 +153,8 @@ static double min_d(double a, double b) { return a < b ? a : b; }
  *     k' = min(top_k, #finite);
  *  3. temperature 0 is greedy: the first entry alone, probability 1;
  *  4. otherwise w_j = exp((l_j - l_0) / T), S = sum_j w_j (in that order),
- *     P_j = w_j / S;
+ *     P_j = w_j / S; under the joint order S also adds, in the same order,
+ *     the weights of the finite tokens beyond the first k';
  *  5. top-p: walk in that order with the mass m accumulated before j; keep j
  *     when j = 0 or m < top_p, stop at the first j that fails; top_p >= 1
  *     keeps all k';
@@ -153,7 +164,7 @@ static double min_d(double a, double b) { return a < b ? a : b; }
  * comparisons made (the distance of that integer decision from its flip).
  * ===================================================================== */
 static int filter_row(const void* row, int dtype, int64_t vocab, double T, int32_t top_k, double top_p,
-                      int32_t* ids, float* probs, uint32_t* flags, double* margin, int* nomem)
+                      int order, int32_t* ids, float* probs, uint32_t* flags, double* margin, int* nomem)
 {
     *margin = INFINITY;
     ref_entry* e = (ref_entry*)malloc((size_t)(vocab > 0 ? vocab : 1) * sizeof(ref_entry));
@@ -195,6 +206,8 @@ static int filter_row(const void* row, int dtype, int64_t vocab, double T, int32
         for (int64_t j = 0; j < kk; ++j) w[j] = exp(((double)e[j].v - (double)e[0].v) / T);
         double S = 0.0;
         for (int64_t j = 0; j < kk; ++j) S += w[j];
+        if (order == ORDER_JOINT)
+            for (int64_t j = kk; j < n; ++j) S += exp(((double)e[j].v - (double)e[0].v) / T);
         if (top_p >= 1.0) {
             kept = kk;
         } else {
@@ -284,6 +297,46 @@ static int check_params(float temperature, int32_t top_k, float top_p)
     return 1;
 }
 
+/* Sampling parameters of a call: request r uses temperature[r * stride],
+ * top_k[r * stride] and top_p[r * stride] (stride 0 gives every request the
+ * same values), and every row of the call is filtered in one order. */
+typedef struct {
+    const float* temperature;
+    const int32_t* top_k;
+    const float* top_p;
+    int64_t stride;
+    int order;
+} ref_params;
+
+static double sp_T(const ref_params* sp, int64_t r) { return (double)sp->temperature[r * sp->stride]; }
+static int32_t sp_k(const ref_params* sp, int64_t r) { return sp->top_k[r * sp->stride]; }
+static double sp_p(const ref_params* sp, int64_t r) { return (double)sp->top_p[r * sp->stride]; }
+
+/* Check the parameters of requests 0 .. nreq-1 (just entry 0 when stride is
+ * 0) and the order; *need receives the largest min(top_k, vocab), the
+ * compact width a row of the call can fill. */
+static int check_call_params(const ref_params* sp, int64_t nreq, int64_t vocab, int32_t* need)
+{
+    if (!sp->temperature || !sp->top_k || !sp->top_p) return 0;
+    if (sp->order != ORDER_TOPK_FIRST && sp->order != ORDER_JOINT) return 0;
+    int64_t n = sp->stride == 0 ? 1 : nreq;
+    int64_t most = 0;
+    for (int64_t r = 0; r < n; ++r) {
+        if (!check_params(sp->temperature[r * sp->stride], sp->top_k[r * sp->stride], sp->top_p[r * sp->stride]))
+            return 0;
+        int64_t k = sp->top_k[r * sp->stride] < vocab ? sp->top_k[r * sp->stride] : vocab;
+        if (k > most) most = k;
+    }
+    *need = (int32_t)most;
+    return 1;
+}
+
+static ref_params scalar_params(const float* temperature, const int32_t* top_k, const float* top_p)
+{
+    ref_params sp = {temperature, top_k, top_p, 0, ORDER_TOPK_FIRST};
+    return sp;
+}
+
 /* =====================================================================
  * uno_ref_filter_softmax: filter every row (see filter_row) and, when
  * has_rng, draw one token per row from the stored compact distribution by
@@ -298,19 +351,25 @@ static int check_params(float temperature, int32_t top_k, float top_p)
  * rows x cap; out_count, out_flags: rows; out_dense (nullable): rows x vocab;
  * out_sample (nullable): rows; out_margin (nullable): rows, the smaller of
  * the top-p and the draw margins.
+ *
+ * uno_ref_filter_softmax_params is the same with one temperature, top_k and
+ * top_p per request (arrays of ceil(rows / rows_per_request) entries) and a
+ * filter order (ORDER_TOPK_FIRST or ORDER_JOINT); cap must hold the largest
+ * min(top_k, vocab) of the call.
  * ===================================================================== */
-int uno_ref_filter_softmax(const void* logits, int dtype, int64_t rows, int64_t vocab, int64_t row_stride,
-                           int32_t rows_per_request, float temperature, int32_t top_k, float top_p, int32_t cap,
-                           int32_t* out_ids, float* out_probs, int32_t* out_count, float* out_dense, int has_rng,
-                           uint64_t seed, uint32_t cycle, uint32_t first_request, int32_t* out_sample,
-                           uint32_t* out_flags, double* out_margin)
+static int filter_softmax_impl(const void* logits, int dtype, int64_t rows, int64_t vocab, int64_t row_stride,
+                               int32_t rows_per_request, const ref_params* sp, int32_t cap, int32_t* out_ids,
+                               float* out_probs, int32_t* out_count, float* out_dense, int has_rng, uint64_t seed,
+                               uint32_t cycle, uint32_t first_request, int32_t* out_sample, uint32_t* out_flags,
+                               double* out_margin)
 {
     if (!logits || !out_ids || !out_probs || !out_count || !out_flags) return REF_ERR_INVALID_ARG;
     if (rows < 0 || vocab <= 0 || row_stride < vocab || rows_per_request < 1) return REF_ERR_INVALID_ARG;
     if (dtype != REF_F32 && dtype != REF_BF16) return REF_ERR_INVALID_ARG;
-    if (!check_params(temperature, top_k, top_p)) return REF_ERR_INVALID_ARG;
+    int32_t need;
+    if (!check_call_params(sp, (rows + rows_per_request - 1) / rows_per_request, vocab, &need))
+        return REF_ERR_INVALID_ARG;
     if (has_rng && !out_sample) return REF_ERR_INVALID_ARG;
-    int64_t need = top_k < vocab ? top_k : vocab;
     if (cap < need) return REF_ERR_UNSUPPORTED;
     size_t esz = dtype == REF_F32 ? 4 : 2;
     for (int64_t r = 0; r < rows; ++r) {
@@ -320,8 +379,9 @@ int uno_ref_filter_softmax(const void* logits, int dtype, int64_t rows, int64_t 
         uint32_t flags = 0;
         double m_top = INFINITY, m_draw = INFINITY;
         int nomem = 0;
-        int cnt = filter_row(row, dtype, vocab, (double)temperature, top_k, (double)top_p, ids, probs, &flags,
-                             &m_top, &nomem);
+        int64_t rq = r / rows_per_request;
+        int cnt = filter_row(row, dtype, vocab, sp_T(sp, rq), sp_k(sp, rq), sp_p(sp, rq), sp->order, ids, probs,
+                             &flags, &m_top, &nomem);
         if (nomem) return REF_ERR_NOMEM;
         for (int j = cnt; j < cap; ++j) {
             ids[j] = -1;
@@ -353,6 +413,31 @@ int uno_ref_filter_softmax(const void* logits, int dtype, int64_t rows, int64_t 
     return REF_OK;
 }
 
+int uno_ref_filter_softmax(const void* logits, int dtype, int64_t rows, int64_t vocab, int64_t row_stride,
+                           int32_t rows_per_request, float temperature, int32_t top_k, float top_p, int32_t cap,
+                           int32_t* out_ids, float* out_probs, int32_t* out_count, float* out_dense, int has_rng,
+                           uint64_t seed, uint32_t cycle, uint32_t first_request, int32_t* out_sample,
+                           uint32_t* out_flags, double* out_margin)
+{
+    ref_params sp = scalar_params(&temperature, &top_k, &top_p);
+    return filter_softmax_impl(logits, dtype, rows, vocab, row_stride, rows_per_request, &sp, cap, out_ids,
+                               out_probs, out_count, out_dense, has_rng, seed, cycle, first_request, out_sample,
+                               out_flags, out_margin);
+}
+
+int uno_ref_filter_softmax_params(const void* logits, int dtype, int64_t rows, int64_t vocab, int64_t row_stride,
+                                  int32_t rows_per_request, const float* temperature, const int32_t* top_k,
+                                  const float* top_p, int order, int32_t cap, int32_t* out_ids, float* out_probs,
+                                  int32_t* out_count, float* out_dense, int has_rng, uint64_t seed, uint32_t cycle,
+                                  uint32_t first_request, int32_t* out_sample, uint32_t* out_flags,
+                                  double* out_margin)
+{
+    ref_params sp = {temperature, top_k, top_p, 1, order};
+    return filter_softmax_impl(logits, dtype, rows, vocab, row_stride, rows_per_request, &sp, cap, out_ids,
+                               out_probs, out_count, out_dense, has_rng, seed, cycle, first_request, out_sample,
+                               out_flags, out_margin);
+}
+
 /* =====================================================================
  * uno_ref_linear_verify: linear-mode rejection sampling for R requests.
  *
@@ -377,22 +462,24 @@ int uno_ref_filter_softmax(const void* logits, int dtype, int64_t rows, int64_t 
  * target_logits: R x (B+1) x vocab; draft_ids: R x B; q_*: (R*B) x q_cap;
  * outputs: out_tokens R x (B+1) (unused slots -1), out_accept_len,
  * out_num_tokens, out_flags, out_margin (nullable): R.
+ *
+ * uno_ref_linear_verify_params is the same with per-request sampling
+ * parameters (arrays of R) and a filter order for the target rows.
  * ===================================================================== */
-int uno_ref_linear_verify(const void* target_logits, int dtype, int32_t R, int32_t B, int64_t vocab,
-                          float temperature, int32_t top_k, float top_p, const int32_t* draft_ids,
-                          const int32_t* q_ids, const float* q_probs, const int32_t* q_count, int32_t q_cap,
-                          uint64_t seed, uint32_t cycle, uint32_t first_request, int32_t* out_tokens,
-                          int32_t* out_accept_len, int32_t* out_num_tokens, uint32_t* out_flags,
-                          double* out_margin)
+static int linear_verify_impl(const void* target_logits, int dtype, int32_t R, int32_t B, int64_t vocab,
+                              const ref_params* sp, const int32_t* draft_ids, const int32_t* q_ids,
+                              const float* q_probs, const int32_t* q_count, int32_t q_cap, uint64_t seed,
+                              uint32_t cycle, uint32_t first_request, int32_t* out_tokens, int32_t* out_accept_len,
+                              int32_t* out_num_tokens, uint32_t* out_flags, double* out_margin)
 {
     if (!target_logits || !draft_ids || !q_ids || !q_probs || !q_count || !out_tokens || !out_accept_len ||
         !out_num_tokens || !out_flags)
         return REF_ERR_INVALID_ARG;
     if (R < 0 || B < 1 || vocab <= 0 || q_cap < 1) return REF_ERR_INVALID_ARG;
     if (dtype != REF_F32 && dtype != REF_BF16) return REF_ERR_INVALID_ARG;
-    if (!check_params(temperature, top_k, top_p)) return REF_ERR_INVALID_ARG;
-    int64_t need = top_k < vocab ? top_k : vocab;
-    int32_t cap = (int32_t)need;
+    int32_t cap;
+    if (!check_call_params(sp, R, vocab, &cap)) return REF_ERR_INVALID_ARG;
+    if (cap < 1) cap = 1;
     size_t esz = dtype == REF_F32 ? 4 : 2;
 
     int32_t* p_ids = (int32_t*)malloc((size_t)(B + 1) * (size_t)cap * sizeof(int32_t));
@@ -411,7 +498,7 @@ int uno_ref_linear_verify(const void* target_logits, int dtype, int32_t R, int32
             const char* row = (const char*)target_logits + ((size_t)r * (size_t)(B + 1) + (size_t)i) * (size_t)vocab * esz;
             double m_top;
             int nomem = 0;
-            p_cnt[i] = filter_row(row, dtype, vocab, (double)temperature, top_k, (double)top_p,
+            p_cnt[i] = filter_row(row, dtype, vocab, sp_T(sp, r), sp_k(sp, r), sp_p(sp, r), sp->order,
                                   p_ids + (size_t)i * (size_t)cap, p_probs + (size_t)i * (size_t)cap, &flags,
                                   &m_top, &nomem);
             if (nomem) {
@@ -491,6 +578,192 @@ int uno_ref_linear_verify(const void* target_logits, int dtype, int32_t R, int32
     }
     free(p_ids); free(p_probs); free(p_cnt); free(wts);
     return REF_OK;
+}
+
+int uno_ref_linear_verify(const void* target_logits, int dtype, int32_t R, int32_t B, int64_t vocab,
+                          float temperature, int32_t top_k, float top_p, const int32_t* draft_ids,
+                          const int32_t* q_ids, const float* q_probs, const int32_t* q_count, int32_t q_cap,
+                          uint64_t seed, uint32_t cycle, uint32_t first_request, int32_t* out_tokens,
+                          int32_t* out_accept_len, int32_t* out_num_tokens, uint32_t* out_flags,
+                          double* out_margin)
+{
+    ref_params sp = scalar_params(&temperature, &top_k, &top_p);
+    return linear_verify_impl(target_logits, dtype, R, B, vocab, &sp, draft_ids, q_ids, q_probs, q_count, q_cap,
+                              seed, cycle, first_request, out_tokens, out_accept_len, out_num_tokens, out_flags,
+                              out_margin);
+}
+
+int uno_ref_linear_verify_params(const void* target_logits, int dtype, int32_t R, int32_t B, int64_t vocab,
+                                 const float* temperature, const int32_t* top_k, const float* top_p, int order,
+                                 const int32_t* draft_ids, const int32_t* q_ids, const float* q_probs,
+                                 const int32_t* q_count, int32_t q_cap, uint64_t seed, uint32_t cycle,
+                                 uint32_t first_request, int32_t* out_tokens, int32_t* out_accept_len,
+                                 int32_t* out_num_tokens, uint32_t* out_flags, double* out_margin)
+{
+    ref_params sp = {temperature, top_k, top_p, 1, order};
+    return linear_verify_impl(target_logits, dtype, R, B, vocab, &sp, draft_ids, q_ids, q_probs, q_count, q_cap,
+                              seed, cycle, first_request, out_tokens, out_accept_len, out_num_tokens, out_flags,
+                              out_margin);
+}
+
+/* =====================================================================
+ * uno_ref_linear_cycle: one linear decoding cycle in the layout the pages
+ * give UNO's two forward passes.
+ *
+ * [UNO PR, Motivation]: a cycle runs two target-model forward passes; the
+ * diffusion-pathway pass yields the first output token and a block of draft
+ * proposals, the AR-pathway pass verifies the proposals.  [eval guide,
+ * 单模型双前向架构]: of a request's B draft rows the first runs on the base
+ * weights and the other B - 1 on the UNO adapter.  [UNO PR, Modifications,
+ * and the review thread on the token counters]: the scheduler slices B + 1
+ * output rows per request, num_correct_drafts = accept_len - 2 counts the
+ * accepted proposals, and a request adds num_correct_drafts + 2 generated
+ * tokens (two tokens of a cycle are not drafts).
+ *
+ * Reading taken (the pages print no formula; the decisions are those of
+ * uno_ref_linear_verify):
+ *   draft row i (i = 0 .. B-1) is filtered and x_i drawn from it by inverse
+ *   CDF (ascending ids) with u_PROPOSAL(r, i);
+ *   x_0, drawn from the base-weights row, is output token 0 with no test;
+ *   target row i (i = 0 .. B-1) is the AR pathway's distribution of output
+ *   token i + 1, i.e. given x_0 .. x_i;
+ *   for i = 1 .. B-1: a = q_i(x_i); a = 0 rejects w.p. 1 (flagged); else
+ *   accept iff u_ACCEPT(r, i) * a < p_{i-1}(x_i); on the first rejection draw
+ *   y from normalise(max(0, p_{i-1} - q_i)) over supp p_{i-1} with
+ *   u_RESIDUAL(r, i) (p_{i-1} itself if that sums to 0, flagged), emit y as
+ *   token i and stop; if every proposal is accepted, draw token B from
+ *   target row B-1 with u_TARGET(r, B).
+ * accept_len = the number of tokens emitted (at most B + 1);
+ * num_correct_drafts = the number of accepted proposals, which is
+ * accept_len - 2 whenever every row reached is finite.  A non-finite draft
+ * row 0 emits nothing; a non-finite draft row i >= 1 has no support
+ * (x_i = -1) and is rejected; a non-finite target row that is reached stops
+ * the request without a further token.  Every non-finite row of the request,
+ * draft or target, sets NONFINITE_ROW.
+ *
+ * draft_logits and target_logits: R x B x vocab each; parameters: one per
+ * request (arrays of R) and one filter order for the rows of both passes;
+ * outputs: out_tokens R x (B+1) (unused slots -1), out_accept_len,
+ * out_num_correct_drafts, out_flags, out_margin (nullable): R.
+ * ===================================================================== */
+int uno_ref_linear_cycle(const void* draft_logits, const void* target_logits, int dtype, int32_t R, int32_t B,
+                         int64_t vocab, const float* temperature, const int32_t* top_k, const float* top_p,
+                         int order, uint64_t seed, uint32_t cycle, uint32_t first_request, int32_t* out_tokens,
+                         int32_t* out_accept_len, int32_t* out_num_correct_drafts, uint32_t* out_flags,
+                         double* out_margin)
+{
+    if (!draft_logits || !target_logits || !out_tokens || !out_accept_len || !out_num_correct_drafts || !out_flags)
+        return REF_ERR_INVALID_ARG;
+    if (R < 0 || B < 1 || vocab <= 0) return REF_ERR_INVALID_ARG;
+    if (dtype != REF_F32 && dtype != REF_BF16) return REF_ERR_INVALID_ARG;
+    ref_params sp = {temperature, top_k, top_p, 1, order};
+    int32_t cap;
+    if (!check_call_params(&sp, R, vocab, &cap)) return REF_ERR_INVALID_ARG;
+    if (cap < 1) cap = 1;
+    size_t esz = dtype == REF_F32 ? 4 : 2;
+    size_t n = (size_t)B * (size_t)cap;
+    int32_t* q_ids = (int32_t*)malloc(n * sizeof(int32_t));
+    float* q_pr = (float*)malloc(n * sizeof(float));
+    int32_t* p_ids = (int32_t*)malloc(n * sizeof(int32_t));
+    float* p_pr = (float*)malloc(n * sizeof(float));
+    int* q_cnt = (int*)malloc((size_t)B * sizeof(int));
+    int* p_cnt = (int*)malloc((size_t)B * sizeof(int));
+    int32_t* x = (int32_t*)malloc((size_t)B * sizeof(int32_t));
+    double* wts = (double*)malloc((size_t)cap * sizeof(double));
+    int nomem = !q_ids || !q_pr || !p_ids || !p_pr || !q_cnt || !p_cnt || !x || !wts;
+    for (int32_t r = 0; r < R && !nomem; ++r) {
+        uint32_t flags = 0;
+        double margin = INFINITY, m;
+        const uint32_t req = first_request + (uint32_t)r;
+        /* the draft pass: filter the B rows and draw x_0 .. x_{B-1} */
+        for (int32_t i = 0; i < B && !nomem; ++i) {
+            const char* row = (const char*)draft_logits + ((size_t)r * (size_t)B + (size_t)i) * (size_t)vocab * esz;
+            int32_t* ids = q_ids + (size_t)i * (size_t)cap;
+            float* pr = q_pr + (size_t)i * (size_t)cap;
+            q_cnt[i] = filter_row(row, dtype, vocab, sp_T(&sp, r), sp_k(&sp, r), sp_p(&sp, r), order, ids, pr, &flags,
+                                  &m, &nomem);
+            margin = min_d(margin, m);
+            x[i] = -1;
+            if (q_cnt[i] > 0) {
+                for (int j = 0; j < q_cnt[i]; ++j) wts[j] = (double)pr[j];
+                int pick = inv_cdf(wts, q_cnt[i], uno_ref_uniform(seed, req, (uint32_t)i, DRAW_PROPOSAL, cycle), &m);
+                margin = min_d(margin, m);
+                x[i] = pick >= 0 ? ids[pick] : -1;
+            }
+        }
+        /* the verify pass: filter the B target rows */
+        for (int32_t i = 0; i < B && !nomem; ++i) {
+            const char* row = (const char*)target_logits + ((size_t)r * (size_t)B + (size_t)i) * (size_t)vocab * esz;
+            p_cnt[i] = filter_row(row, dtype, vocab, sp_T(&sp, r), sp_k(&sp, r), sp_p(&sp, r), order,
+                                  p_ids + (size_t)i * (size_t)cap, p_pr + (size_t)i * (size_t)cap, &flags, &m,
+                                  &nomem);
+            margin = min_d(margin, m);
+        }
+        if (nomem) break;
+        int32_t* toks = out_tokens + (size_t)r * (size_t)(B + 1);
+        for (int32_t t = 0; t <= B; ++t) toks[t] = -1;
+        int32_t emitted = 0, correct = 0;
+        if (q_cnt[0] > 0) {
+            toks[0] = x[0]; /* the base-weights token: emitted untested */
+            emitted = 1;
+            int stopped = 0;
+            for (int32_t i = 1; i < B; ++i) {
+                const int32_t* pi_ids = p_ids + (size_t)(i - 1) * (size_t)cap;
+                const float* pi_pr = p_pr + (size_t)(i - 1) * (size_t)cap;
+                const int32_t* qi_ids = q_ids + (size_t)i * (size_t)cap;
+                const float* qi_pr = q_pr + (size_t)i * (size_t)cap;
+                if (p_cnt[i - 1] == 0) { /* a non-finite target row is reached */
+                    stopped = 1;
+                    break;
+                }
+                double a = x[i] >= 0 ? lookup_prob(qi_ids, qi_pr, q_cnt[i], x[i]) : 0.0;
+                double px = x[i] >= 0 ? lookup_prob(pi_ids, pi_pr, p_cnt[i - 1], x[i]) : 0.0;
+                if (a > 0.0) {
+                    double u = uno_ref_uniform(seed, req, (uint32_t)i, DRAW_ACCEPT, cycle);
+                    margin = min_d(margin, fabs(u * a - px) / a);
+                    if (u * a < px) {
+                        toks[i] = x[i];
+                        ++emitted;
+                        ++correct;
+                        continue;
+                    }
+                } else {
+                    flags |= FLAG_DRAFT_NOT_IN_SUPPORT;
+                }
+                double tot = 0.0;
+                for (int j = 0; j < p_cnt[i - 1]; ++j) {
+                    double d = (double)pi_pr[j] - lookup_prob(qi_ids, qi_pr, q_cnt[i], pi_ids[j]);
+                    wts[j] = d > 0.0 ? d : 0.0;
+                    tot += wts[j];
+                }
+                if (!(tot > 0.0)) {
+                    flags |= FLAG_RESIDUAL_EMPTY;
+                    for (int j = 0; j < p_cnt[i - 1]; ++j) wts[j] = (double)pi_pr[j];
+                }
+                int pick = inv_cdf(wts, p_cnt[i - 1], uno_ref_uniform(seed, req, (uint32_t)i, DRAW_RESIDUAL, cycle), &m);
+                margin = min_d(margin, m);
+                toks[i] = pick >= 0 ? pi_ids[pick] : -1;
+                ++emitted;
+                stopped = 1;
+                break;
+            }
+            if (!stopped && p_cnt[B - 1] > 0) { /* every proposal accepted: the bonus token */
+                const int32_t* pb_ids = p_ids + (size_t)(B - 1) * (size_t)cap;
+                const float* pb_pr = p_pr + (size_t)(B - 1) * (size_t)cap;
+                for (int j = 0; j < p_cnt[B - 1]; ++j) wts[j] = (double)pb_pr[j];
+                int pick = inv_cdf(wts, p_cnt[B - 1], uno_ref_uniform(seed, req, (uint32_t)B, DRAW_TARGET, cycle), &m);
+                margin = min_d(margin, m);
+                toks[B] = pick >= 0 ? pb_ids[pick] : -1;
+                ++emitted;
+            }
+        }
+        out_accept_len[r] = emitted;
+        out_num_correct_drafts[r] = correct;
+        out_flags[r] = flags;
+        if (out_margin) out_margin[r] = margin;
+    }
+    free(q_ids); free(q_pr); free(p_ids); free(p_pr); free(q_cnt); free(p_cnt); free(x); free(wts);
+    return nomem ? REF_ERR_NOMEM : REF_OK;
 }
 
 /* =====================================================================
@@ -642,12 +915,15 @@ int uno_ref_tree_topk_expand(const int32_t* q_ids, const float* q_probs, const i
  * target_logits: R x V x vocab (one row per node); node_*: R x V;
  * outputs R x (B+1) for tokens and path_nodes (unused slots -1), and R for
  * accept_len, num_tokens, flags, margin (nullable).
+ *
+ * uno_ref_tree_verify_params is the same with per-request sampling
+ * parameters (arrays of R) and a filter order for the node rows.
  * ===================================================================== */
-int uno_ref_tree_verify(const void* target_logits, int dtype, int32_t R, int32_t B, int32_t V, int64_t vocab,
-                        float temperature, int32_t top_k, float top_p, const int32_t* node_token,
-                        const int32_t* node_parent, const int32_t* num_nodes, uint64_t seed, uint32_t cycle,
-                        uint32_t first_request, int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
-                        int32_t* out_path_nodes, uint32_t* out_flags, double* out_margin)
+static int tree_verify_impl(const void* target_logits, int dtype, int32_t R, int32_t B, int32_t V, int64_t vocab,
+                            const ref_params* sp, const int32_t* node_token, const int32_t* node_parent,
+                            const int32_t* num_nodes, uint64_t seed, uint32_t cycle, uint32_t first_request,
+                            int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                            int32_t* out_path_nodes, uint32_t* out_flags, double* out_margin)
 {
     if (!target_logits || !node_token || !node_parent || !num_nodes || !out_tokens || !out_accept_len ||
         !out_num_tokens || !out_path_nodes || !out_flags)
@@ -655,9 +931,9 @@ int uno_ref_tree_verify(const void* target_logits, int dtype, int32_t R, int32_t
     if (R < 0 || B < 1 || V < 1 || vocab <= 0) return REF_ERR_INVALID_ARG;
     if (V < B || V > 128) return REF_ERR_INVALID_ARG;
     if (dtype != REF_F32 && dtype != REF_BF16) return REF_ERR_INVALID_ARG;
-    if (!check_params(temperature, top_k, top_p)) return REF_ERR_INVALID_ARG;
-    int64_t need = top_k < vocab ? top_k : vocab;
-    int32_t cap = (int32_t)need;
+    int32_t cap;
+    if (!check_call_params(sp, R, vocab, &cap)) return REF_ERR_INVALID_ARG;
+    if (cap < 1) cap = 1;
     size_t esz = dtype == REF_F32 ? 4 : 2;
     int32_t* ids = (int32_t*)malloc((size_t)cap * sizeof(int32_t));
     float* pr = (float*)malloc((size_t)cap * sizeof(float));
@@ -686,7 +962,8 @@ int uno_ref_tree_verify(const void* target_logits, int dtype, int32_t R, int32_t
             uint32_t f = 0;
             double mt;
             int nomem = 0;
-            int c = filter_row(row, dtype, vocab, (double)temperature, top_k, (double)top_p, ids, pr, &f, &mt, &nomem);
+            int c = filter_row(row, dtype, vocab, sp_T(sp, r), sp_k(sp, r), sp_p(sp, r), sp->order, ids, pr, &f, &mt,
+                               &nomem);
             if (nomem) {
                 free(ids); free(pr); free(wts);
                 return REF_ERR_NOMEM;
@@ -701,7 +978,8 @@ int uno_ref_tree_verify(const void* target_logits, int dtype, int32_t R, int32_t
             uint32_t f = 0;
             double mt;
             int nomem = 0;
-            int c = filter_row(row, dtype, vocab, (double)temperature, top_k, (double)top_p, ids, pr, &f, &mt, &nomem);
+            int c = filter_row(row, dtype, vocab, sp_T(sp, r), sp_k(sp, r), sp_p(sp, r), sp->order, ids, pr, &f, &mt,
+                               &nomem);
             if (nomem) {
                 free(ids); free(pr); free(wts);
                 return REF_ERR_NOMEM;
@@ -741,4 +1019,29 @@ int uno_ref_tree_verify(const void* target_logits, int dtype, int32_t R, int32_t
     }
     free(ids); free(pr); free(wts);
     return REF_OK;
+}
+
+int uno_ref_tree_verify(const void* target_logits, int dtype, int32_t R, int32_t B, int32_t V, int64_t vocab,
+                        float temperature, int32_t top_k, float top_p, const int32_t* node_token,
+                        const int32_t* node_parent, const int32_t* num_nodes, uint64_t seed, uint32_t cycle,
+                        uint32_t first_request, int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                        int32_t* out_path_nodes, uint32_t* out_flags, double* out_margin)
+{
+    ref_params sp = scalar_params(&temperature, &top_k, &top_p);
+    return tree_verify_impl(target_logits, dtype, R, B, V, vocab, &sp, node_token, node_parent, num_nodes, seed,
+                            cycle, first_request, out_tokens, out_accept_len, out_num_tokens, out_path_nodes,
+                            out_flags, out_margin);
+}
+
+int uno_ref_tree_verify_params(const void* target_logits, int dtype, int32_t R, int32_t B, int32_t V, int64_t vocab,
+                               const float* temperature, const int32_t* top_k, const float* top_p, int order,
+                               const int32_t* node_token, const int32_t* node_parent, const int32_t* num_nodes,
+                               uint64_t seed, uint32_t cycle, uint32_t first_request, int32_t* out_tokens,
+                               int32_t* out_accept_len, int32_t* out_num_tokens, int32_t* out_path_nodes,
+                               uint32_t* out_flags, double* out_margin)
+{
+    ref_params sp = {temperature, top_k, top_p, 1, order};
+    return tree_verify_impl(target_logits, dtype, R, B, V, vocab, &sp, node_token, node_parent, num_nodes, seed,
+                            cycle, first_request, out_tokens, out_accept_len, out_num_tokens, out_path_nodes,
+                            out_flags, out_margin);
 }

@@ -3,7 +3,9 @@
 These do not restate the oracle's code: top-k comes from ``numpy.lexsort``, the
 softmax from ``scipy.special.softmax``, the top-p cut from its defining
 property (the shortest prefix, in logit-descending order, whose renormalised
-top-k mass reaches top_p) via ``numpy.cumsum``/``searchsorted``.
+top-k mass reaches top_p) via ``numpy.cumsum``/``searchsorted``.  Under the
+"joint" order the prefix mass is read from the softmax of the whole row, and
+the kept prefix is then cut to the top-k.
 """
 from __future__ import annotations
 
@@ -15,16 +17,33 @@ def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def filtered_dist(logits: np.ndarray, temperature: float, top_k: int, top_p: float) -> np.ndarray:
+def _prefix_mass(l: np.ndarray, idx: np.ndarray, temperature: float, top_k: int, order: str) -> np.ndarray:
+    """Probabilities, in logit-descending order, whose running sum the top-p
+    cut reads: the renormalised top-k set, or the whole row's softmax."""
+    if order == "joint":
+        return special.softmax(l / temperature)[idx]
+    assert order == "topk_first", order
+    return special.softmax(l[idx[:min(top_k, l.size)]] / temperature)
+
+
+def filtered_dist(logits: np.ndarray, temperature: float, top_k: int, top_p: float,
+                  order: str = "topk_first") -> np.ndarray:
     """Dense filtered distribution of one finite row (float64, sums to 1)."""
     l = np.asarray(logits, dtype=np.float64)
     n = l.size
-    order = np.lexsort((np.arange(n), -l))  # logit desc, id asc
+    idx = np.lexsort((np.arange(n), -l))  # logit desc, id asc
     k = min(top_k, n)
-    top = order[:k]
+    top = idx[:k]
     out = np.zeros(n)
     if temperature == 0:
         out[top[0]] = 1.0
+        return out
+    if order == "joint" and top_p < 1.0:
+        c = np.cumsum(_prefix_mass(l, idx, temperature, top_k, order))
+        L = min(max(int(np.searchsorted(c, top_p, side="left")) + 1, 1), k)
+        top = idx[:L]
+        p = special.softmax(l[top] / temperature)
+        out[top] = p
         return out
     p = special.softmax(l[top] / temperature)
     if top_p < 1.0:
@@ -38,14 +57,15 @@ def filtered_dist(logits: np.ndarray, temperature: float, top_k: int, top_p: flo
     return out
 
 
-def top_p_margin(logits: np.ndarray, temperature: float, top_k: int, top_p: float) -> float:
+def top_p_margin(logits: np.ndarray, temperature: float, top_k: int, top_p: float,
+                 order: str = "topk_first") -> float:
     """Distance of the top-p cut from flipping (min |prefix mass - top_p|)."""
     l = np.asarray(logits, dtype=np.float64)
-    order = np.lexsort((np.arange(l.size), -l))
+    idx = np.lexsort((np.arange(l.size), -l))
     k = min(top_k, l.size)
     if temperature == 0 or top_p >= 1.0:
         return np.inf
-    p = special.softmax(l[order[:k]] / temperature)
+    p = _prefix_mass(l, idx, temperature, top_k, order)[:k]
     c = np.cumsum(p)[:-1]
     return float(np.min(np.abs(c - top_p))) if c.size else np.inf
 

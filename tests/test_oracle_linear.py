@@ -25,13 +25,13 @@ class TinyAR:
             for pre in itertools.product(range(vocab), repeat=L):
                 self.rows[pre] = (rng.standard_normal(vocab) * scale).astype(np.float32)
 
-    def dist(self, prefix, T, k, p):
-        return filtered_dist(self.rows[tuple(prefix)], T, k, p)
+    def dist(self, prefix, T, k, p, order="topk_first"):
+        return filtered_dist(self.rows[tuple(prefix)], T, k, p, order)
 
-    def seq_prob(self, seq, T, k, p):
+    def seq_prob(self, seq, T, k, p, order="topk_first"):
         pr = 1.0
         for t in range(len(seq)):
-            pr *= self.dist(seq[:t], T, k, p)[seq[t]]
+            pr *= self.dist(seq[:t], T, k, p, order)[seq[t]]
         return pr
 
 
