@@ -132,6 +132,30 @@ def _check(fn, status):
         raise UnoError(fn, status)
 
 
+# Shape checks run before anything touches a device: the kernels index these
+# arrays by the sizes passed alongside them, so a short array would be read
+# past its end.
+def _need(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _check_compact(q_ids, q_probs, q_count, rows):
+    """q_ids and q_probs [rows, cap] of the same shape; q_count [rows]."""
+    _need(q_ids.dim() == 2 and q_ids.shape[0] == rows and q_ids.shape[1] >= 1,
+          f"q_ids must be [{rows}, cap] (one compact row per draft position)")
+    _need(tuple(q_probs.shape) == tuple(q_ids.shape), "q_probs must have the shape of q_ids")
+    _need(q_count.numel() == rows, f"q_count must hold {rows} entries")
+
+
+def _check_linear(target_logits, draft_ids, q_ids, q_probs, q_count, R, B):
+    _need(R >= 1 and B >= 1, "R and B must be positive")
+    _need(target_logits.dim() >= 1 and target_logits.numel() == R * (B + 1) * target_logits.shape[-1],
+          "target_logits must hold R*(B+1) rows")
+    _need(draft_ids.numel() == R * B, "draft_ids must hold R*B tokens")
+    _check_compact(q_ids, q_probs, q_count, R * B)
+
+
 def _dev(t: torch.Tensor, device) -> torch.Tensor:
     return t if t.device == device else t.to(device, non_blocking=True)
 
@@ -160,11 +184,10 @@ def uno_filter_softmax(logits, *, temperature, top_k, top_p, rows_per_request=1,
     flags [rows] uint32 as int32, and sample [rows] when rng=(seed, cycle),
     dense [rows, vocab] when dense=True)."""
     lib = load_library()
+    _need(logits.dim() == 2 and logits.stride(1) == 1, "logits must be [rows, vocab] with unit inner stride")
     host = not logits.is_cuda
     device = _device_of(logits)
     x = _dev(logits, device)
-    if x.dim() != 2 or x.stride(1) != 1:
-        raise ValueError("logits must be [rows, vocab] with unit inner stride")
     rows, vocab = x.shape
     if cap is None:
         cap = min(int(top_k), vocab)
@@ -199,18 +222,15 @@ def uno_linear_verify(target_logits, draft_ids, q_ids, q_probs, q_count, *, R, B
     for the R*B draft rows.  Returns dict(tokens [R, B+1], accept_len,
     num_tokens, flags)."""
     lib = load_library()
+    _check_linear(target_logits, draft_ids, q_ids, q_probs, q_count, R, B)
     host = not target_logits.is_cuda
     device = _device_of(target_logits, draft_ids, q_ids)
     x = _dev(target_logits, device).contiguous()
     vocab = x.shape[-1]
-    if x.numel() != R * (B + 1) * vocab:
-        raise ValueError("target_logits must hold R*(B+1) rows")
     d = _dev(draft_ids, device).to(torch.int32).contiguous()
     qi = _dev(q_ids, device).to(torch.int32).contiguous()
     qp = _dev(q_probs, device).to(torch.float32).contiguous()
     qc = _dev(q_count, device).to(torch.int32).contiguous()
-    if d.numel() != R * B or qi.shape[0] != R * B or qc.numel() != R * B:
-        raise ValueError("draft_ids / q rows must cover R*B draft positions")
     stream = torch.cuda.current_stream(device)
     kw = dict(dtype=torch.int32, device=device)
     toks = torch.empty((R, B + 1), **kw)
@@ -233,13 +253,13 @@ def uno_tree_topk_expand(q_ids, q_probs, q_count, *, R, B, K, V):
     dict(node_token, node_parent, node_depth [R, V] int32, node_score [R, V]
     float32, num_nodes [R])."""
     lib = load_library()
+    _need(R >= 1 and B >= 1, "R and B must be positive")
+    _check_compact(q_ids, q_probs, q_count, R * B)
     host = not q_ids.is_cuda
     device = _device_of(q_ids)
     qi = _dev(q_ids, device).to(torch.int32).contiguous()
     qp = _dev(q_probs, device).to(torch.float32).contiguous()
     qc = _dev(q_count, device).to(torch.int32).contiguous()
-    if qi.shape[0] != R * B:
-        raise ValueError("q rows must cover R*B marginals")
     stream = torch.cuda.current_stream(device)
     kw = dict(dtype=torch.int32, device=device)
     tok = torch.empty((R, V), **kw)
@@ -259,12 +279,16 @@ def uno_tree_verify(target_logits, node_token, node_parent, num_nodes, *, R, B, 
     per node).  Returns dict(tokens [R, B+1], accept_len, num_tokens,
     path_nodes [R, B+1], flags)."""
     lib = load_library()
+    _need(R >= 1 and V >= 1, "R and V must be positive")
+    _need(target_logits.dim() >= 1 and target_logits.numel() == R * V * target_logits.shape[-1],
+          "target_logits must hold R*V rows")
+    _need(node_token.numel() == R * V and node_parent.numel() == R * V,
+          "node_token and node_parent must hold R*V entries")
+    _need(num_nodes.numel() == R, "num_nodes must hold R entries")
     host = not target_logits.is_cuda
     device = _device_of(target_logits, node_token)
     x = _dev(target_logits, device).contiguous()
     vocab = x.shape[-1]
-    if x.numel() != R * V * vocab:
-        raise ValueError("target_logits must hold R*V rows")
     tk = _dev(node_token, device).to(torch.int32).contiguous()
     pa = _dev(node_parent, device).to(torch.int32).contiguous()
     nn = _dev(num_nodes, device).to(torch.int32).contiguous()
@@ -293,12 +317,11 @@ def uno_linear_verify_noalloc(target_logits, draft_ids, q_ids, q_probs, q_count,
     library.  Same arguments and results as uno_linear_verify; only the output
     tensors are allocated here, by PyTorch, as for every entry point."""
     lib = load_library()
+    _check_linear(target_logits, draft_ids, q_ids, q_probs, q_count, R, B)
     host = not target_logits.is_cuda
     device = _device_of(target_logits, draft_ids, q_ids)
     x = _dev(target_logits, device).contiguous()
     vocab = x.shape[-1]
-    if x.numel() != R * (B + 1) * vocab:
-        raise ValueError("target_logits must hold R*(B+1) rows")
     d = _dev(draft_ids, device).to(torch.int32).contiguous()
     qi = _dev(q_ids, device).to(torch.int32).contiguous()
     qp = _dev(q_probs, device).to(torch.float32).contiguous()
