@@ -42,6 +42,11 @@ What pins each function (the tests under ``tests/test_oracle_*.py``):
   emits when the first draft row is also the first target row; its counters
   satisfy num_correct_drafts = accept_len - 2 and sum to the generated-token
   count; its output is distributed as the target-only process (chi-square).
+* ``suffix_attention`` (a module of its own, numpy float64): the LSE merge of
+  the prefix state with the tree-suffix attention equals attention over the
+  union of the key sets (``scipy.special.softmax``); a chain tree equals
+  causal attention (torch ``scaled_dot_product_attention``); grouped
+  key/value heads equal repeated heads.
 
 Parity unpinned: the boundary-event margin below which a GPU/oracle decision
 difference is excused (``BOUNDARY_EPS``) is a stated tolerance, not a value the
