@@ -241,6 +241,42 @@ uno_status uno_linear_verify_noalloc(const void* target_logits, uno_dtype dt, in
                                      int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
                                      uint32_t* out_flags, void* stream);
 
+/* ------------------------------------------------------------------------
+ * uno_tree_suffix_attention_merge -- tree-suffix attention of the V tree
+ * nodes, merged with the prefix attention state by log-sum-exp.
+ * [UNO PR, Modifications]: tree mode verifies its V nodes with EAGLE's
+ * cascade attention, and UNO adds a fused kernel for the tree-suffix
+ * attention and the LSE merge.  The pages print no formula; the standard
+ * cascade split is taken.  Node j's query attends, within the tree, to its
+ * ancestors and itself, with scores scale * <q, k>.  That gives a partial
+ * state (o_s, l_s), where l_s = log sum exp(scores) in natural logarithms.
+ * The prefix part arrives as (o_p, l_p) from another attention kernel.  The
+ * result is o = (e^l_p o_p + e^l_s o_s) / (e^l_p + e^l_s) and
+ * l = log(e^l_p + e^l_s).  Query head h reads key/value head h / (H / Hkv).
+ * Arithmetic is binary32.
+ *
+ * q            [R][V][H][d]; k and v [R][V][Hkv][d]; dtype dt, contiguous.
+ * node_parent  [R][V] int32, with parent[0] = -1 and parent[j] < j;
+ *              num_nodes [R].  Both are as written by uno_tree_topk_expand.
+ *              Nodes at or past num_nodes[r] are not read; they get o = 0
+ *              and lse = -inf.
+ * o_prefix     [R][V][H][d] float; lse_prefix [R][V][H] float.  An lse of
+ *              -inf marks an empty prefix, and its o_prefix is then not read.
+ * out_o        [R][V][H][d] float; out_lse [R][V][H] float.
+ * out_flags    nullable [R]: UNO_FLAG_BAD_TREE when a node's parent breaks
+ *              the rule above.  That node then attends to itself alone.
+ * Limits: 1 <= V <= UNO_MAX_TREE_NODES, d <= 256, H a multiple of Hkv, and
+ * the key and value tiles of one head, 2 * V * (d + 1) floats, within shared
+ * memory; UNO_ERR_UNSUPPORTED otherwise.  One CTA runs per (request,
+ * key/value head).  No workspace.
+ * ---------------------------------------------------------------------- */
+#define UNO_FLAG_BAD_TREE 16u
+uno_status uno_tree_suffix_attention_merge(const void* q, const void* k, const void* v, uno_dtype dt, int32_t R,
+                                           int32_t V, int32_t H, int32_t Hkv, int32_t d, float scale,
+                                           const int32_t* node_parent, const int32_t* num_nodes,
+                                           const float* o_prefix, const float* lse_prefix, float* out_o,
+                                           float* out_lse, uint32_t* out_flags, void* stream);
+
 /* Text of a status code (static storage). */
 const char* uno_status_string(uno_status s);
 

@@ -6,6 +6,7 @@ generator used by the tests and the benchmark.
 """
 from ._binding import (  # noqa: F401
     EXPORTED,
+    FLAG_BAD_TREE,
     FLAG_DRAFT_NOT_IN_SUPPORT,
     FLAG_NONFINITE_ROW,
     FLAG_RESIDUAL_EMPTY,
@@ -15,6 +16,7 @@ from ._binding import (  # noqa: F401
     uno_filter_softmax,
     uno_linear_verify,
     uno_linear_verify_noalloc,
+    uno_tree_suffix_attention_merge,
     uno_tree_topk_expand,
     uno_tree_verify,
 )

@@ -21,6 +21,7 @@ LIB_PATH = _PKG / "libuno_filter.so"
 
 UNO_F32, UNO_BF16 = 0, 1
 FLAG_NONFINITE_ROW, FLAG_DRAFT_NOT_IN_SUPPORT, FLAG_RESIDUAL_EMPTY = 1, 2, 4
+FLAG_BAD_TREE = 16
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported argument", 3: "CUDA launch error",
           4: "workspace missing or too small"}
 
@@ -30,6 +31,7 @@ EXPORTED = (
     "uno_tree_topk_expand",
     "uno_tree_verify_workspace_bytes", "uno_tree_verify",
     "uno_linear_verify_noalloc",
+    "uno_tree_suffix_attention_merge",
     "uno_status_string",
 )
 
@@ -90,6 +92,9 @@ def load_library():
         lib.uno_linear_verify_noalloc.argtypes = [P, ctypes.c_int, i32, i32, i64, _Params, P, P, P, P, i32, _Rng,
                                                   P, P, P, P, P]
         lib.uno_linear_verify_noalloc.restype = ctypes.c_int
+        lib.uno_tree_suffix_attention_merge.argtypes = [P, P, P, ctypes.c_int, i32, i32, i32, i32, i32,
+                                                         ctypes.c_float, P, P, P, P, P, P, P, P]
+        lib.uno_tree_suffix_attention_merge.restype = ctypes.c_int
         lib.uno_status_string.argtypes = [ctypes.c_int]
         lib.uno_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -338,3 +343,39 @@ def uno_linear_verify_noalloc(target_logits, draft_ids, q_ids, q_probs, q_count,
                                        _ptr(flags), ctypes.c_void_p(stream.cuda_stream))
     _check("uno_linear_verify_noalloc", st)
     return _host_back(dict(tokens=toks, accept_len=acc, num_tokens=ntok, flags=flags), host)
+
+
+def uno_tree_suffix_attention_merge(q, k, v, node_parent, num_nodes, o_prefix, lse_prefix, *, scale):
+    """Tree-suffix attention merged with the prefix state by log-sum-exp.
+
+    q [R, V, H, d], k and v [R, V, Hkv, d] (float32 or bfloat16, one dtype);
+    node_parent [R, V], num_nodes [R]; o_prefix [R, V, H, d] and lse_prefix
+    [R, V, H] float32 (lse -inf: empty prefix).  Returns dict(o [R, V, H, d],
+    lse [R, V, H] float32, flags [R])."""
+    lib = load_library()
+    _need(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k and v must be [R, V, heads, d]")
+    R, V, H, d = q.shape
+    Hkv = k.shape[2]
+    _need(tuple(k.shape) == (R, V, Hkv, d) and tuple(v.shape) == tuple(k.shape),
+          "k and v must be [R, V, Hkv, d] with q's R, V and d")
+    _need(k.dtype == q.dtype and v.dtype == q.dtype, "q, k and v must share one dtype")
+    _need(node_parent.numel() == R * V and num_nodes.numel() == R, "node_parent [R, V] and num_nodes [R]")
+    _need(tuple(o_prefix.shape) == (R, V, H, d) and tuple(lse_prefix.shape) == (R, V, H),
+          "o_prefix must be [R, V, H, d] and lse_prefix [R, V, H]")
+    host = not q.is_cuda
+    device = _device_of(q, k, v)
+    code = _dtype_code(q)
+    qd, kd, vd = (_dev(t, device).contiguous() for t in (q, k, v))
+    pa = _dev(node_parent, device).to(torch.int32).contiguous()
+    nn = _dev(num_nodes, device).to(torch.int32).contiguous()
+    op = _dev(o_prefix, device).to(torch.float32).contiguous()
+    lp = _dev(lse_prefix, device).to(torch.float32).contiguous()
+    stream = torch.cuda.current_stream(device)
+    o = torch.empty((R, V, H, d), dtype=torch.float32, device=device)
+    lse = torch.empty((R, V, H), dtype=torch.float32, device=device)
+    flags = torch.empty(R, dtype=torch.int32, device=device)
+    st = lib.uno_tree_suffix_attention_merge(_ptr(qd), _ptr(kd), _ptr(vd), code, R, V, H, Hkv, d, float(scale),
+                                             _ptr(pa), _ptr(nn), _ptr(op), _ptr(lp), _ptr(o), _ptr(lse),
+                                             _ptr(flags), ctypes.c_void_p(stream.cuda_stream))
+    _check("uno_tree_suffix_attention_merge", st)
+    return _host_back(dict(o=o, lse=lse, flags=flags), host)

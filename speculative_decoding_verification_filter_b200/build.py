@@ -11,7 +11,7 @@ ROOT = PKG.parent
 CSRC = PKG / "csrc"
 INCLUDE = ROOT / "include"
 LIB = PKG / "libuno_filter.so"
-SOURCES = [CSRC / "uno_filter.cu"]
+SOURCES = [CSRC / "uno_filter.cu", CSRC / "uno_suffix_attention.cu"]
 DEPS = SOURCES + [CSRC / "uno_device.cuh", INCLUDE / "uno_filter.h"]
 
 NVCC_FLAGS = [

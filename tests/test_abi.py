@@ -87,3 +87,21 @@ def test_tree_shapes_rejected_on_the_host():
     st = lib.uno_tree_verify(fake, 1, 1, 4, 8, 1000, sp, fake, fake, fake, b._Rng(1, 0), fake, fake, fake, fake,
                              fake, fake, 16, None)
     assert st == 4
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(V=129), 1), (dict(V=0), 1), (dict(H=6, Hkv=4), 1), (dict(d=0), 1), (dict(dt=7), 1),
+    (dict(scale=float("nan")), 1), (dict(null_q=True), 1), (dict(d=257), 2), (dict(V=128, d=256), 2),
+])
+def test_suffix_attention_rejects_bad_arguments_on_the_host(bad, status):
+    """Argument errors return before any device work (fake pointers are
+    never dereferenced)."""
+    from speculative_decoding_verification_filter_b200 import _binding as b
+    lib = b.load_library()
+    fake = ctypes.c_void_p(0x1000)
+    a = dict(R=2, V=8, H=4, Hkv=2, d=16, dt=0, scale=0.25)
+    a.update({k: v for k, v in bad.items() if k != "null_q"})
+    q = None if bad.get("null_q") else fake
+    st = lib.uno_tree_suffix_attention_merge(q, fake, fake, a["dt"], a["R"], a["V"], a["H"], a["Hkv"], a["d"],
+                                             a["scale"], fake, fake, fake, fake, fake, fake, None, None)
+    assert st == status

@@ -91,3 +91,16 @@ def test_tree_verify_shapes():
                    dict(node_parent=_i32(R - 1, V)), dict(num_nodes=_i32(R + 1))]:
         with pytest.raises(ValueError):
             b.uno_tree_verify(**dict(ok, **change), R=R, B=B, V=V, rng=(1, 0), **SP)
+
+
+def test_suffix_attention_shapes():
+    R, V, H, Hkv, d = 2, 5, 4, 2, 8
+    ok = dict(q=_f32(R, V, H, d), k=_f32(R, V, Hkv, d), v=_f32(R, V, Hkv, d), node_parent=_i32(R, V),
+              num_nodes=_i32(R), o_prefix=_f32(R, V, H, d), lse_prefix=_f32(R, V, H))
+    with pytest.raises(_Reached):
+        b.uno_tree_suffix_attention_merge(**ok, scale=0.3)
+    for change in [dict(q=_f32(R, V, H * d)), dict(k=_f32(R, V, Hkv, d + 1)), dict(v=_f32(R, V - 1, Hkv, d)),
+                   dict(k=torch.zeros((R, V, Hkv, d), dtype=torch.bfloat16)), dict(node_parent=_i32(R, V + 1)),
+                   dict(num_nodes=_i32(R + 1)), dict(o_prefix=_f32(R, V, H, d - 1)), dict(lse_prefix=_f32(R, V))]:
+        with pytest.raises(ValueError):
+            b.uno_tree_suffix_attention_merge(**dict(ok, **change), scale=0.3)
