@@ -95,6 +95,8 @@ def _bind(lib):
     lib.uno_ref_philox4x32_10.restype = None
     lib.uno_ref_uniform.argtypes = [u64, u32, u32, u32, u32]
     lib.uno_ref_uniform.restype = ctypes.c_double
+    lib.uno_ref_set_uniforms.argtypes = [P, i64, i32]
+    lib.uno_ref_set_uniforms.restype = None
     lib.uno_ref_filter_softmax.argtypes = [P, ctypes.c_int, i64, i64, i64, i32, f32, i32, f32, i32,
                                            P, P, P, P, ctypes.c_int, u64, u32, u32, P, P, P]
     lib.uno_ref_filter_softmax.restype = ctypes.c_int
@@ -219,6 +221,26 @@ def philox(ctr, key):
 
 def uniform(seed, request, position, draw, cycle=0):
     return _load().uno_ref_uniform(int(seed), int(request), int(position), int(draw), int(cycle))
+
+
+class injected_uniforms:
+    """Context manager: while active, the oracle's decisions take their
+    uniforms from ``table[request, position, draw]`` (shape [nreq, npos, 4],
+    float64 in [0, 1)) instead of Philox; requests or positions outside the
+    table still draw from Philox.  Used by the exact-enumeration pins, which
+    run the oracle's own decision code at chosen uniforms."""
+
+    def __init__(self, table):
+        self.table = np.ascontiguousarray(table, dtype=np.float64)
+        assert self.table.ndim == 3 and self.table.shape[2] == 4
+
+    def __enter__(self):
+        _load().uno_ref_set_uniforms(_ptr(self.table), self.table.shape[0], self.table.shape[1])
+        return self
+
+    def __exit__(self, *exc):
+        _load().uno_ref_set_uniforms(None, 0, 0)
+        return False
 
 
 def filter_softmax(logits, dtype, temperature, top_k, top_p, *, rows_per_request=1, cap=None,

@@ -87,8 +87,28 @@ void uno_ref_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], u
  * 32 bits of output followed by the top 21 bits of the second word form a
  * 53-bit integer m, and u = m * 2^-53 lies in [0, 1).  Counter-based, so any
  * draw of any cycle can be recomputed on its own. */
+/* Uniform injection, for the exact-enumeration pins only: while a table is
+ * set, the uniform of (request r, position i, draw d) with r < nreq and
+ * i < npos is table[(r * npos + i) * 4 + d] instead of the Philox draw (seed
+ * and cycle are then ignored).  Every decision of the oracle takes its
+ * uniform from uno_ref_uniform, so a test can run the oracle's own decision
+ * code at chosen uniforms and measure, by bisection on the 53-bit grid, the
+ * exact probability of each branch. */
+static const double* g_u_table = NULL;
+static int64_t g_u_nreq = 0;
+static int32_t g_u_npos = 0;
+
+void uno_ref_set_uniforms(const double* table, int64_t nreq, int32_t npos)
+{
+    g_u_table = (table != NULL && nreq > 0 && npos > 0) ? table : NULL;
+    g_u_nreq = g_u_table ? nreq : 0;
+    g_u_npos = g_u_table ? npos : 0;
+}
+
 double uno_ref_uniform(uint64_t seed, uint32_t request, uint32_t position, uint32_t draw, uint32_t cycle)
 {
+    if (g_u_table != NULL && (int64_t)request < g_u_nreq && (int32_t)position < g_u_npos && draw < 4u)
+        return g_u_table[((int64_t)request * g_u_npos + (int64_t)position) * 4 + (int64_t)draw];
     uint32_t ctr[4] = {request, position, draw, cycle};
     uint32_t key[2] = {(uint32_t)(seed & 0xFFFFFFFFu), (uint32_t)(seed >> 32)};
     uint32_t x[4];

@@ -11,6 +11,7 @@ import pytest
 
 import oracle
 import test_oracle_cycle as tc
+import test_oracle_exact as tex
 import test_oracle_filter as tf
 import test_oracle_linear as tl
 import test_oracle_params as tpa
@@ -43,6 +44,12 @@ MUTATIONS = {
     "residual not clipped": ("qc, pi_ids[j]);\n                wts[j] = d > 0.0 ? d : 0.0;",
                              "qc, pi_ids[j]);\n                wts[j] = d > 0.0 ? d : -d;",
                              lambda: tl.test_linear_output_is_the_target_process(4, 2, 1.0, 4, 1.0, 11)),
+    # With full supports (every token in supp q) this mistake changes nothing,
+    # so the sampling pin on such rows passes it; the exact enumeration on
+    # rows whose supports differ catches it.
+    "residual over supp q only": ("qc, pi_ids[j]);\n                wts[j] = d > 0.0 ? d : 0.0;",
+                                  "qc, pi_ids[j]);\n                wts[j] = (d > 0.0 && lookup_prob(qi_ids, qi_pr, qc, pi_ids[j]) > 0.0) ? d : 0.0;",
+                                  lambda: tex.test_linear_exact_distribution_is_the_target_process(*tex.LINEAR_CASES[1])),
     "bonus from wrong row": ("for (int j = 0; j < p_cnt[B]; ++j) wts[j] = (double)p_probs[(size_t)B * (size_t)cap + (size_t)j];",
                              "for (int j = 0; j < p_cnt[B]; ++j) wts[j] = (double)p_probs[(size_t)(B - 1) * (size_t)cap + (size_t)j];",
                              lambda: tl.test_linear_output_is_the_target_process(4, 2, 1.0, 4, 1.0, 11)),
