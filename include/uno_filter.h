@@ -34,8 +34,11 @@
  *   UNO_WORKSPACE_COUNTER_BYTES hold arrival counters: zero-fill them once,
  *   before the first use (zero-filling the whole buffer is simplest).  Every
  *   call leaves them at zero again and writes nothing else there, so one
- *   workspace serves any later call of any entry point and size.  The rest is
- *   scratch the library overwrites.  Calls that run at the same time on the
+ *   workspace serves any later call of any entry point and size.  The next
+ *   UNO_WORKSPACE_HINT_BYTES hold threshold hints that a call leaves for the
+ *   next call of the same entry point (see uno_filter_softmax): a speed aid
+ *   only, whatever they hold (zero included) the results are the same.  The
+ *   rest is scratch the library overwrites.  Calls that run at the same time on the
  *   GPU must not share a workspace.  Verifiers take at most
  *   UNO_WORKSPACE_COUNTER_BYTES / 8 requests per call.
  * Compact distributions.  A filtered row is stored as `count` pairs
@@ -98,6 +101,7 @@ typedef struct {
 
 #define UNO_MAX_TOP_K 1024
 #define UNO_WORKSPACE_COUNTER_BYTES (1 << 20)
+#define UNO_WORKSPACE_HINT_BYTES 8192
 #define UNO_MAX_TREE_NODES 128   /* V <= 128   ([eval guide, 启动期硬性约束]) */
 #define UNO_MAX_TREE_FRONTIER 2048 /* V*K <= 2048 (same section) */
 

@@ -174,6 +174,7 @@ __device__ __forceinline__ uint32_t kth_high_regs(const uint64_t* buf, int n, in
         v[j] = i < n ? (uint32_t)(buf[i] >> 32) : 0u;  // 0 is below every real key
     }
     uint32_t x = 0;
+#pragma unroll 1
     for (int b = 31; b >= 0; --b) {
         const uint32_t t = x | (1u << b);
         uint32_t c = 0;
@@ -190,6 +191,7 @@ __device__ __noinline__ uint32_t warp_kth_high(const uint64_t* buf, int n, int k
     if (n <= 256) return kth_high_regs<8>(buf, n, k, lane);
     if (n <= 512) return kth_high_regs<16>(buf, n, k, lane);
     uint32_t x = 0;  // large n: count from shared memory
+#pragma unroll 1
     for (int b = 31; b >= 0; --b) {
         const uint32_t t = x | (1u << b);
         uint32_t c = 0;
@@ -213,6 +215,7 @@ __device__ __forceinline__ uint32_t kth_low_regs(const uint64_t* buf, int n, uin
         lo[j] = (uint32_t)key;
     }
     uint32_t y = 0;
+#pragma unroll 1
     for (int b = 31; b >= 0; --b) {
         const uint32_t t = y | (1u << b);
         uint32_t c = 0;
@@ -247,6 +250,7 @@ __device__ __noinline__ uint64_t warp_select_kth(const uint64_t* buf, int n, int
         y = kth_low_regs<16>(buf, n, x, need, lane);
     } else {
         y = 0;
+#pragma unroll 1
         for (int b = 31; b >= 0; --b) {
             const uint32_t t = y | (1u << b);
             uint32_t c = 0;

@@ -67,6 +67,9 @@ struct RowJob {
     uint64_t* part_keys;   // [rows*S][k]
     int32_t* part_count;   // [rows*S]
     uint32_t* part_flags;  // [rows*S]
+    uint64_t* part_spec;   // pipelined kernel: the predicted threshold each piece used
+    int32_t* redo;         // pipelined kernel: rows each CTA reads again (rows + grid entries)
+    uint64_t* hint;        // pipelined kernel: per CTA, the prediction carried to the next call
     int32_t* c_ids;        // [rows][ks]  compact target rows (verifiers)
     float* c_probs;        // [rows][ks]
     int32_t ks;            // their row stride: k rounded up to a multiple of 4 (16-byte rows)
@@ -769,10 +772,13 @@ __device__ __forceinline__ double warp_incl_scan_d(double v, int lane) {
     return v;
 }
 // Ascending bitonic sort of 64 keys, element e = lane in a, e = lane + 32 in b.
+// The loops stay rolled: this runs once per row beside the streaming loop,
+// and a small body stays in the instruction cache where an unrolled one
+// would be fetched cold every time.
 __device__ __forceinline__ void warp_sort64(uint64_t& a, uint64_t& b, int lane) {
-#pragma unroll
+#pragma unroll 1
     for (int size = 2; size <= 64; size <<= 1) {
-#pragma unroll
+#pragma unroll 1
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
             if (stride == 32) {
                 const uint64_t lo = a < b ? a : b, hi = a < b ? b : a;
@@ -1236,7 +1242,8 @@ __device__ __forceinline__ void cta_rank_topk(const uint64_t* uni, int U, int k,
 
 template <int MODE>
 __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n, uint32_t rowbad,
-                                const uint64_t* sel, double* wd, unsigned char* tail_smem, FinishShared& fs, int lane) {
+                                const uint64_t* sel, double* wd, unsigned char* tail_smem, FinishShared& fs, int lane,
+                                uint64_t* pairs) {
     const bool bad = rowbad != 0u || n == 0;
     int kept = 0;
     uint64_t oa = ~0ull, ob = ~0ull;  // (id, prob) pairs, ascending id after the sort
@@ -1248,14 +1255,14 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
             wa = lane == 0 ? 1.0 : 0.0;
         } else {
             const double v0 = (double)key_value(sel[0]);
-            const double temp = (double)J.temperature;
-            if (lane < n) wa = exp(((double)key_value(ka) - v0) / temp);
-            if (lane + 32 < n) wb = exp(((double)key_value(kb) - v0) / temp);
+            const double inv_t = 1.0 / (double)J.temperature;
+            if (lane < n) wa = exp(((double)key_value(ka) - v0) * inv_t);
+            if (lane + 32 < n) wb = exp(((double)key_value(kb) - v0) * inv_t);
             if (J.top_p >= 1.0f) {
                 kept = n;
             } else {
-                const double S = warp_sum_d(wa + wb);
-                const double pa = wa / S, pb = wb / S;
+                const double inv_s = 1.0 / warp_sum_d(wa + wb);
+                const double pa = wa * inv_s, pb = wb * inv_s;
                 // mass before rank j
                 const double ia = warp_incl_scan_d(pa, lane);
                 const double ta = __shfl_sync(kFull, ia, 31);
@@ -1272,12 +1279,27 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
             }
         }
         const double ra = lane < kept ? wa : 0.0, rb = lane + 32 < kept ? wb : 0.0;
-        const double W = warp_sum_d(ra + rb);
+        const double inv_w = 1.0 / warp_sum_d(ra + rb);
         if (lane < kept)
-            oa = ((uint64_t)(uint32_t)key_id(ka) << 32) | (uint64_t)__float_as_uint((float)(wa / W));
+            oa = ((uint64_t)(uint32_t)key_id(ka) << 32) | (uint64_t)__float_as_uint((float)(wa * inv_w));
         if (lane + 32 < kept)
-            ob = ((uint64_t)(uint32_t)key_id(kb) << 32) | (uint64_t)__float_as_uint((float)(wb / W));
-        warp_sort64(oa, ob, lane);
+            ob = ((uint64_t)(uint32_t)key_id(kb) << 32) | (uint64_t)__float_as_uint((float)(wb * inv_w));
+        // ascending id order: each pair goes to its rank among the kept ids
+        // (distinct), counted against sel[] in shared memory
+        const uint32_t ida = (uint32_t)key_id(ka), idb = (uint32_t)key_id(kb);
+        int pa = 0, pb = 0;
+#pragma unroll 4
+        for (int j = 0; j < kept; ++j) {
+            const uint32_t x = (uint32_t)key_id(sel[j]);
+            pa += x < ida ? 1 : 0;
+            pb += x < idb ? 1 : 0;
+        }
+        __syncwarp();
+        if (lane < kept) pairs[pa] = oa;
+        if (lane + 32 < kept) pairs[pb] = ob;
+        __syncwarp();
+        oa = lane < kept ? pairs[lane] : ~0ull;
+        ob = lane + 32 < kept ? pairs[lane + 32] : ~0ull;
     }
     // bit 0 of rowbad: NaN / +inf (or no finite logit); bit 1: a wait gave up
     const uint32_t rflags = !bad ? 0u : (rowbad & 2u) ? (kFlagTimeout | ((rowbad & 1u) ? kFlagNonfinite : 0u))
@@ -1635,7 +1657,7 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const __grid_constant_
     }
 
     if (J.k <= 64) {
-        if (warp == 0) finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, smem + J.tail_off, fs, lane);
+        if (warp == 0) finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, smem + J.tail_off, fs, lane, outk);
     } else {
         finish_row<MODE>(J, row, req, n, rowbad, sel, outk, wd, pd, smem + J.tail_off, fs, warp, lane);
     }
@@ -1643,28 +1665,48 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const __grid_constant_
 
 // ---------------------------------------------------------------------------
 // The pipelined row kernel (k <= 64, no dense row): one persistent CTA per
-// SM works through a static list of items (row segments: item = row * S +
-// segment, CTA b takes items b, b + grid, ...).
+// SM.  The rows are laid end to end as one sequence of 16-byte units and
+// CTA b of G streams the b-th G-th of it (balanced pieces, below), so every
+// CTA moves the same number of bytes.
 //
 //   warp 0      producer: lane 0 keeps a ring of `nst` 16 KB stages filled
-//               with bulk copies (TMA, no multicast), running across item
+//               with bulk copies (TMA, no multicast), running across piece
 //               boundaries, each stage tracked by a `full` mbarrier, a fill
 //               tag and an `empty` mbarrier;
-//   warps 1..8  consumers: per item, a threshold seed from the lane maxima
-//               of the first eight stages (every warp reads a slice of
-//               each), then each warp filters the stages it owns (stage st
-//               of the item goes to warp st % 8) into its candidate buffer
-//               of the item's slot;
-//   warps 9..10 finishers: finisher f takes the items whose ordinal in the
-//               CTA's list is f mod 2 from slot f -- exact top-k of the
-//               slot's candidates with a warp bitonic merge, then the
-//               softmax / top-p / output / request-tail work of the row.
+//   warps 1..8  consumers: ring element q goes to consumer q % 8, whatever
+//               piece it belongs to.  A consumer reads each of its stages
+//               once, as it lands: the maxima of its units, then every
+//               element at or above the piece's threshold into its
+//               candidate buffer of the piece's slot (lane-parallel, one
+//               warp scan for the write positions);
+//   warps 9..10 finishers: finisher f takes the pieces whose ordinal in the
+//               CTA's list is f mod 2 from slot f: it gathers the keys at or
+//               above the piece's final threshold, hands the slot back, and
+//               selects the exact top-k from its copy; a split row's pieces
+//               publish their partial top-k and the last one merges; then
+//               the softmax / top-p / output work of the row.
 //
-// The streaming never waits for a row's serial work: while a finisher works
-// on one row the producer and consumers are already on the next ones.  Every
-// wait is bounded; a wait that gives up sets the CTA's abort word, every
-// role stops at its next check, and rows that were not finished are written
-// with UNO_FLAG_TIMEOUT.
+// Thresholds.  A piece runs in one of two modes.
+//   * boot: the piece's first stages (up to 8) wait until the k-th largest
+//     of their lane maxima is known, then every stage is filtered by it.
+//     The k-th largest of any set of disjoint group maxima of a row is at
+//     most the row's k-th largest element, so this loses nothing.  A CTA's
+//     first piece runs this way.
+//   * predicted: the piece is filtered by a threshold taken from an earlier
+//     piece of the same CTA (a value that about 2k elements of that piece
+//     reached, from the maxima of its 1024-element groups), with no waiting.
+//     Decoding cycles give rows of one distribution, so the prediction holds
+//     almost always; it is checked exactly: the row's k-th kept key must be
+//     at or above every threshold its pieces used, which means at least k
+//     elements of the row reach them and nothing of the top k was dropped.
+//     A row that fails the check is re-read whole, in boot mode, at the end
+//     of the CTA's list (the redo pass), before the kernel exits.
+// At the end of a piece its final threshold, the k-th largest of its group
+// maxima, is what the finisher gathers by, so the finisher sorts about k keys.
+//
+// Every wait is bounded; a wait that gives up sets the CTA's abort word,
+// every role stops at its next check, and rows that were not finished are
+// written with UNO_FLAG_TIMEOUT.
 // ---------------------------------------------------------------------------
 constexpr int kPipeConsumers = 8;
 constexpr int kPipeFinishers = 2;
@@ -1672,18 +1714,21 @@ constexpr int kPipeSlots = kPipeFinishers;
 constexpr int kPipeWarps = 1 + kPipeConsumers + kPipeFinishers;
 constexpr int kPipeThreads = 32 * kPipeWarps;
 constexpr int kPipeMaxK = 64;
-// A pipelined stage is 16 KB (1024 units).  In the select pass consumer warp
-// st % kPipeConsumers owns stage st of an item whole: lane l takes units l,
-// l + 32, ... (conflict-free shared loads).  In the seed pass every consumer
-// warp reads a slice of each seed stage: warp c units [c*S, (c+1)*S) with
-// S = kPSliceUnits, S / 32 per lane.
+// A pipelined stage is 16 KB (1024 units); its owner's lane l takes units
+// l, l + 32, ... (conflict-free shared loads), 32 units per lane.
 constexpr int kPStageBytes = 16384;
 constexpr int kPStageUnits = kPStageBytes / 16;                 // 1024
 constexpr int kPLaneUnits = kPStageUnits / 32;                  // 32 per lane per stage
-constexpr int kPSliceUnits = kPStageUnits / kPipeConsumers;     // 128 (seed pass)
-constexpr int kPBootStages = 8;                                 // stages of the threshold seed
-constexpr int kPipeMinStages = 10, kPipeMaxStages = 12;
-static_assert(kPipeMinStages > kPBootStages, "a stage beyond the seed stages is in flight");
+constexpr int kPGroups = 4;                                     // groups of 8 units per lane (one-stage seed)
+constexpr int kPBootStages = 8;                                 // stages of a piece's seed
+constexpr int kPGather = 256;                                   // keys a finisher gathers for its select
+constexpr int kPipeMinStages = 6, kPipeMaxStages = 12;
+// The largest grid: part slots of split rows are sized for it.
+constexpr int kPipeMaxGrid = 256;
+// A piece of a row is at least this many units when rows are few.
+constexpr int64_t kPipeMinPieceUnits = 4 * kPStageUnits;
+// A row is cut into at most this many pieces (one merge warp).
+constexpr int kPipeMaxPieces = 32;
 // Suspend hint of the off-path waits (ns): the waiting thread sleeps until
 // the phase completes or the hint runs out, instead of polling.
 constexpr uint32_t kNapNs = 2000;
@@ -1692,14 +1737,22 @@ struct __align__(16) PipeShared {
     uint64_t full[kPipeMaxStages];          // stage bytes arrived
     uint64_t empty[kPipeMaxStages];         // the stage's owner warp is done with it
     uint32_t fill[kPipeMaxStages];          // ring element each buffer holds or is receiving
-    uint64_t slot_full[kPipeSlots];         // every consumer warp is done with the slot's item
+    uint64_t slot_full[kPipeSlots];         // every consumer warp is done with the slot's piece
     uint64_t slot_empty[kPipeSlots];        // the finisher is done with the slot's buffers
-    unsigned long long tau[2];              // CTA threshold of the current item (by item parity)
-    __align__(16) uint32_t boot[2][kPipeConsumers * 32];  // lane maxima of the seed stages (read as uint4)
-    uint32_t seed[2];                       // the seed threshold's high word (by item parity)
+    unsigned long long tau[kPipeSlots];     // CTA threshold key of the slot's piece
+    unsigned long long used[kPipeSlots];    // largest predicted threshold the piece was filtered by
+    __align__(16) uint32_t boot[kPipeSlots][kPBootStages * 32];  // lane maxima of the seed stages
+    int boot_cnt[kPipeSlots];               // seed stages done
+    uint32_t boot_ready[kPipeSlots];        // the seed is in tau
+    uint32_t mode[kPipeSlots];              // the piece's mode, set by its first consumer (1 predicted, 2 not)
+    int cnt[kPipeSlots][kPipeConsumers];    // candidates per consumer warp of the slot's piece
     int wcnt[kPipeConsumers];               // candidate counts (compaction bookkeeping)
-    int cnt[kPipeSlots][kPipeConsumers];    // candidates per consumer warp of the slot's item
-    uint32_t bad[kPipeSlots];               // NaN / +inf (bit 0) or gave-up (bit 1) of the slot's item
+    uint32_t bad[kPipeSlots];               // NaN / +inf (bit 0) or gave-up (bit 1) of the slot's piece
+    unsigned long long spec;                // the latest prediction (a threshold key)
+    uint32_t spec_set;                      // a prediction exists
+    int fin_done;                           // finishers done with the CTA's list
+    int redo_n;                             // rows of the redo pass
+    uint32_t redo_ready;                    // redo_n is final
     int abort;
 };
 
@@ -1711,25 +1764,83 @@ __device__ __forceinline__ bool item_active(const RowJob& J, int64_t row) {
     return (int32_t)(row % J.V) < nn;
 }
 
-// 16-byte units [ub, ue) of a row segment and its stage count.
-struct SegGeom {
+// ---------------------------------------------------------------------------
+// Balanced pieces.  Row r owns the virtual units [r*nu, (r+1)*nu) of a
+// sequence of T = rows*nu, nu = floor(vocab / elements per unit) (a row's
+// real unit count is nu or nu - 1, by its alignment; units past it are
+// empty).  CTA b of G takes [b*T/G, (b+1)*T/G).  A row that a CTA boundary
+// cuts is split; each of its pieces publishes its partial top-k in a part
+// slot of its CTA (2b for the CTA's first row, 2b + 1 for its last) and
+// takes a ticket at the row's first CTA, which no other split row shares.
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t part_start(int64_t b, int64_t T, int64_t G) { return b * T / G; }
+// the CTA whose range holds virtual unit x (the largest b with start(b) <= x)
+__host__ __device__ __forceinline__ int64_t part_cta(int64_t x, int64_t T, int64_t G) {
+    return ((x + 1) * G + T - 1) / T - 1;
+}
+
+struct Piece {
     RowGeom g;
     const unsigned char* ubase;  // unit 0 of the row (16-byte aligned)
-    int ub, ue, nstage;
+    int ub, ue, nstage;          // the piece: units [ub, ue) of the row
+    int seg, np;                 // index of the piece in its row; pieces of the row
+    int64_t first_cta;           // CTA of the row's first piece
+};
+
+struct CtaRange {
+    int64_t nu, T, G, b, s, e, row0, row1;  // rows [row0, row1]
 };
 
 template <typename T>
-__device__ __forceinline__ SegGeom seg_geom(const RowJob& J, int64_t row, int seg) {
-    SegGeom s;
-    s.g = row_geom<T>(J, row);
-    s.ubase = s.g.base + (size_t)s.g.head * Elem<T>::kBytes;
-    const int64_t per = (s.g.nunit + J.S - 1) / J.S;
-    const int64_t vb = per * seg < s.g.nunit ? per * seg : s.g.nunit;
-    const int64_t ve = vb + per < s.g.nunit ? vb + per : s.g.nunit;
-    s.ub = (int)vb;
-    s.ue = (int)ve;
-    s.nstage = (int)((ve - vb + kPStageUnits - 1) / kPStageUnits);
-    return s;
+__device__ __forceinline__ CtaRange cta_range(const RowJob& J) {
+    CtaRange c;
+    const int64_t nu = J.vocab / Elem<T>::kPerUnit;
+    c.nu = nu > 0 ? nu : 1;
+    c.T = J.rows * c.nu;
+    c.G = gridDim.x;
+    c.b = blockIdx.x;
+    c.s = part_start(c.b, c.T, c.G);
+    c.e = part_start(c.b + 1, c.T, c.G);
+    c.row0 = c.s / c.nu;
+    c.row1 = c.e > c.s ? (c.e - 1) / c.nu : c.row0 - 1;
+    return c;
+}
+
+template <typename T>
+__device__ __forceinline__ Piece piece_of(const RowJob& J, const CtaRange& c, int64_t row) {
+    Piece p;
+    p.g = row_geom<T>(J, row);
+    p.ubase = p.g.base + (size_t)p.g.head * Elem<T>::kBytes;
+    const int64_t r0 = row * c.nu;
+    const int64_t vb = (c.s > r0 ? c.s : r0) - r0;
+    const int64_t ve = (c.e < r0 + c.nu ? c.e : r0 + c.nu) - r0;
+    p.ub = (int)(vb < p.g.nunit ? vb : p.g.nunit);
+    p.ue = (int)(ve < p.g.nunit ? ve : p.g.nunit);
+    p.nstage = (p.ue - p.ub + kPStageUnits - 1) / kPStageUnits;
+    p.first_cta = part_cta(r0, c.T, c.G);
+    p.seg = (int)(c.b - p.first_cta);
+    p.np = (int)(part_cta(r0 + c.nu - 1, c.T, c.G) - p.first_cta + 1);
+    return p;
+}
+
+// A whole row as one piece (the redo pass).
+template <typename T>
+__device__ __forceinline__ Piece whole_row(const RowJob& J, const CtaRange& c, int64_t row) {
+    Piece p;
+    p.g = row_geom<T>(J, row);
+    p.ubase = p.g.base + (size_t)p.g.head * Elem<T>::kBytes;
+    p.ub = 0;
+    p.ue = (int)p.g.nunit;
+    p.nstage = (p.ue + kPStageUnits - 1) / kPStageUnits;
+    p.first_cta = c.b;
+    p.seg = 0;
+    p.np = 1;
+    return p;
+}
+
+// Part slot of row `row`'s piece in CTA b.
+__device__ __forceinline__ int64_t part_slot(const CtaRange& c, int64_t b, int64_t row) {
+    return 2 * b + ((part_start(b, c.T, c.G) / c.nu) == row ? 0 : 1);
 }
 
 __device__ __forceinline__ bool pipe_aborted(const PipeShared& P) {
@@ -1756,6 +1867,29 @@ __device__ __forceinline__ bool pipe_wait(uint64_t* bar, uint32_t parity, const 
     for (uint32_t it = 0; it < (kMaxWaitTries >> 4); ++it) {
         if (mbar_try_wait_hint(bar, parity, kNapNs)) return true;
         if (pipe_aborted(P)) return false;
+    }
+    return false;
+}
+
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait by polling with short naps: the waiter sees the phase within
+// a few tens of nanoseconds of its completion (a suspending try_wait can
+// sleep well past it).  For the waits on the streaming path.
+constexpr uint32_t kSpinTries = 1u << 25;  // about a second at the nap below
+__device__ __forceinline__ bool pipe_spin(uint64_t* bar, uint32_t parity, const PipeShared& P) {
+    for (uint32_t it = 0; it < kSpinTries; ++it) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((it & 255u) == 255u && pipe_aborted(P)) return false;
+        __nanosleep(20);
     }
     return false;
 }
@@ -1787,57 +1921,7 @@ __device__ __forceinline__ bool pipe_wait_stage(PipeShared& P, uint32_t qq, uint
         if (!ok && (it & 15u) == 15u && pipe_aborted(P)) break;
     }
     if (!__all_sync(kFull, ok)) return false;
-    return pipe_wait_warp(&P.full[b], (qq / nst) & 1u, P);
-}
-
-// Consumer barrier over the filter warps (named barrier 1) returning the OR of v.
-__device__ __forceinline__ bool consumers_sync_or(bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n .reg .pred p, q;\n setp.ne.u32 q, %1, 0;\n bar.red.or.pred p, 1, %2, q;\n selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(r)
-        : "r"((uint32_t)v), "n"(kPipeConsumers * 32)
-        : "memory");
-    return r != 0;
-}
-
-// Plain consumer barrier (named barrier 1).
-__device__ __forceinline__ void consumers_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kPipeConsumers * 32) : "memory");
-}
-
-// Producer (one thread).
-template <typename T, int MODE>
-__device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring) {
-    const int64_t nitems = J.rows * J.S;
-    const uint32_t nst = (uint32_t)J.nst;
-    uint32_t q = 0;
-    bool ok = true;
-    for (int64_t it = blockIdx.x; ok && it < nitems; it += gridDim.x) {
-        const int64_t row = it / J.S;
-        if (!item_active<MODE>(J, row)) continue;
-        const SegGeom s = seg_geom<T>(J, row, (int)(it % J.S));
-        for (int st = 0; st < s.nstage; ++st) {
-            const uint32_t b = q % nst;
-            if (q >= nst && !pipe_wait(&P.empty[b], ((q / nst) - 1u) & 1u, P)) {
-                ok = false;
-                break;
-            }
-            if (pipe_aborted(P)) {
-                ok = false;
-                break;
-            }
-            const int u0 = s.ub + st * kPStageUnits;
-            const int nu = (s.ue - u0) < kPStageUnits ? (s.ue - u0) : kPStageUnits;
-            st_release_shared(&P.fill[b], q);  // the buffer now belongs to element q
-            mbar_expect_tx(&P.full[b], (uint32_t)nu * 16u);
-            bulk_g2s(ring + (size_t)b * kPStageBytes, s.ubase + (size_t)u0 * 16, (uint32_t)nu * 16u, &P.full[b]);
-            ++q;
-        }
-    }
-    if (!ok) atomicExch(&P.abort, 1);
-    // the copies still in flight land before the CTA may exit (bounded)
-    for (uint32_t d = q > nst ? q - nst : 0u; d < q; ++d) (void)mbar_wait_bounded(&P.full[d % nst], (d / nst) & 1u);
+    return __all_sync(kFull, pipe_spin(&P.full[b], (qq / nst) & 1u, P));
 }
 
 // Hand a stage back to the producer.  The warp's shared loads of it have
@@ -1848,30 +1932,20 @@ __device__ __forceinline__ void pipe_release(PipeShared& P, uint32_t b, int lane
     if (lane == 0) mbar_arrive(&P.empty[b]);
 }
 
-// A valid threshold from the lane maxima of every filter warp (0 = no
-// element): the largest x with a zero low half such that at least k of them
-// are >= x.  Distinct lanes hold distinct elements, so at least k elements of
-// the segment are >= x.  Two bits per step: the counts of three trial values
-// travel packed in one warp reduction (10 bits each; a count is at most 512).
-constexpr int kSeedPerLane = kPipeConsumers;  // lane maxima per lane of the searching warp
-static_assert(kSeedPerLane % 4 == 0 && kSeedPerLane * 32 < 1024, "packed 10-bit counts");
-__device__ __forceinline__ uint32_t seed_threshold(const uint32_t* bv, int k, int lane) {
-    uint32_t v[kSeedPerLane];
-#pragma unroll
-    for (int j = 0; j < kSeedPerLane; j += 4) {
-        const uint4 x = reinterpret_cast<const uint4*>(bv + lane * kSeedPerLane)[j / 4];
-        v[j] = x.x;
-        v[j + 1] = x.y;
-        v[j + 2] = x.z;
-        v[j + 3] = x.w;
-    }
+// The largest x with a zero low half such that at least k of the warp's
+// values (PER ordered keys per lane; 0 = no element) are >= x; 0 when fewer
+// than k are nonzero.  Two bits per step: the counts of three trial values
+// travel packed in one warp reduction (10 bits each).
+template <int PER>
+__device__ __forceinline__ uint32_t warp_kth_hi16(const uint32_t (&v)[PER], int k) {
+    static_assert(PER * 32 < 1024, "packed 10-bit counts");
     uint32_t p = 0;  // high bits of the answer found so far
-#pragma unroll
+#pragma unroll 1
     for (int sh = 14; sh >= 0; sh -= 2) {
         const uint32_t t1 = (p | (1u << sh)) << 16, t2 = (p | (2u << sh)) << 16, t3 = (p | (3u << sh)) << 16;
         uint32_t c = 0;
 #pragma unroll
-        for (int j = 0; j < kSeedPerLane; ++j)
+        for (int j = 0; j < PER; ++j)
             c += (v[j] >= t1 ? 1u : 0u) + (v[j] >= t2 ? (1u << 10) : 0u) + (v[j] >= t3 ? (1u << 20) : 0u);
         c = __reduce_add_sync(kFull, c);
         const uint32_t kk = (uint32_t)k;
@@ -1880,6 +1954,186 @@ __device__ __forceinline__ uint32_t seed_threshold(const uint32_t* bv, int k, in
     }
     return p << 16;
 }
+
+// A 16-byte load from shared memory by its shared-window address.
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
+    return r;
+}
+
+// One pass over a lane's 32 units of a stage (unit u = stage unit lane + 32u,
+// present when 32u < left): the units' maxima in registers (NaN propagates,
+// absent units are -inf) and the ordered maxima of its four groups of eight
+// units (NaN skipped; 0 = no finite element).
+template <typename T>
+struct StageScan;
+
+template <>
+struct StageScan<__nv_bfloat16> {
+    typedef __nv_bfloat162 B2;
+    typedef __nv_bfloat162 Cmp;
+    __device__ __forceinline__ static B2 w2(uint32_t w) { return *reinterpret_cast<const B2*>(&w); }
+    __device__ __forceinline__ static uint32_t gkey(B2 m) {
+        const float f = fmaxf(__low2float(m), __high2float(m));
+        return (f > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(f, 0.0f)) : 0u;
+    }
+    __device__ __forceinline__ static B2 ninf2() { return w2(0xff80ff80u); }
+    // NaN or +inf in either half of a NaN-propagating maximum
+    __device__ __forceinline__ static bool nonfinite(B2 m) {
+        return !(__low2float(m) < __int_as_float(0x7f800000)) || !(__high2float(m) < __int_as_float(0x7f800000));
+    }
+    // The lane's units of a stage (unit u = stage unit lane + 32u, present when
+    // 32u < left), one pass: bit u of the result is set when unit u is present
+    // and some element of it is >= tau or NaN; lm gets the ordered key of the
+    // lane's largest finite element (0: none), `bad` whether some element is
+    // NaN or +inf.
+    __device__ __forceinline__ static uint32_t flags_fused(const uint4* lsp, int left, Cmp tau, uint32_t& lm,
+                                                           bool& bad) {
+        const uint32_t sa = smem_u32(lsp);
+        const uint4 ninf = Elem<__nv_bfloat16>::neg_inf_unit();
+        uint32_t ub = 0;
+        B2 mx = ninf2(), nn = ninf2();
+#pragma unroll 4
+        for (int u = 0; u < kPLaneUnits; ++u) {
+            const bool here = 32 * u < left;
+            const uint4 x = lds128(sa + (uint32_t)u * 512u);
+            const uint4 r = here ? x : ninf;
+            const B2 m = Elem<__nv_bfloat16>::umax(r);
+            nn = __hmax2_nan(nn, m);
+            mx = __hmax2(mx, m);
+            ub |= (here && __hgeu2_mask(m, tau) != 0u ? 1u : 0u) << u;
+        }
+        lm = gkey(mx);
+        bad = nonfinite(nn);
+        return ub;
+    }
+    // Statistics only (the threshold is not known yet): the ordered maxima of
+    // the lane's four groups of eight units; returns the lane's maximum key.
+    __device__ __forceinline__ static uint32_t stats(const uint4* lsp, int left, uint32_t (&gk)[kPGroups], bool& bad) {
+        const uint32_t sa = smem_u32(lsp);
+        const uint4 ninf = Elem<__nv_bfloat16>::neg_inf_unit();
+        B2 nn = ninf2();
+        uint32_t lm = 0;
+#pragma unroll
+        for (int g = 0; g < kPGroups; ++g) {
+            B2 mx = ninf2();
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const int u = 8 * g + v;
+                const uint4 x = lds128(sa + (uint32_t)u * 512u);
+                const uint4 r = (32 * u < left) ? x : ninf;
+                const B2 m = Elem<__nv_bfloat16>::umax(r);
+                nn = __hmax2_nan(nn, m);
+                mx = __hmax2(mx, m);
+            }
+            gk[g] = gkey(mx);
+            lm = gk[g] > lm ? gk[g] : lm;
+        }
+        bad = nonfinite(nn);
+        return lm;
+    }
+    // Flags only (a second pass once the threshold is known).
+    __device__ __forceinline__ static uint32_t flags(const uint4* lsp, int left, Cmp tau) {
+        const uint32_t sa = smem_u32(lsp);
+        uint32_t ub = 0;
+#pragma unroll 4
+        for (int u = 0; u < kPLaneUnits; ++u) {
+            const bool here = 32 * u < left;
+            const uint4 x = lds128(sa + (uint32_t)u * 512u);
+            const uint4 r = here ? x : Elem<__nv_bfloat16>::neg_inf_unit();
+            ub |= (here && __hgeu2_mask(Elem<__nv_bfloat16>::umax(r), tau) != 0u ? 1u : 0u) << u;
+        }
+        return ub;
+    }
+    // the unit comparand of a threshold value (rounded down to bf16)
+    __device__ __forceinline__ static Cmp unit_cmp(float t) { return Elem<__nv_bfloat16>::make_tau(t); }
+    // the element comparand of a threshold value: rounded down to bf16, and
+    // never below the lowest finite value (so -inf elements stay out)
+    __device__ __forceinline__ static Cmp cmp_of(float t) {
+        const float lo = -3.3895313892515355e38f;  // lowest finite bf16
+        const __nv_bfloat16 b = __float2bfloat16_rd(t > lo ? t : lo);
+        return __halves2bfloat162(b, b);
+    }
+    // bit e: element e of the unit is >= c (NaN is not)
+    __device__ __forceinline__ static uint32_t ge_mask(const uint4& r, Cmp c) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+        uint32_t m = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t g = __hge2_mask(w2(w[q]), c);
+            m |= ((g & 1u) | ((g >> 15) & 2u)) << (2 * q);
+        }
+        return m;
+    }
+};
+
+template <>
+struct StageScan<float> {
+    typedef float Cmp;
+    __device__ __forceinline__ static uint32_t gkey(float f) {
+        return (f > -__int_as_float(0x7f800000)) ? ord_of_float(__fadd_rn(f, 0.0f)) : 0u;
+    }
+    __device__ __forceinline__ static uint32_t flags_fused(const uint4* lsp, int left, Cmp tau, uint32_t& lm,
+                                                           bool& bad) {
+        const uint32_t sa = smem_u32(lsp);
+        uint32_t ub = 0;
+        float mx = -__int_as_float(0x7f800000), nn = -__int_as_float(0x7f800000);
+#pragma unroll 4
+        for (int u = 0; u < kPLaneUnits; ++u) {
+            const bool here = 32 * u < left;
+            const uint4 x = lds128(sa + (uint32_t)u * 512u);
+            const uint4 r = here ? x : Elem<float>::neg_inf_unit();
+            const float m = Elem<float>::umax(r);
+            nn = Elem<float>::max_nan(nn, m);
+            mx = fmaxf(mx, m);
+            ub |= (here && !(m < tau) ? 1u : 0u) << u;
+        }
+        lm = gkey(mx);
+        bad = !(nn < __int_as_float(0x7f800000));
+        return ub;
+    }
+    __device__ __forceinline__ static uint32_t stats(const uint4* lsp, int left, uint32_t (&gk)[kPGroups], bool& bad) {
+        const uint32_t sa = smem_u32(lsp);
+        float nn = -__int_as_float(0x7f800000);
+        uint32_t lm = 0;
+#pragma unroll
+        for (int g = 0; g < kPGroups; ++g) {
+            float mx = -__int_as_float(0x7f800000);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const int u = 8 * g + v;
+                const uint4 x = lds128(sa + (uint32_t)u * 512u);
+                const uint4 r = (32 * u < left) ? x : Elem<float>::neg_inf_unit();
+                const float m = Elem<float>::umax(r);
+                nn = Elem<float>::max_nan(nn, m);
+                mx = fmaxf(mx, m);
+            }
+            gk[g] = gkey(mx);
+            lm = gk[g] > lm ? gk[g] : lm;
+        }
+        bad = !(nn < __int_as_float(0x7f800000));
+        return lm;
+    }
+    __device__ __forceinline__ static uint32_t flags(const uint4* lsp, int left, Cmp tau) {
+        const uint32_t sa = smem_u32(lsp);
+        uint32_t ub = 0;
+#pragma unroll 4
+        for (int u = 0; u < kPLaneUnits; ++u) {
+            const bool here = 32 * u < left;
+            const uint4 x = lds128(sa + (uint32_t)u * 512u);
+            const uint4 r = here ? x : Elem<float>::neg_inf_unit();
+            ub |= (here && !(Elem<float>::umax(r) < tau) ? 1u : 0u) << u;
+        }
+        return ub;
+    }
+    __device__ __forceinline__ static Cmp unit_cmp(float t) { return t; }
+    __device__ __forceinline__ static Cmp cmp_of(float t) { return t > -3.402823466e38f ? t : -3.402823466e38f; }
+    __device__ __forceinline__ static uint32_t ge_mask(const uint4& r, Cmp c) {
+        return (__uint_as_float(r.x) >= c ? 1u : 0u) | (__uint_as_float(r.y) >= c ? 2u : 0u) |
+               (__uint_as_float(r.z) >= c ? 4u : 0u) | (__uint_as_float(r.w) >= c ? 8u : 0u);
+    }
+};
 
 // One consumer warp's candidates of one stage: every element of the lane's
 // eight units that is >= the threshold (or NaN) is re-read from the stage
@@ -1933,7 +2187,7 @@ __device__ __noinline__ AppendState pipe_append(uint64_t* buf, int* wcnt, Append
 // per-lane counts.  A round that would overflow the buffer goes one element
 // per lane at a time with compaction in between (pipe_append).
 template <typename T>
-__device__ __forceinline__ AppendState pipe_units(uint64_t* buf, int* wcnt, AppendState st, uint32_t ub,
+__device__ __noinline__ AppendState pipe_units(uint64_t* buf, int* wcnt, AppendState st, uint32_t ub,
                                                const uint4* sp, uint32_t id0, int hw, int cap_w, int k,
                                                unsigned long long* s_tau, int lane) {
     constexpr int KPU = Elem<T>::kPerUnit;
@@ -1978,75 +2232,239 @@ __device__ __forceinline__ AppendState pipe_units(uint64_t* buf, int* wcnt, Appe
     return st;
 }
 
-// Consumer warp c (0 .. kPipeConsumers-1).
+// The candidates of one stage, lane-parallel: every lane counts the
+// elements >= the threshold value in its flagged units, one warp scan gives
+// each lane its write position, and each lane writes its own keys.  Returns
+// the new count, or -1 (nothing written) when they would not fit in cap_w.
+template <typename T>
+__device__ __forceinline__ int extract_fast(uint64_t* buf, int cnt, uint32_t ub, const uint4* lsp, uint64_t tau,
+                                            uint32_t id0, int cap_w, int lane) {
+    typedef StageScan<T> SS;
+    constexpr int KPU = Elem<T>::kPerUnit;
+    const typename SS::Cmp cmp = SS::cmp_of(tau_value(tau));
+    int c = 0;
+    const uint32_t sa = smem_u32(lsp);
+    for (uint32_t m = ub; m != 0u; m &= m - 1u) c += __popc(SS::ge_mask(lds128(sa + (uint32_t)(__ffs(m) - 1) * 512u), cmp));
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += t;
+    }
+    const int total = __shfl_sync(kFull, incl, 31);
+    if (cnt + total > cap_w) return -1;
+    int pos = cnt + incl - c;
+    for (uint32_t m = ub; m != 0u; m &= m - 1u) {
+        const int u = __ffs(m) - 1;
+        const uint4 r = lds128(sa + (uint32_t)u * 512u);
+        uint32_t em = SS::ge_mask(r, cmp);
+        const uint32_t idu = id0 + (uint32_t)(u * 32 * KPU);
+        while (em != 0u) {
+            const int e = __ffs(em) - 1;
+            em &= em - 1u;
+            buf[pos++] = make_key(Elem<T>::get(r, e), idu + (uint32_t)e);
+        }
+    }
+    __syncwarp();
+    return cnt + total;
+}
+
+// The CTA threshold of a piece, read once and given to the whole warp (so
+// that every lane takes the same branches).
+__device__ __forceinline__ uint64_t read_tau(const unsigned long long* s_tau) {
+    uint64_t v = 0ull;
+    if ((threadIdx.x & 31) == 0) v = *reinterpret_cast<const volatile unsigned long long*>(s_tau);
+    return __shfl_sync(kFull, v, 0);
+}
+
+// Whole warp or one thread: wait until a shared flag is set (acquire).
+__device__ __forceinline__ bool wait_flag(const uint32_t* f, const PipeShared& P) {
+    for (uint32_t it = 0; it < kMaxWaitTries; ++it) {
+        if (ld_acquire_shared(f) != 0u) return true;
+        if ((it & 15u) == 15u && pipe_aborted(P)) return false;
+        __nanosleep(64);
+    }
+    return false;
+}
+
+// The CTA's list of items: one per row its range touches (main items), then
+// the rows of its redo pass.  Every role walks it in the same order.
+struct PipeList {
+    CtaRange cr;
+    int64_t nmain, rbase;  // main items; the redo rows' offset in J.redo
+    bool rot;              // the last row is cut by the CTA's end: it goes first
+    int64_t nredo;         // known after the main items (-1 before)
+    int64_t full_units;    // units of a whole row (for "big" pieces)
+    bool spec_ok;          // rows are long enough for predictions
+};
+
+template <typename T>
+__device__ __forceinline__ PipeList pipe_list(const RowJob& J) {
+    PipeList L;
+    L.cr = cta_range<T>(J);
+    L.nmain = L.cr.row1 - L.cr.row0 + 1;
+    L.rbase = L.cr.row0 + L.cr.b;
+    // a row split across two CTAs is merged by the one that finishes its
+    // piece last; taking the CTA's last (split) row first, as the next CTA
+    // takes it first too, keeps merges away from the end of the kernel
+    L.rot = L.nmain > 1 && (L.cr.e % L.cr.nu) != 0;
+    L.nredo = -1;
+    L.full_units = L.cr.nu;
+    // predictions read the spacing of a row's k best values; rows must hold
+    // several times k elements
+    L.spec_ok = J.k >= 8 && L.cr.nu * Elem<T>::kPerUnit >= (int64_t)16 * J.k;
+    return L;
+}
+
+// Row of main item i.
+__device__ __forceinline__ int64_t main_row(const PipeList& L, int64_t i) {
+    if (!L.rot) return L.cr.row0 + i;
+    return i == 0 ? L.cr.row1 : L.cr.row0 + i - 1;
+}
+
+// A main piece whose group maxima publish a prediction: at least a quarter
+// of a row.
+__device__ __forceinline__ bool piece_big(const PipeList& L, const Piece& p) {
+    return L.spec_ok && (int64_t)(p.ue - p.ub) * 4 >= L.full_units;
+}
+
+// Producer (one thread).
+template <typename T, int MODE>
+__device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring) {
+    PipeList L = pipe_list<T>(J);
+    const uint32_t nst = (uint32_t)J.nst;
+    uint32_t q = 0;
+    bool ok = true;
+    auto issue = [&](const Piece& p) {
+        for (int st = 0; ok && st < p.nstage; ++st) {
+            const uint32_t b = q % nst;
+            if (q >= nst && !pipe_spin(&P.empty[b], ((q / nst) - 1u) & 1u, P)) {
+                ok = false;
+                break;
+            }
+            if (pipe_aborted(P)) {
+                ok = false;
+                break;
+            }
+            const int u0 = p.ub + st * kPStageUnits;
+            const int nu = (p.ue - u0) < kPStageUnits ? (p.ue - u0) : kPStageUnits;
+            st_release_shared(&P.fill[b], q);  // the buffer now belongs to element q
+            mbar_expect_tx(&P.full[b], (uint32_t)nu * 16u);
+            bulk_g2s(ring + (size_t)b * kPStageBytes, p.ubase + (size_t)u0 * 16, (uint32_t)nu * 16u, &P.full[b]);
+            ++q;
+        }
+    };
+    for (int64_t i = 0; ok && i < L.nmain; ++i) {
+        const int64_t row = main_row(L, i);
+        if (item_active<MODE>(J, row)) issue(piece_of<T>(J, L.cr, row));
+    }
+    // the redo pass: rows whose prediction failed, read whole
+    if (ok && wait_flag(&P.redo_ready, P)) {
+        const int n = *reinterpret_cast<volatile int*>(&P.redo_n);
+        for (int j = 0; ok && j < n; ++j) issue(whole_row<T>(J, L.cr, (int64_t)__ldcg(J.redo + L.rbase + j)));
+    } else {
+        ok = false;
+    }
+    if (!ok) atomicExch(&P.abort, 1);
+    // the copies still in flight land before the CTA may exit (bounded)
+    for (uint32_t d = q > nst ? q - nst : 0u; d < q; ++d) (void)mbar_wait_bounded(&P.full[d % nst], (d / nst) & 1u);
+}
+
+// The item of ordinal i for a consumer or finisher warp (whole warp): false
+// past the end of the list.  Waits for the redo list at the end of the main
+// items.
+template <typename T>
+__device__ __forceinline__ bool pipe_item(const RowJob& J, PipeShared& P, PipeList& L, int64_t i, int64_t& row,
+                                          bool& redo) {
+    if (i < L.nmain) {
+        row = main_row(L, i);
+        redo = false;
+        return true;
+    }
+    if (L.nredo < 0) {
+        const bool ok = __all_sync(kFull, wait_flag(&P.redo_ready, P));
+        L.nredo = ok ? (int64_t)*reinterpret_cast<volatile int*>(&P.redo_n) : 0;
+        L.nredo = __shfl_sync(kFull, L.nredo, 0);
+    }
+    if (i >= L.nmain + L.nredo) return false;
+    row = (int64_t)__ldcg(J.redo + L.rbase + (i - L.nmain));
+    redo = true;
+    return true;
+}
+
+// A piece's seed from the lane maxima of its first nA stages (32 per
+// stage; stage j's at bv[32 j .. 32 j + 31]).  Distinct lanes of distinct
+// stages hold distinct elements, so at least k elements are >= the result.
+__device__ __forceinline__ uint32_t boot_threshold(const uint32_t* bv, int nA, int k, int lane) {
+    uint32_t v[kPBootStages];
+    const bool mine = (lane * kPBootStages) / 32 < nA;  // lane's values belong to stage lane / 4
+#pragma unroll
+    for (int j = 0; j < kPBootStages; j += 4) {
+        const uint4 x = mine ? reinterpret_cast<const uint4*>(bv + lane * kPBootStages)[j / 4] : make_uint4(0, 0, 0, 0);
+        v[j] = x.x;
+        v[j + 1] = x.y;
+        v[j + 2] = x.z;
+        v[j + 3] = x.w;
+    }
+    return warp_kth_hi16<kPBootStages>(v, k);
+}
+
+
+// Consumer warp c (0 .. kPipeConsumers-1): ring elements q with q % 8 == c.
 template <typename T, int MODE>
 __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char* ring, uint64_t* slots, int c,
                              int lane) {
-    typedef typename Elem<T>::Tau Tau;
+    typedef StageScan<T> SS;
     constexpr int KPU = Elem<T>::kPerUnit;
-    const int64_t nitems = J.rows * J.S;
+    PipeList L = pipe_list<T>(J);
     const uint32_t nst = (uint32_t)J.nst;
-    const int k = J.k, hw = J.hw, cap_w = J.cap_w, S = J.S;
-    uint32_t q = 0;              // ring element of the item's first stage
-    uint32_t a = 0;              // active items so far
+    const int k = J.k, hw = J.hw, cap_w = J.cap_w;
+    uint32_t q = 0;              // ring element of the piece's first stage
     uint32_t used = 0, par = 0;  // per slot: used before; parity of its current use
     bool fail = false;
-    int64_t i = 0;
-    for (int64_t it = blockIdx.x; it < nitems; it += gridDim.x, ++i) {
-        const int64_t row = it / S;
-        const int seg = (int)(it % S);
+    int64_t row = 0;
+    bool redo = false;
+    for (int64_t i = 0; pipe_item<T>(J, P, L, i, row, redo); ++i) {
         if (!item_active<MODE>(J, row)) continue;
         const int slot = (int)(i % kPipeSlots);
         const uint32_t sb = 1u << slot;
-        // the finisher is done with this slot's previous item
+        // the finisher is done with this slot's previous piece
         if ((used & sb) && !pipe_wait_warp(&P.slot_empty[slot], (par & sb) ? 0u : 1u, P)) fail = true;
-        const SegGeom s = seg_geom<T>(J, row, seg);
-        const int nA = s.nstage < kPBootStages ? s.nstage : kPBootStages;
-
-        // pass 1: lane maxima of this warp's slice of the first nA stages
-        typename Elem<T>::Top m1 = Elem<T>::top_init();
-        for (int st = 0; st < nA && !fail; ++st) {
-            const uint32_t qq = q + st;
-            const uint32_t b = qq % nst;
-            if (!pipe_wait_stage(P, qq, nst)) {
-                fail = true;
-                break;
-            }
-            const int u0 = s.ub + st * kPStageUnits + c * kPSliceUnits + lane;
-            const uint4* sp = reinterpret_cast<const uint4*>(ring + (size_t)b * kPStageBytes) + c * kPSliceUnits + lane;
-#pragma unroll
-            for (int u = 0; u < kPSliceUnits / 32; ++u)
-                if (u0 + u * 32 < s.ue) Elem<T>::max_update(m1, sp[u * 32]);
+        const Piece p = redo ? whole_row<T>(J, L.cr, row) : piece_of<T>(J, L.cr, row);
+        // the first consumer warp to start the piece fixes its mode: predicted
+        // when a prediction exists by then (nobody waits for one)
+        uint32_t mode = 0;
+        if (lane == 0) {
+            const uint32_t want = (!redo && L.spec_ok && ld_acquire_shared(&P.spec_set) != 0u) ? 1u : 2u;
+            const uint32_t old = atomicCAS(&P.mode[slot], 0u, want);
+            mode = old == 0u ? want : old;
         }
-        P.boot[a & 1][c * 32 + lane] = fail ? 0u : Elem<T>::lane_max_ord(m1);
-        // every consumer warp takes the same exit decision here
-        if (consumers_sync_or(fail || pipe_aborted(P))) {
-            if (lane == 0) atomicExch(&P.abort, 1);
-            return;
+        const bool predicted = __shfl_sync(kFull, mode, 0) == 1u;
+        const int nA = p.nstage < kPBootStages ? p.nstage : kPBootStages;
+        // a seed from lane maxima needs about 2k lanes that hold elements
+        // (a short last stage has fewer); else each stage seeds itself
+        int lanes = 0;
+        for (int st = 0; st < nA; ++st) {
+            const int u = p.ue - (p.ub + st * kPStageUnits);
+            lanes += u < 32 ? u : 32;
         }
-        unsigned long long* s_tau = &P.tau[a & 1];
+        const bool boot = !predicted && lanes >= 2 * k;
+        unsigned long long* s_tau = &P.tau[slot];
 
         WarpState ws;
         ws.buf = slots + ((size_t)slot * kPipeConsumers + c) * cap_w;
         ws.wcnt = &P.wcnt[c];
         ws.cnt = 0;
         ws.bad = 0u;
-        if (c == 0) {
-            // the threshold seed, for every consumer warp
-            const uint32_t t0 = seed_threshold(P.boot[a & 1], k, lane);
-            if (lane == 0) {
-                P.seed[a & 1] = t0;
-                P.tau[(a + 1) & 1] = 0ull;  // nobody reads the previous item's threshold now
-            }
-        } else if (c == 1 && seg == 0) {
+        if (c == 1 && p.seg == 0) {
             // row head / tail scalars (fewer than 16): every finite one
-            const int64_t ntail = J.vocab - s.g.tail_begin;
-            const int64_t nsc = s.g.head + ntail;
+            const int64_t ntail = J.vocab - p.g.tail_begin;
+            const int64_t nsc = p.g.head + ntail;
             uint64_t key = 0ull;
             bool has = false;
             if (lane < nsc) {
-                const int64_t id = (lane < s.g.head) ? (int64_t)lane : s.g.tail_begin + (lane - s.g.head);
-                const float v = Elem<T>::load_scalar(s.g.base + (size_t)id * Elem<T>::kBytes);
+                const int64_t id = (lane < p.g.head) ? (int64_t)lane : p.g.tail_begin + (lane - p.g.head);
+                const float v = Elem<T>::load_scalar(p.g.base + (size_t)id * Elem<T>::kBytes);
                 if (v != v || v == __int_as_float(0x7f800000)) {
                     ws.bad |= 1u;
                 } else if (v != -__int_as_float(0x7f800000)) {
@@ -2058,46 +2476,109 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
             if (has) ws.buf[__popc(bal & lanemask_lt())] = key;
             ws.cnt = __popc(bal);
         }
-        consumers_sync();
-        ws.tau = (uint64_t)P.seed[a & 1] << 32;
+        ws.tau = read_tau(s_tau);
+        if (predicted) {
+            // the latest prediction of this CTA
+            const uint64_t t = read_tau(&P.spec);
+            if (t > ws.tau) ws.tau = t;
+            if (lane == 0) {
+                atomicMax(&P.used[slot], (unsigned long long)t);
+                atomicMax(s_tau, (unsigned long long)t);
+            }
+        }
 
-        // pass 2: select, this warp's stages of the item
-        const uint32_t id_base = (uint32_t)s.g.head;
-        Tau tau_v = Elem<T>::make_tau(tau_value(ws.tau));
-        for (int st = c; st < s.nstage && !fail; st += kPipeConsumers) {
+        const uint32_t id_base = (uint32_t)p.g.head;
+        const int st0 = (int)((uint32_t)(c + kPipeConsumers) - q % kPipeConsumers) % kPipeConsumers;
+        for (int st = st0; st < p.nstage && !fail; st += kPipeConsumers) {
             const uint32_t qq = q + st;
             const uint32_t b = qq % nst;
             if (!pipe_wait_stage(P, qq, nst)) {
                 fail = true;
                 break;
             }
-            const int us = s.ub + st * kPStageUnits + lane;  // the lane's first unit in the row
+            const int su = p.ub + st * kPStageUnits;  // the stage's first unit in the row
+            const int left = (p.ue - su) - lane;       // the lane's unit u is present when 32 u < left
             const uint4* lsp = reinterpret_cast<const uint4*>(ring + (size_t)b * kPStageBytes) + lane;
-            uint32_t ub = 0;  // bit j: the lane's unit j (unit us + 32 j) may hold a candidate
-            if (s.ue - (s.ub + st * kPStageUnits) >= kPStageUnits) {
+            uint32_t ub, lm;
+            bool nonfin = false;
+            if (predicted) {
+                // one pass: the threshold is known
+                {
+                    const uint64_t stv = read_tau(s_tau);
+                    if (stv > ws.tau) ws.tau = stv;
+                }
+                ub = SS::flags_fused(lsp, left, SS::unit_cmp(tau_value(ws.tau)), lm, nonfin);
+            } else {
+                uint32_t gk[kPGroups];
+                lm = SS::stats(lsp, left, gk, nonfin);
+                if (boot) {
+                    // the piece's seed: lane maxima of its first nA stages; the
+                    // consumer that completes them searches, every stage waits
+                    if (st < nA) {
+                        P.boot[slot][st * 32 + lane] = lm;
+                        __threadfence_block();
+                        __syncwarp();
+                        int last = 0;
+                        if (lane == 0) last = atomicAdd(&P.boot_cnt[slot], 1) == nA - 1;
+                        if (__shfl_sync(kFull, last, 0)) {
+                            __threadfence_block();
+                            const uint64_t t = (uint64_t)boot_threshold(P.boot[slot], nA, k, lane) << 32;
+                            if (lane == 0) {
+                                atomicMax(s_tau, (unsigned long long)t);
+                                // until a big piece completes, its seed is the CTA's
+                                // prediction (about 2.6 k elements of a row reach it)
+                                if (!redo && piece_big(L, p) && P.spec_set == 0u) {
+                                    P.spec = t;
+                                    __threadfence_block();
+                                    st_release_shared(&P.spec_set, 1u);
+                                }
+                                st_release_shared(&P.boot_ready[slot], 1u);
+                            }
+                        }
+                    }
+                    if (!__all_sync(kFull, wait_flag(&P.boot_ready[slot], P))) fail = true;
+                } else {
+                    // one-stage seed: the k-th largest of this stage's group maxima
+                    const uint32_t th = (uint32_t)(ws.tau >> 32);
+                    uint32_t n = 0;
 #pragma unroll
-                for (int u = 0; u < kPLaneUnits; ++u) ub |= Elem<T>::maybe(lsp[u * 32], tau_v) ? (1u << u) : 0u;
-            } else {  // the segment's last stage: only its units (the rest holds older data)
-                const int left = s.ue - us;
-#pragma unroll
-                for (int u = 0; u < kPLaneUnits; ++u)
-                    if (32 * u < left) ub |= Elem<T>::maybe(lsp[u * 32], tau_v) ? (1u << u) : 0u;
+                    for (int g = 0; g < kPGroups; ++g) n += gk[g] > th ? 1u : 0u;
+                    if (__reduce_add_sync(kFull, n) >= (uint32_t)k) {
+                        const uint64_t t = (uint64_t)warp_kth_hi16<kPGroups>(gk, k) << 32;
+                        if (t > ws.tau) {
+                            ws.tau = t;
+                            if (lane == 0) atomicMax(s_tau, (unsigned long long)t);
+                        }
+                    }
+                }
+                {
+                    const uint64_t stv = read_tau(s_tau);
+                    if (stv > ws.tau) ws.tau = stv;
+                }
+                ub = SS::flags(lsp, left, SS::unit_cmp(tau_value(ws.tau)));
             }
+            if (nonfin) ws.bad |= 1u;
             if (__any_sync(kFull, ub != 0u)) {
-                const AppendState r = pipe_units<T>(ws.buf, ws.wcnt, AppendState{ws.cnt, ws.tau, ws.bad}, ub, lsp,
-                                                    id_base + (uint32_t)us * KPU, hw, cap_w, k, s_tau, lane);
-                ws.cnt = r.cnt;
-                ws.tau = r.tau;
-                ws.bad = r.bad;
+                const uint32_t id0 = id_base + (uint32_t)(su + lane) * KPU;
+                const int nc = extract_fast<T>(ws.buf, ws.cnt, ub, lsp, ws.tau, id0, cap_w, lane);
+                if (nc >= 0) {
+                    ws.cnt = nc;
+                    if (ws.cnt > hw) {
+                        const Compacted cp = warp_compact(ws.buf, ws.wcnt, ws.cnt, ws.tau, k, s_tau, lane);
+                        ws.cnt = cp.cnt;
+                        ws.tau = cp.tau;
+                    }
+                } else {  // rare: the stage's candidates overflow the buffer; append with compaction
+                    const AppendState r = pipe_units<T>(ws.buf, ws.wcnt, AppendState{ws.cnt, ws.tau, 0u}, ub, lsp,
+                                                        id0, hw, cap_w, k, s_tau, lane);
+                    ws.cnt = r.cnt;
+                    ws.tau = r.tau;
+                }
             }
             pipe_release(P, b, lane);
-            // adopt a better threshold found by another warp
-            const unsigned long long stv = *reinterpret_cast<volatile unsigned long long*>(s_tau);
-            if (stv > ws.tau) ws.tau = stv;
-            tau_v = Elem<T>::make_tau(tau_value(ws.tau));
         }
         {
-            const unsigned long long stv = *reinterpret_cast<volatile unsigned long long*>(s_tau);
+            const uint64_t stv = read_tau(s_tau);
             if (stv > ws.tau) ws.tau = stv;
             ws.cnt = warp_keep_ge(ws.buf, ws.cnt, ws.tau, lane);
         }
@@ -2108,8 +2589,7 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
             mbar_arrive(&P.slot_full[slot]);
         }
         if (fail && lane == 0) atomicExch(&P.abort, 1);
-        q += (uint32_t)s.nstage;
-        ++a;
+        q += (uint32_t)p.nstage;
         par ^= sb;
         used |= sb;
     }
@@ -2123,7 +2603,7 @@ __device__ __forceinline__ void warp_merge64(uint64_t& a, uint64_t& b, int lane)
         a = lo;
         b = hi;
     }
-#pragma unroll
+#pragma unroll 1
     for (int stride = 16; stride > 0; stride >>= 1) {
         const uint64_t pa = __shfl_xor_sync(kFull, a, stride), pb = __shfl_xor_sync(kFull, b, stride);
         const bool lower = (lane & stride) == 0;
@@ -2160,14 +2640,90 @@ __device__ __forceinline__ int warp_topk64(int U, int k, const Get& get, uint64_
     return n;
 }
 
+// The best min(k, U) of U distinct keys g[0..U) (U <= kPGather), into
+// sel[] in descending order, by rank: each key's rank is the number of
+// larger keys, counted against g[] in shared memory (independent loads, no
+// shuffle chain).  One warp.
+__device__ __noinline__ int warp_rank_topk(const uint64_t* g, int U, int k, uint64_t* sel, int lane) {
+    for (int i0 = 0; i0 < U; i0 += 64) {
+        const int ia = i0 + lane, ib = i0 + 32 + lane;
+        const uint64_t ka = ia < U ? g[ia] : ~0ull, kb = ib < U ? g[ib] : ~0ull;
+        int ra = 0, rb = 0;
+#pragma unroll 4
+        for (int j = 0; j < U; ++j) {
+            const uint64_t x = g[j];
+            ra += x > ka ? 1 : 0;
+            rb += x > kb ? 1 : 0;
+        }
+        if (ia < U && ra < k) sel[ra] = ka;
+        if (ib < U && rb < k) sel[rb] = kb;
+    }
+    __syncwarp();
+    return U < k ? U : k;
+}
+
+// The best min(k, U) of U distinct keys g[0..U) (U <= kPGather), into
+// sel[] in descending order: first cut g to the keys whose high half reaches
+// the k-th largest high half (a warp radix search), then rank the rest.
+__device__ __noinline__ int warp_select_topk(uint64_t* g, int U, int k, uint64_t* sel, int lane) {
+    if (U > k + 8) {
+        constexpr int PER = kPGather / 32;
+        uint32_t v[PER];
+#pragma unroll
+        for (int j = 0; j < PER; ++j) v[j] = lane + 32 * j < U ? (uint32_t)(g[lane + 32 * j] >> 32) : 0u;
+        const uint64_t x = (uint64_t)warp_kth_hi16<PER>(v, k) << 32;
+        __syncwarp();
+        U = warp_keep_ge(g, U, x, lane);
+    }
+    return warp_rank_topk(g, U, k, sel, lane);
+}
+
+// The CTA's next prediction from a finished row's best keys sel[0..n)
+// (descending): the value that about 2.5 k elements of a row like it reach.
+// Near the top of a row the values fall about linearly in the log of the
+// rank, so the drop from rank k/2 to rank k, scaled by log(2.5k / k) /
+// log(k / (k/2)), extrapolates to rank 2.5 k.  A row that failed its
+// prediction (fewer than k kept at or above it) lowers the next one below
+// its last kept value by twice the same spread.  0 when there is no basis.
+__device__ __forceinline__ uint64_t next_prediction(const uint64_t* sel, int n, int k, bool held) {
+    if (n < 2) return 0ull;
+    const int last = (held ? k : n) - 1;
+    const int mid = last / 2;
+    const float vl = key_value(sel[last]), vm = key_value(sel[mid]);
+    const float d = vm - vl;
+    if (!(d > 0.0f)) return 0ull;
+    const float f = held ? logf(2.5f * (float)(last + 1)) - logf((float)(last + 1)) : 2.0f * logf((float)(last + 1) / (float)(mid + 1));
+    const float v = vl - d * f / logf((float)(last + 1) / (float)(mid + 1));
+    if (!(v > -3.0e38f) || !(v < 3.0e38f)) return 0ull;
+    return (uint64_t)ord_of_float(__fadd_rn(v, 0.0f)) << 32;
+}
+
 // The last finishing warp of a split row: the best min(k, U) keys of the U
-// keys its segments published, into sel[] (descending); rowbad gets the OR
-// of the segments' flags.  Segment t's keys occupy indices [excl_t,
-// excl_t + count_t) of the merged order (lane t holds excl_t; S <= 16).
-__device__ __noinline__ int merge_partials(const RowJob& J, int64_t row, uint64_t* sel, uint32_t& rowbad, int lane) {
-    const size_t p0 = (size_t)row * J.S;
-    const int c_l = lane < J.S ? __ldcg(J.part_count + p0 + lane) : 0;
-    rowbad = __reduce_or_sync(kFull, lane < J.S ? __ldcg(J.part_flags + p0 + lane) : 0u);
+// keys its pieces published, into sel[] (descending); rowbad gets the OR of
+// the pieces' flags and `spec` the largest predicted threshold any piece
+// was filtered by.  Piece t's keys sit in part slot slot_t and occupy
+// indices [excl_t, excl_t + count_t) of the merged order (lane t holds
+// both; at most kPipeMaxPieces pieces).
+struct Merged {
+    int n;
+    uint32_t rowbad;
+    uint64_t spec;
+};
+__device__ __noinline__ Merged merge_pieces(const RowJob& J, int64_t T, int64_t G, int64_t nu, int64_t row,
+                                            int64_t first_cta, int np, uint64_t* sel, int lane) {
+    CtaRange c;
+    c.T = T;
+    c.G = G;
+    c.nu = nu;
+    const int64_t myslot = lane < np ? part_slot(c, first_cta + lane, row) : 0;
+    const int c_l = lane < np ? __ldcg(J.part_count + myslot) : 0;
+    const uint32_t rowbad = __reduce_or_sync(kFull, lane < np ? __ldcg(J.part_flags + myslot) : 0u);
+    uint64_t sp = lane < np ? (uint64_t)__ldcg(reinterpret_cast<const unsigned long long*>(J.part_spec) + myslot) : 0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t t = __shfl_xor_sync(kFull, sp, o);
+        sp = t > sp ? t : sp;
+    }
     int incl = c_l;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -2177,19 +2733,20 @@ __device__ __noinline__ int merge_partials(const RowJob& J, int64_t row, uint64_
     const int U = __shfl_sync(kFull, incl, 31);
     const int excl = incl - c_l;
     const int kk = J.k;
-    const unsigned long long* pbase = reinterpret_cast<const unsigned long long*>(J.part_keys + p0 * kk);
+    const unsigned long long* pbase = reinterpret_cast<const unsigned long long*>(J.part_keys);
     uint64_t ra = ~0ull, rb = ~0ull;
     for (int base = 0; base < U; base += 64) {
         const int ga = base + lane, gb = base + 32 + lane;
         int sa = 0, sg = 0;
-        for (int t = 1; t < J.S; ++t) {
+        for (int t = 1; t < np; ++t) {
             const int e = __shfl_sync(kFull, excl, t);
             sa = (e <= ga) ? t : sa;
             sg = (e <= gb) ? t : sg;
         }
         const int ea = __shfl_sync(kFull, excl, sa), eb = __shfl_sync(kFull, excl, sg);
-        uint64_t xa = ga < U ? ~(uint64_t)__ldcg(pbase + (size_t)sa * kk + (ga - ea)) : ~0ull;
-        uint64_t xb = gb < U ? ~(uint64_t)__ldcg(pbase + (size_t)sg * kk + (gb - eb)) : ~0ull;
+        const int64_t pa = __shfl_sync(kFull, myslot, sa), pb = __shfl_sync(kFull, myslot, sg);
+        uint64_t xa = ga < U ? ~(uint64_t)__ldcg(pbase + (size_t)pa * kk + (ga - ea)) : ~0ull;
+        uint64_t xb = gb < U ? ~(uint64_t)__ldcg(pbase + (size_t)pb * kk + (gb - eb)) : ~0ull;
         warp_sort64(xa, xb, lane);
         if (base == 0) {
             ra = xa;
@@ -2205,7 +2762,17 @@ __device__ __noinline__ int merge_partials(const RowJob& J, int64_t row, uint64_
     if (lane < n) sel[lane] = ~ra;
     if (lane + 32 < n) sel[lane + 32] = ~rb;
     __syncwarp();
-    return n;
+    return Merged{n, rowbad, sp};
+}
+
+// The slot's per-piece state starts afresh for its next piece (one thread).
+__device__ __forceinline__ void slot_reset(PipeShared& P, int slot) {
+    P.bad[slot] = 0u;
+    P.tau[slot] = 0ull;
+    P.used[slot] = 0ull;
+    P.boot_cnt[slot] = 0;
+    P.boot_ready[slot] = 0u;
+    P.mode[slot] = 0u;
 }
 
 // Finishing warp f.
@@ -2214,75 +2781,142 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
                             int lane) {
     uint64_t* sel = reinterpret_cast<uint64_t*>(scratch);            // [kPipeMaxK]
     double* wd = reinterpret_cast<double*>(sel + kPipeMaxK);         // [kPipeMaxK]
-    unsigned char* tail = reinterpret_cast<unsigned char*>(wd + kPipeMaxK);
+    uint64_t* gat = reinterpret_cast<uint64_t*>(wd + kPipeMaxK);     // [kPGather]
+    unsigned char* tail = reinterpret_cast<unsigned char*>(gat + kPGather);
     FinishShared unused_fs;
-    const int64_t nitems = J.rows * J.S;
+    PipeList L = pipe_list<T>(J);
     const int slot = f;
     const uint64_t* sbuf = slots + (size_t)slot * kPipeConsumers * J.cap_w;
     uint32_t use = 0;
-    for (int64_t it = blockIdx.x + (int64_t)f * gridDim.x; it < nitems; it += (int64_t)kPipeFinishers * gridDim.x) {
-        const int64_t row = it / J.S;
-        const int seg = (int)(it % J.S);
-        const int32_t req = (int32_t)(row / J.rpr);
+    int64_t row = 0;
+    bool redo = false;
+    for (int64_t i = 0;; ++i) {
+        if (i == L.nmain) {
+            // this finisher's main items are done (their failed rows recorded):
+            // the second one to get here opens the redo pass
+            if (lane == 0 && atomicAdd(&P.fin_done, 1) == kPipeFinishers - 1) {
+                __threadfence_block();
+                st_release_shared(&P.redo_ready, 1u);
+            }
+            __syncwarp();
+        }
+        if (!pipe_item<T>(J, P, L, i, row, redo)) break;
+        if ((int)(i % kPipeSlots) != slot) continue;
         if (!item_active<MODE>(J, row)) continue;  // nothing to filter (the tails run afterwards)
+        const int32_t req = (int32_t)(row / J.rpr);
         uint32_t rowbad = 2u;
+        uint64_t spec = 0ull;
         int n = 0;
         const bool ok = pipe_wait_warp(&P.slot_full[slot], use & 1u, P);
         ++use;
         if (ok) {
-            int cw[kPipeConsumers];
-            int U = 0;
-#pragma unroll
-            for (int w = 0; w < kPipeConsumers; ++w) {
-                cw[w] = P.cnt[slot][w];
-                U += cw[w];
-            }
+            // gather the keys at or above the piece's best threshold into this
+            // warp's scratch, hand the slot back, then select from the copy
+            const uint64_t tf = P.tau[slot];
             rowbad = P.bad[slot];
-            const int cap_w = J.cap_w;
-            auto get = [&](int g) -> uint64_t {
-                int w = 0, off = g;
-#pragma unroll
-                for (int t = 0; t < kPipeConsumers - 1; ++t) {
-                    if (w == t && off >= cw[t]) {
-                        off -= cw[t];
-                        w = t + 1;
-                    }
+            spec = P.used[slot];
+            int U = 0;
+            for (int w = 0; w < kPipeConsumers; ++w) {
+                const int cw = P.cnt[slot][w];
+                const uint64_t* wb = sbuf + (size_t)w * J.cap_w;
+                for (int base = 0; base < cw; base += 32) {
+                    const uint64_t key = base + lane < cw ? wb[base + lane] : 0ull;
+                    const bool keep = base + lane < cw && key >= tf;
+                    const unsigned bal = __ballot_sync(kFull, keep);
+                    const int at = U + __popc(bal & lanemask_lt());
+                    if (keep && at < kPGather) gat[at] = key;
+                    U += __popc(bal);
                 }
-                return sbuf[(size_t)w * cap_w + off];
-            };
-            n = warp_topk64(U, J.k, get, sel, lane);
+            }
             __syncwarp();
-            if (lane == 0) {
-                P.bad[slot] = 0u;
-                mbar_arrive(&P.slot_empty[slot]);
+            if (U <= kPGather) {
+                if (lane == 0) {
+                    slot_reset(P, slot);
+                    mbar_arrive(&P.slot_empty[slot]);
+                }
+                n = warp_select_topk(gat, U, J.k, sel, lane);
+            } else {  // more keys than the scratch holds: select from the slot itself
+                int cw[kPipeConsumers];
+                U = 0;
+#pragma unroll
+                for (int w = 0; w < kPipeConsumers; ++w) {
+                    cw[w] = P.cnt[slot][w];
+                    U += cw[w];
+                }
+                const int cap_w = J.cap_w;
+                auto get = [&](int g) -> uint64_t {
+                    int w = 0, off = g;
+#pragma unroll
+                    for (int t = 0; t < kPipeConsumers - 1; ++t) {
+                        if (w == t && off >= cw[t]) {
+                            off -= cw[t];
+                            w = t + 1;
+                        }
+                    }
+                    return sbuf[(size_t)w * cap_w + off];
+                };
+                n = warp_topk64(U, J.k, get, sel, lane);
+                __syncwarp();
+                if (lane == 0) {
+                    slot_reset(P, slot);
+                    mbar_arrive(&P.slot_empty[slot]);
+                }
             }
         } else if (lane == 0) {
             atomicExch(&P.abort, 1);
         }
-        if (J.S > 1) {
-            // publish this segment's best; the last segment of the row merges
-            const size_t pslot = (size_t)row * J.S + seg;
-            uint64_t* pk = J.part_keys + pslot * J.k;
+        const Piece p = redo ? whole_row<T>(J, L.cr, row) : piece_of<T>(J, L.cr, row);
+        if (p.np > 1) {
+            // publish this piece's best; the last piece of the row merges
+            const int64_t ps = part_slot(L.cr, L.cr.b, row);
+            uint64_t* pk = J.part_keys + ps * J.k;
             if (lane < n) pk[lane] = sel[lane];
             if (lane + 32 < n) pk[lane + 32] = sel[lane + 32];
             __syncwarp();
             int last = 0;
             if (lane == 0) {
-                J.part_count[pslot] = n;
-                J.part_flags[pslot] = rowbad;
+                J.part_count[ps] = n;
+                J.part_flags[ps] = rowbad;
+                J.part_spec[ps] = spec;
                 __threadfence();
-                const uint32_t t = atomicAdd(J.row_ticket + row, 1u);
-                last = (t == (uint32_t)(J.S - 1));
+                const uint32_t t = atomicAdd(J.row_ticket + p.first_cta, 1u);
+                last = (t == (uint32_t)(p.np - 1));
                 if (last) {
-                    atomicExch(J.row_ticket + row, 0u);
+                    atomicExch(J.row_ticket + p.first_cta, 0u);
                     __threadfence();
                 }
             }
             last = __shfl_sync(kFull, last, 0);
             if (!last) continue;
-            n = merge_partials(J, row, sel, rowbad, lane);
+            const Merged m = merge_pieces(J, L.cr.T, L.cr.G, L.cr.nu, row, p.first_cta, p.np, sel, lane);
+            n = m.n;
+            rowbad = m.rowbad;
+            spec = m.spec;
         }
-        finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, tail, unused_fs, lane);
+        // a predicted threshold holds when the row's k-th kept key reaches it:
+        // then at least k elements of the row do, and none of the top k was
+        // dropped.  Otherwise the row is read again, whole, in the redo pass.
+        const bool held = !(spec != 0ull && rowbad == 0u && (n < J.k || sel[J.k - 1] < spec));
+        if (L.spec_ok && rowbad == 0u && lane == 0) {
+            // the row's best values set the prediction of the pieces that follow
+            // (and of the next call); no basis leaves it as it is
+            const uint64_t t = next_prediction(sel, n, J.k, held);
+            if (t != 0ull) {
+                P.spec = t;
+                __threadfence_block();
+                st_release_shared(&P.spec_set, 1u);
+            }
+        }
+        if (!held) {
+            if (lane == 0) {
+                const int at = atomicAdd(&P.redo_n, 1);
+                J.redo[L.rbase + at] = (int32_t)row;
+                __threadfence();
+            }
+            __syncwarp();
+            continue;
+        }
+        finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, tail, unused_fs, lane, gat);
     }
 }
 
@@ -2303,10 +2937,15 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_cons
         for (int s = 0; s < kPipeSlots; ++s) {
             mbar_init(&P.slot_full[s], kPipeConsumers);
             mbar_init(&P.slot_empty[s], 1);
-            P.bad[s] = 0u;
+            slot_reset(P, s);
         }
-        P.tau[0] = 0ull;
-        P.tau[1] = 0ull;
+        // the prediction this CTA left at the end of the previous call
+        const uint64_t h = J.hint != nullptr ? J.hint[blockIdx.x] : 0ull;
+        P.spec = h;
+        P.spec_set = h != 0ull ? 1u : 0u;
+        P.fin_done = 0;
+        P.redo_n = 0;
+        P.redo_ready = 0u;
         P.abort = 0;
         fence_mbar_init();
     }
@@ -2319,6 +2958,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_cons
         const int f = warp - 1 - kPipeConsumers;
         pipe_finish<T, MODE>(J, P, slots, fin + (size_t)f * J.fin_stride, f, lane);
     }
+    // carry this CTA's latest prediction to the next call (a hint only: the
+    // rows it predicts are checked exactly)
+    __syncthreads();
+    if (threadIdx.x == 0 && J.hint != nullptr && P.spec_set != 0u && P.abort == 0) J.hint[blockIdx.x] = P.spec;
 }
 
 // ---------------------------------------------------------------------------
@@ -2540,22 +3183,30 @@ constexpr int64_t kCounterWords = UNO_WORKSPACE_COUNTER_BYTES / 4;
 constexpr int64_t kRowCounterWords = kCounterWords / 2;
 
 struct WsLayout {
-    size_t row_ticket, req_ticket, part_keys, part_count, part_flags, c_ids, c_probs, c_count, c_flags, total;
+    size_t row_ticket, req_ticket, part_keys, part_count, part_flags, part_spec, redo, c_ids, c_probs, c_count,
+        c_flags, total;
 };
 
 static WsLayout ws_layout(int64_t rows, int32_t k, bool compact) {
     WsLayout L{};
     const int sb = split_bound(rows);
-    const size_t nslot = sb > 1 ? (size_t)rows * sb : 0;
+    // part slots: split rows of the general kernel (rows x splits) or of the
+    // pipelined kernel (two per CTA)
+    size_t nslot = sb > 1 ? (size_t)rows * sb : 0;
+    if (nslot < (size_t)2 * kPipeMaxGrid) nslot = (size_t)2 * kPipeMaxGrid;
     L.row_ticket = 0;
     L.req_ticket = (size_t)kRowCounterWords * 4;
-    size_t off = (size_t)UNO_WORKSPACE_COUNTER_BYTES;
+    size_t off = (size_t)UNO_WORKSPACE_COUNTER_BYTES + UNO_WORKSPACE_HINT_BYTES;
     L.part_keys = off;
     off = align_up(off + nslot * (size_t)k * 8, 256);
     L.part_count = off;
     off = align_up(off + nslot * 4, 256);
     L.part_flags = off;
     off = align_up(off + nslot * 4, 256);
+    L.part_spec = off;
+    off = align_up(off + nslot * 8, 256);
+    L.redo = off;
+    off = align_up(off + ((size_t)rows + kPipeMaxGrid) * 4, 256);
     L.c_ids = off;
     const size_t crow = compact ? (size_t)rows : 0;
     const size_t ks = (size_t)((k + 3) & ~3);
@@ -2597,32 +3248,24 @@ static size_t row_smem_bytes(RowJob& J) {
     return (size_t)J.fin_off + finish;
 }
 
-// The pipelined kernel: segments per row, ring depth and shared memory.
+// The pipelined kernel: grid (balanced pieces), ring depth and shared memory.
 // Returns UNO_ERR_UNSUPPORTED (nothing launched) when it does not fit.
 template <typename T, int MODE>
 static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     J.hw = J.k + 16 > 64 ? J.k + 16 : 64;
-    J.cap_w = J.hw + 64;  // a round of unit appends that fits, else one element per lane per round
-    const int G = sm_count();
-    // segments per row, only when rows are fewer than the SMs: spread the
-    // items over the SMs, each segment at least one full stage, a price per
-    // extra segment (its seed and the merge)
-    int smax = J.rows <= kRowCounterWords ? split_bound(J.rows) : 1;
-    const int64_t by_work = J.vocab / Elem<T>::kPerUnit / kPStageUnits;
-    if (smax > by_work) smax = by_work < 1 ? 1 : (int)by_work;
-    int S = 1;
-    if (J.rows < G) {
-        double best = 1e300;
-        for (int s = 1; s <= smax; ++s) {
-            const int64_t rounds = (J.rows * s + G - 1) / G;
-            const double cost = (double)rounds / s + 0.03 * (s - 1);
-            if (cost < best - 1e-9) {
-                best = cost;
-                S = s;
-            }
-        }
+    J.cap_w = J.hw + 32;  // a stage's candidates that fit are written at once, else appended with compaction
+    // one CTA per SM; with fewer rows than SMs, pieces of at least
+    // kPipeMinPieceUnits and at most kPipeMaxPieces per row
+    int64_t grid = sm_count() < kPipeMaxGrid ? sm_count() : kPipeMaxGrid;
+    if (J.rows < grid) {
+        const int64_t nu = J.vocab / Elem<T>::kPerUnit > 0 ? J.vocab / Elem<T>::kPerUnit : 1;
+        int64_t g = J.rows * nu / kPipeMinPieceUnits;
+        if (g > J.rows * (kPipeMaxPieces - 2)) g = J.rows * (kPipeMaxPieces - 2);
+        if (g < J.rows) g = J.rows;
+        if (g < grid) grid = g;
     }
-    J.S = S;
+    J.S = 1;
+    if (J.hint != nullptr) J.hint += (size_t)MODE * kPipeMaxGrid;  // each entry point keeps its own
     // shared memory: ring | candidate slots | per finisher: sel, wd, tail
     const size_t slot_bytes = (size_t)kPipeSlots * kPipeConsumers * J.cap_w * 8;
     size_t tail = 0;
@@ -2631,7 +3274,7 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     else if (MODE == kModeTree)
         tail = 16 + (size_t)J.V * J.ks * 8 + (size_t)J.V * 12 + (size_t)(J.B + 1) * 8;
     const size_t dyn_max = 227 * 1024 - sizeof(PipeShared);
-    auto stride_of = [](size_t tb) { return align_up((size_t)2 * kPipeMaxK * 8 + tb, 128); };
+    auto stride_of = [](size_t tb) { return align_up((size_t)2 * kPipeMaxK * 8 + (size_t)kPGather * 8 + tb, 128); };
     auto stages_of = [&](size_t tb) -> int64_t {
         const size_t fixed = slot_bytes + (size_t)kPipeFinishers * stride_of(tb);
         return fixed >= dyn_max ? 0 : (int64_t)((dyn_max - fixed) / kPStageBytes);
@@ -2647,8 +3290,6 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     auto kern = pipe_kernel<T, MODE>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
         return UNO_ERR_CUDA;
-    const int64_t items = J.rows * S;
-    const int64_t grid = items < G ? items : G;
     if (grid <= 0) return UNO_OK;
     kern<<<(unsigned)grid, kPipeThreads, dyn, stream>>>(J);
     if (cudaGetLastError() != cudaSuccess) return UNO_ERR_CUDA;
@@ -2718,6 +3359,9 @@ static void bind_workspace(RowJob& J, void* ws, const WsLayout& L) {
     J.part_keys = reinterpret_cast<uint64_t*>(b + L.part_keys);
     J.part_count = reinterpret_cast<int32_t*>(b + L.part_count);
     J.part_flags = reinterpret_cast<uint32_t*>(b + L.part_flags);
+    J.part_spec = reinterpret_cast<uint64_t*>(b + L.part_spec);
+    J.redo = reinterpret_cast<int32_t*>(b + L.redo);
+    J.hint = reinterpret_cast<uint64_t*>(b + UNO_WORKSPACE_COUNTER_BYTES);
     J.c_ids = reinterpret_cast<int32_t*>(b + L.c_ids);
     J.ks = (J.k + 3) & ~3;
     J.c_probs = reinterpret_cast<float*>(b + L.c_probs);

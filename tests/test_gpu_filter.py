@@ -134,3 +134,23 @@ def test_repeated_calls_reuse_the_workspace():
         assert torch.equal(o["ids"], outs[0]["ids"]) and torch.equal(o["probs"], outs[0]["probs"])
     r = oracle.filter_softmax(np_of(x.view(torch.int16)).view(np.uint16), "bf16", 1.0, 50, 0.95, rng=(5, 3))
     assert np.array_equal(np_of(outs[3]["sample"]), r["sample"])
+
+
+@pytest.mark.parametrize("dtype,rows,vocab,k,p,pattern", [
+    ("bf16", 600, 20000, 8, 0.9, (1.0, 20.0)),
+    ("f32", 600, 20000, 8, 0.9, (1.0, 1.0, 1.0, 20.0, 20.0, 20.0)),
+    ("bf16", 400, 70001, 16, 0.95, (30.0, 1.0, 1.0)),
+    ("f32", 450, 40000, 50, 0.95, (1.0, 25.0)),
+])
+def test_rows_of_changing_scale_match_oracle(dtype, rows, vocab, k, p, pattern):
+    """Consecutive rows of very different scale: a threshold predicted from
+    one row is far too high or far too low for the next, so rows are re-read
+    in the redo pass or flood the candidate buffers.  Results must still
+    equal the oracle's."""
+    rng = np.random.default_rng(rows + vocab + k)
+    scale = np.resize(np.asarray(pattern, dtype=np.float32), rows)[:, None]
+    x = _encode(_rows(rng, rows, vocab, scale=1.0, peak=4.0) * scale, dtype)
+    ev = Events()
+    g, r = _run(x, dtype, 1.0, k, p, rpr=3, rng=(77, 2))
+    compare_filter(g, r, ev, sample=True)
+    ev.check()
