@@ -101,7 +101,7 @@ typedef struct {
 
 #define UNO_MAX_TOP_K 1024
 #define UNO_WORKSPACE_COUNTER_BYTES (1 << 20)
-#define UNO_WORKSPACE_HINT_BYTES 8192
+#define UNO_WORKSPACE_HINT_BYTES 16384
 #define UNO_MAX_TREE_NODES 128   /* V <= 128   ([eval guide, 启动期硬性约束]) */
 #define UNO_MAX_TREE_FRONTIER 2048 /* V*K <= 2048 (same section) */
 
@@ -166,6 +166,47 @@ uno_status uno_linear_verify(const void* target_logits, uno_dtype dt, int32_t R,
                              const float* q_probs, const int32_t* q_count, int32_t q_cap, uno_rng rng,
                              int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
                              uint32_t* out_flags, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * uno_linear_cycle -- one whole linear cycle: filter the draft marginals and
+ * draw the proposals, filter the target rows, and verify, in one launch over
+ * all the cycle's rows (then one short launch for the request decisions).
+ * [UNO PR, Motivation]: one model, two forward passes per cycle; the
+ * diffusion pass drafts B tokens and produces the first output token, the
+ * autoregressive pass verifies; [UNO PR, Modifications]: the B + 1 output
+ * layout and the counters (num_correct_drafts = accept_len - 2).
+ *
+ * layout UNO_LAYOUT_GENERIC: B draft rows and B + 1 target rows per request;
+ *   every proposal x_i is tested against target row i, target row B gives
+ *   the bonus (uno_filter_softmax with a draw, then uno_linear_verify).
+ * layout UNO_LAYOUT_TWO_PASS: B draft rows and B target rows per request, the
+ *   pages' layout: draft row 0 comes from the base weights and its draw x_0
+ *   is emitted untested; target row i - 1 (the distribution of output token
+ *   i) tests proposal x_i (i = 1 .. B-1); if all are accepted target row
+ *   B - 1 gives the bonus with the target draw at position B.
+ * Draws: proposal i with (request, i, PROPOSAL), its test with (request, i,
+ *   ACCEPT), the correction with (request, i, RESIDUAL), the bonus with
+ *   (request, B, TARGET), as in the separate calls.
+ *
+ * draft_logits  [R][B][vocab]; target_logits [R][B+1][vocab] (generic) or
+ *               [R][B][vocab] (two-pass); dtype dt, contiguous.
+ * out_tokens    [R][B+1] emitted tokens, unused slots -1.
+ * out_num_accepted [R]: proposals accepted by the test (generic: the
+ *               accept length in [0, B]; two-pass: num_correct_drafts in
+ *               [0, B-1], x_0 not counted).
+ * out_num_tokens [R]: tokens emitted (two-pass: the pages' accept_len).
+ * out_flags     [R]: OR of the flags of the request's draft rows, target rows
+ *               and decisions.
+ * out_draft_ids [R][B] the proposals (nullable).
+ * workspace     see uno_linear_cycle_workspace_bytes (same rules as above).
+ * ---------------------------------------------------------------------- */
+#define UNO_LAYOUT_GENERIC 0
+#define UNO_LAYOUT_TWO_PASS 1
+size_t uno_linear_cycle_workspace_bytes(int32_t R, int32_t B, int64_t vocab, int32_t top_k, int32_t layout);
+uno_status uno_linear_cycle(const void* draft_logits, const void* target_logits, uno_dtype dt, int32_t R, int32_t B,
+                            int64_t vocab, int32_t layout, uno_sampling_params sp, uno_rng rng, int32_t* out_tokens,
+                            int32_t* out_num_accepted, int32_t* out_num_tokens, uint32_t* out_flags,
+                            int32_t* out_draft_ids, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * uno_tree_topk_expand -- top-K candidates per marginal and a V-node tree.

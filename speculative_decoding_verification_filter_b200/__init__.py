@@ -6,6 +6,8 @@ generator used by the tests and the benchmark.
 """
 from ._binding import (  # noqa: F401
     EXPORTED,
+    LAYOUT_GENERIC,
+    LAYOUT_TWO_PASS,
     FLAG_BAD_TREE,
     FLAG_DRAFT_NOT_IN_SUPPORT,
     FLAG_NONFINITE_ROW,
@@ -14,6 +16,7 @@ from ._binding import (  # noqa: F401
     UnoError,
     load_library,
     uno_filter_softmax,
+    uno_linear_cycle,
     uno_linear_verify,
     uno_linear_verify_noalloc,
     uno_tree_suffix_attention_merge,

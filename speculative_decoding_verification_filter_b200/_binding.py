@@ -28,6 +28,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported argument", 3: "CUDA la
 EXPORTED = (
     "uno_filter_softmax_workspace_bytes", "uno_filter_softmax",
     "uno_linear_verify_workspace_bytes", "uno_linear_verify",
+    "uno_linear_cycle_workspace_bytes", "uno_linear_cycle",
     "uno_tree_topk_expand",
     "uno_tree_verify_workspace_bytes", "uno_tree_verify",
     "uno_linear_verify_noalloc",
@@ -82,6 +83,11 @@ def load_library():
         lib.uno_linear_verify.argtypes = [P, ctypes.c_int, i32, i32, i64, _Params, P, P, P, P, i32, _Rng,
                                           P, P, P, P, P, sz, P]
         lib.uno_linear_verify.restype = ctypes.c_int
+        lib.uno_linear_cycle_workspace_bytes.argtypes = [i32, i32, i64, i32, i32]
+        lib.uno_linear_cycle_workspace_bytes.restype = sz
+        lib.uno_linear_cycle.argtypes = [P, P, ctypes.c_int, i32, i32, i64, i32, _Params, _Rng, P, P, P, P, P, P, sz,
+                                         P]
+        lib.uno_linear_cycle.restype = ctypes.c_int
         lib.uno_tree_topk_expand.argtypes = [P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P, P]
         lib.uno_tree_topk_expand.restype = ctypes.c_int
         lib.uno_tree_verify_workspace_bytes.argtypes = [i32, i32, i64, i32]
@@ -251,6 +257,42 @@ def uno_linear_verify(target_logits, draft_ids, q_ids, q_probs, q_count, *, R, B
                                ctypes.c_void_p(stream.cuda_stream))
     _check("uno_linear_verify", st)
     return _host_back(dict(tokens=toks, accept_len=acc, num_tokens=ntok, flags=flags), host)
+
+
+LAYOUT_GENERIC, LAYOUT_TWO_PASS = 0, 1
+
+
+def uno_linear_cycle(draft_logits, target_logits, *, R, B, temperature, top_k, top_p, rng, layout=LAYOUT_GENERIC):
+    """One linear cycle in one call: draft_logits [R*B, vocab] (or [R, B,
+    vocab]); target_logits [R*(B+1), vocab] for layout LAYOUT_GENERIC, [R*B,
+    vocab] for LAYOUT_TWO_PASS (x_0 untested, target row i-1 tests x_i).
+    Returns dict(tokens [R, B+1], num_accepted [R], num_tokens [R], flags [R],
+    drafts [R, B])."""
+    lib = load_library()
+    _need(R >= 1 and B >= 1 and layout in (LAYOUT_GENERIC, LAYOUT_TWO_PASS), "R, B >= 1 and a known layout")
+    host = not draft_logits.is_cuda
+    device = _device_of(draft_logits, target_logits)
+    d = _dev(draft_logits, device).contiguous()
+    t = _dev(target_logits, device).contiguous()
+    vocab = d.shape[-1]
+    _need(t.shape[-1] == vocab and d.dtype == t.dtype, "draft and target logits share vocab and dtype")
+    _need(d.numel() == R * B * vocab, "draft_logits must hold R*B rows")
+    _need(t.numel() == R * (B + 1 - layout) * vocab, "target_logits must hold R*(B+1) rows (R*B two-pass)")
+    stream = torch.cuda.current_stream(device)
+    kw = dict(dtype=torch.int32, device=device)
+    toks = torch.empty((R, B + 1), **kw)
+    nacc = torch.empty(R, **kw)
+    ntok = torch.empty(R, **kw)
+    flags = torch.empty(R, **kw)
+    drafts = torch.empty((R, B), **kw)
+    nbytes = lib.uno_linear_cycle_workspace_bytes(R, B, vocab, int(top_k), int(layout))
+    ws = workspace(nbytes, device, stream)
+    st = lib.uno_linear_cycle(_ptr(d), _ptr(t), _dtype_code(d), R, B, vocab, int(layout),
+                              _Params(float(temperature), int(top_k), float(top_p)), _rng(rng), _ptr(toks),
+                              _ptr(nacc), _ptr(ntok), _ptr(flags), _ptr(drafts), _ptr(ws), ws.numel(),
+                              ctypes.c_void_p(stream.cuda_stream))
+    _check("uno_linear_cycle", st)
+    return _host_back(dict(tokens=toks, num_accepted=nacc, num_tokens=ntok, flags=flags, drafts=drafts), host)
 
 
 def uno_tree_topk_expand(q_ids, q_probs, q_count, *, R, B, K, V):

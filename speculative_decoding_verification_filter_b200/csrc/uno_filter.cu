@@ -31,7 +31,7 @@
 
 namespace uno {
 
-enum Mode { kModeFilter = 0, kModeLinear = 1, kModeTree = 2 };
+enum Mode { kModeFilter = 0, kModeLinear = 1, kModeTree = 2, kModeCycle = 3 };
 
 
 struct RowJob {
@@ -75,8 +75,15 @@ struct RowJob {
     int32_t ks;            // their row stride: k rounded up to a multiple of 4 (16-byte rows)
     int32_t* c_count;      // [rows]
     uint32_t* c_flags;     // [rows]
+    // a whole cycle in one launch: rows [0, nq2) are draft rows from `logits`
+    // (filtered, one proposal drawn each), rows [nq2, rows) target rows from
+    // `logits2` (rows past nq2 count from its start)
+    const unsigned char* logits2;
+    int64_t nq2;
     // linear verification
     int32_t B;
+    int32_t sh;                  // 1: the two-pass layout (x_0 untested, target row i-1 tests x_i)
+    const uint32_t* q_flags;     // flags of the draft rows (nullable)
     const int32_t* draft_ids;
     const int32_t* q_ids;
     const float* q_probs;
@@ -312,7 +319,9 @@ struct RowGeom {
 template <typename T>
 __device__ __forceinline__ RowGeom row_geom(const RowJob& J, int64_t row) {
     RowGeom g;
-    g.base = J.logits + (size_t)row * (size_t)J.row_stride * Elem<T>::kBytes;
+    g.base = (J.logits2 == nullptr || row < J.nq2)
+                 ? J.logits + (size_t)row * (size_t)J.row_stride * Elem<T>::kBytes
+                 : J.logits2 + (size_t)(row - J.nq2) * (size_t)J.row_stride * Elem<T>::kBytes;
     const uintptr_t addr = reinterpret_cast<uintptr_t>(g.base);
     int64_t head = (int64_t)(((16u - (addr & 15u)) & 15u) / Elem<T>::kBytes);
     if (head > J.vocab) head = J.vocab;
@@ -607,21 +616,38 @@ __device__ __forceinline__ double lookup_sorted(const int32_t* ids, const float*
     return 0.0;
 }
 
+// Linear verification of request r from global memory (one warp): any k, any
+// B.  Generic layout (sh = 0): target row i tests proposal x_i, row B gives
+// the bonus.  Two-pass layout (sh = 1): x_0 is emitted untested, row i - 1
+// tests x_i, row B - 1 gives the bonus.
 __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd, int lane) {
     const int32_t B = J.B;
-    const int64_t base = (int64_t)r * (B + 1);
+    const int sh = J.sh;
+    const int64_t base = (int64_t)r * (B + 1 - sh);
     uint32_t flags = 0;
-    for (int i = lane; i <= B; i += 32) flags |= __ldcg(J.c_flags + base + i);
+    for (int i = lane; i <= B - sh; i += 32) flags |= __ldcg(J.c_flags + base + i);
+    if (J.q_flags != nullptr)
+        for (int i = lane; i < B; i += 32) flags |= __ldcg(J.q_flags + (int64_t)r * B + i);
     flags = __reduce_or_sync(kFull, flags);
     int32_t acc = B, ntok = B + 1;
     int32_t* toks = J.out_tokens + (size_t)r * (B + 1);
     for (int i = lane; i <= B; i += 32) toks[i] = -1;
     __syncwarp();
     bool stopped = false;
-    for (int i = 0; i < B && !stopped; ++i) {
-        const int pc = __ldcg(J.c_count + base + i);
-        const int32_t* pid = J.c_ids + (size_t)(base + i) * J.ks;
-        const float* ppr = J.c_probs + (size_t)(base + i) * J.ks;
+    if (sh == 1) {
+        // the base-weights token, untested
+        if (__ldcg(J.q_count + (int64_t)r * B) > 0) {
+            if (lane == 0) toks[0] = __ldcg(J.draft_ids + (size_t)r * B);
+        } else {
+            acc = 0;
+            ntok = 0;
+            stopped = true;
+        }
+    }
+    for (int i = sh; i < B && !stopped; ++i) {
+        const int pc = __ldcg(J.c_count + base + i - sh);
+        const int32_t* pid = J.c_ids + (size_t)(base + i - sh) * J.ks;
+        const float* ppr = J.c_probs + (size_t)(base + i - sh) * J.ks;
         if (pc == 0) {
             acc = i;
             ntok = i;
@@ -629,11 +655,11 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
             break;
         }
         const int64_t qrow = (int64_t)r * B + i;
-        int qc = J.q_count[qrow];
+        int qc = __ldcg(J.q_count + qrow);
         qc = qc < 0 ? 0 : (qc > J.q_cap ? J.q_cap : qc);
         const int32_t* qid = J.q_ids + (size_t)qrow * J.q_cap;
         const float* qpr = J.q_probs + (size_t)qrow * J.q_cap;
-        const int32_t x = J.draft_ids[(size_t)r * B + i];
+        const int32_t x = __ldcg(J.draft_ids + (size_t)r * B + i);
         const bool xin = x >= 0 && (int64_t)x < J.vocab;
         const double a = xin ? lookup_sorted(qid, qpr, qc, x) : 0.0;
         const double px = xin ? lookup_sorted(pid, ppr, pc, x) : 0.0;
@@ -648,7 +674,7 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
             if (lane == 0) toks[i] = x;
             continue;
         }
-        // residual max(0, p_i - q_i) over supp p_i (ascending ids)
+        // residual max(0, p - q_i) over supp p (ascending ids)
         for (int j = lane; j < pc; j += 32) {
             const double d = (double)__ldcg(ppr + j) - lookup_sorted(qid, qpr, qc, __ldcg(pid + j));
             wd[j] = d > 0.0 ? d : 0.0;
@@ -673,12 +699,12 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
         stopped = true;
     }
     if (!stopped) {
-        const int pc = __ldcg(J.c_count + base + B);
+        const int pc = __ldcg(J.c_count + base + B - sh);
         if (pc == 0) {
             ntok = B;
         } else if (lane == 0) {
-            const int32_t* pid = J.c_ids + (size_t)(base + B) * J.ks;
-            const float* ppr = J.c_probs + (size_t)(base + B) * J.ks;
+            const int32_t* pid = J.c_ids + (size_t)(base + B - sh) * J.ks;
+            const float* ppr = J.c_probs + (size_t)(base + B - sh) * J.ks;
             for (int j = 0; j < pc; ++j) wd[j] = (double)__ldcg(ppr + j);
             const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)B, kDrawTarget, J.cycle);
             const int pick = inv_cdf_serial(wd, pc, u);
@@ -686,7 +712,7 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
         }
     }
     if (lane == 0) {
-        J.out_accept_len[r] = acc;
+        J.out_accept_len[r] = acc > sh ? acc - sh : 0;
         J.out_num_tokens[r] = ntok;
         J.out_req_flags[r] = flags;
     }
@@ -939,6 +965,8 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     const int kc = J.k, ks = J.ks;
     constexpr int QS = 64;  // q entries kept per row
     if (kc > 64 || B > 31) return false;
+    const int sh = J.sh;      // 1: two-pass layout (x_0 untested, target row i-1 tests x_i)
+    const int P = B + 1 - sh;  // target rows per request
     const size_t need = 16 + (size_t)(B + 1) * ks * 8 + 2 * ((size_t)B * QS * 4 + 16) + (size_t)(4 * B + 2) * 4;
     if (need > (size_t)J.tail_bytes) return false;
     // the draft rows as one byte range per array (stride q_cap) when short
@@ -958,7 +986,7 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     int32_t* qcnt = pcnt + (B + 1);                                                  // [B]
     int32_t* dft = qcnt + B;                                                         // [B]
     int32_t* otok = dft + B;                                                         // [B+1] emitted tokens
-    const int64_t base = (int64_t)r * (B + 1);
+    const int64_t base = (int64_t)r * P;
     const uint32_t req = J.first_request + (uint32_t)r;
     // The request's compact target rows and draft rows arrive by bulk copies
     // (TMA) on one mbarrier: one round trip, whatever the memory system's
@@ -966,7 +994,7 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     if (lane == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
-        const uint32_t pb = (uint32_t)((B + 1) * ks * 4);
+        const uint32_t pb = (uint32_t)(P * ks * 4);
         const uint32_t qb = qflat ? range_bulk_bytes(qsi, qn) + range_bulk_bytes(qsp, qn) : 0u;
         mbar_expect_tx(bar, 2 * pb + qb);  // before any copy is issued
         bulk_g2s(pid, J.c_ids + (size_t)base * ks, pb, bar);
@@ -978,13 +1006,14 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     }
     int pc_l = 0, qc_l = 0, d_l = 0;
     uint32_t f_l = 0;
-    if (lane <= B) {
+    if (lane < P) {
         pc_l = __ldcg(J.c_count + base + lane);
         f_l = __ldcg(J.c_flags + base + lane);
     }
     if (lane < B) {
-        qc_l = J.q_count[(int64_t)r * B + lane];
-        d_l = J.draft_ids[(size_t)r * B + lane];
+        qc_l = __ldcg(J.q_count + (int64_t)r * B + lane);
+        d_l = __ldcg(J.draft_ids + (size_t)r * B + lane);
+        if (J.q_flags != nullptr) f_l |= __ldcg(J.q_flags + (int64_t)r * B + lane);
     }
     if (!qflat)
         warp_copy_rows<false>(J.q_ids + (size_t)r * B * J.q_cap, J.q_probs + (size_t)r * B * J.q_cap, J.q_cap, B, QS,
@@ -1005,10 +1034,8 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     qc_l = qc_l < 0 ? 0 : (qc_l > J.q_cap ? J.q_cap : qc_l);
     if (__any_sync(kFull, lane < B && qc_l > QS)) return false;
     uint32_t flags = __reduce_or_sync(kFull, f_l);
-    if (lane <= B) {
-        pcnt[lane] = pc_l;
-        otok[lane] = -1;
-    }
+    if (lane <= B) otok[lane] = -1;
+    if (lane < P) pcnt[lane] = pc_l;
     if (lane < B) {
         qcnt[lane] = qc_l;
         dft[lane] = d_l;
@@ -1023,16 +1050,22 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     bool stop_i = false, empty_i = false, notin_i = false;
     int32_t x_i = -1;
     if (lane < B) {
-        const int pc = pcnt[lane];
         x_i = dft[lane];
-        if (pc == 0) {
-            stop_i = empty_i = true;  // a non-finite target row
+        if (lane < sh) {
+            // the base-weights token is emitted untested (none when its row is empty)
+            stop_i = empty_i = qcnt[0] == 0;
         } else {
-            const bool xin = x_i >= 0 && (int64_t)x_i < J.vocab;
-            const double a = xin ? smem_lookup(qid + lane * qs, qpr + lane * qs, qcnt[lane], x_i) : 0.0;
-            const double px = xin ? smem_lookup(pid + lane * ks, ppr + lane * ks, pc, x_i) : 0.0;
-            notin_i = !(a > 0.0);
-            stop_i = notin_i || !(ua * a < px);
+            const int pr = lane - sh;  // the target row that tests position `lane`
+            const int pc = pcnt[pr];
+            if (pc == 0) {
+                stop_i = empty_i = true;  // a non-finite target row
+            } else {
+                const bool xin = x_i >= 0 && (int64_t)x_i < J.vocab;
+                const double a = xin ? smem_lookup(qid + lane * qs, qpr + lane * qs, qcnt[lane], x_i) : 0.0;
+                const double px = xin ? smem_lookup(pid + pr * ks, ppr + pr * ks, pc, x_i) : 0.0;
+                notin_i = !(a > 0.0);
+                stop_i = notin_i || !(ua * a < px);
+            }
         }
     }
     const unsigned stops = __ballot_sync(kFull, stop_i);
@@ -1045,10 +1078,11 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
         ntok = empty ? istop : istop + 1;
         if (!empty) {
             if (__shfl_sync(kFull, notin_i, istop)) flags |= kFlagDraftNotInSupport;
-            // residual max(0, p_i - q_i) over supp p_i, ascending ids
-            const int i = istop, pc = pcnt[i];
-            const int32_t* pi = pid + i * ks;
-            const float* pp = ppr + i * ks;
+            // residual max(0, p - q_i) over supp p, ascending ids (p: the
+            // target row that tests position i)
+            const int i = istop, pc = pcnt[i - sh];
+            const int32_t* pi = pid + (i - sh) * ks;
+            const float* pp = ppr + (i - sh) * ks;
             const int32_t* qi = qid + i * qs;
             const float* qp = qpr + i * qs;
             double ra = 0.0, rb = 0.0, pa = 0.0, pb = 0.0;
@@ -1071,21 +1105,21 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
             if (lane == 0) otok[i] = pick >= 0 ? pi[pick] : -1;
         }
     } else {
-        const int pc = pcnt[B];
+        const int pc = pcnt[B - sh];  // the bonus row
         if (pc == 0) {
             ntok = B;
         } else {
-            const float* pp = ppr + B * ks;
+            const float* pp = ppr + (B - sh) * ks;
             const double wa = lane < pc ? (double)pp[lane] : 0.0, wb = lane + 32 < pc ? (double)pp[lane + 32] : 0.0;
             const double u = __shfl_sync(kFull, ur, B);
             const int pick = warp_inv_cdf(wa, wb, u, lane);
-            if (lane == 0) otok[B] = pick >= 0 ? pid[B * ks + pick] : -1;
+            if (lane == 0) otok[B] = pick >= 0 ? pid[(B - sh) * ks + pick] : -1;
         }
     }
     __syncwarp();
     for (int t = lane; t <= B; t += 32) toks[t] = otok[t];
     if (lane == 0) {
-        J.out_accept_len[r] = acc;
+        J.out_accept_len[r] = acc > sh ? acc - sh : 0;  // accepted proposals (x_0 of the two-pass layout is not one)
         J.out_num_tokens[r] = ntok;
         J.out_req_flags[r] = flags;
     }
@@ -1184,7 +1218,7 @@ __device__ __noinline__ bool tree_tail_fast(const RowJob& J, int32_t r, unsigned
 template <int MODE>
 __device__ __forceinline__ void request_tail(const RowJob& J, int32_t req, double* wd, unsigned char* tail_smem,
                                              int lane) {
-    if (MODE == kModeLinear) {
+    if (MODE == kModeLinear || MODE == kModeCycle) {
         if (!linear_tail_fast(J, req, tail_smem, lane)) linear_tail(J, req, wd, lane);
     } else {
         if (!tree_tail_fast(J, req, tail_smem, lane)) tree_tail(J, req, wd, lane);
@@ -1304,7 +1338,7 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
     // bit 0 of rowbad: NaN / +inf (or no finite logit); bit 1: a wait gave up
     const uint32_t rflags = !bad ? 0u : (rowbad & 2u) ? (kFlagTimeout | ((rowbad & 1u) ? kFlagNonfinite : 0u))
                                                        : kFlagNonfinite;
-    if (MODE == kModeFilter) {
+    if (MODE == kModeFilter || (MODE == kModeCycle && row < J.nq2)) {
         int32_t* ids = J.out_ids + (size_t)row * J.cap;
         float* pr = J.out_probs + (size_t)row * J.cap;
         // lanes write their own two slots, then the rest of the row's slots
@@ -1340,6 +1374,7 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
             if (J.has_rng) J.out_sample[row] = tok;
         }
     } else {
+        if (MODE == kModeCycle) row -= J.nq2;  // the cycle's target rows
         int32_t* ids = J.c_ids + (size_t)row * J.ks;
         float* pr = J.c_probs + (size_t)row * J.ks;
         if (lane < kept) {
@@ -1748,13 +1783,19 @@ struct __align__(16) PipeShared {
     int cnt[kPipeSlots][kPipeConsumers];    // candidates per consumer warp of the slot's piece
     int wcnt[kPipeConsumers];               // candidate counts (compaction bookkeeping)
     uint32_t bad[kPipeSlots];               // NaN / +inf (bit 0) or gave-up (bit 1) of the slot's piece
-    unsigned long long spec;                // the latest prediction (a threshold key)
-    uint32_t spec_set;                      // a prediction exists
+    unsigned long long spec[2];             // the latest prediction (a threshold key), per row set
+    uint32_t spec_set[2];                   // a prediction exists
     int fin_done;                           // finishers done with the CTA's list
     int redo_n;                             // rows of the redo pass
     uint32_t redo_ready;                    // redo_n is final
     int abort;
 };
+
+// A cycle's draft rows (0) and target rows (1) differ in scale.
+template <int MODE>
+__device__ __forceinline__ int row_set(const RowJob& J, int64_t row) {
+    return (MODE == kModeCycle && row >= J.nq2) ? 1 : 0;
+}
 
 template <int MODE>
 __device__ __forceinline__ bool item_active(const RowJob& J, int64_t row) {
@@ -2431,11 +2472,13 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
         // the finisher is done with this slot's previous piece
         if ((used & sb) && !pipe_wait_warp(&P.slot_empty[slot], (par & sb) ? 0u : 1u, P)) fail = true;
         const Piece p = redo ? whole_row<T>(J, L.cr, row) : piece_of<T>(J, L.cr, row);
+        // a cycle's draft rows and target rows keep separate predictions
+        const int pset = row_set<MODE>(J, row);
         // the first consumer warp to start the piece fixes its mode: predicted
         // when a prediction exists by then (nobody waits for one)
         uint32_t mode = 0;
         if (lane == 0) {
-            const uint32_t want = (!redo && L.spec_ok && ld_acquire_shared(&P.spec_set) != 0u) ? 1u : 2u;
+            const uint32_t want = (!redo && L.spec_ok && ld_acquire_shared(&P.spec_set[pset]) != 0u) ? 1u : 2u;
             const uint32_t old = atomicCAS(&P.mode[slot], 0u, want);
             mode = old == 0u ? want : old;
         }
@@ -2479,7 +2522,7 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
         ws.tau = read_tau(s_tau);
         if (predicted) {
             // the latest prediction of this CTA
-            const uint64_t t = read_tau(&P.spec);
+            const uint64_t t = read_tau(&P.spec[pset]);
             if (t > ws.tau) ws.tau = t;
             if (lane == 0) {
                 atomicMax(&P.used[slot], (unsigned long long)t);
@@ -2527,10 +2570,10 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
                                 atomicMax(s_tau, (unsigned long long)t);
                                 // until a big piece completes, its seed is the CTA's
                                 // prediction (about 2.6 k elements of a row reach it)
-                                if (!redo && piece_big(L, p) && P.spec_set == 0u) {
-                                    P.spec = t;
+                                if (!redo && piece_big(L, p) && P.spec_set[pset] == 0u) {
+                                    P.spec[pset] = t;
                                     __threadfence_block();
-                                    st_release_shared(&P.spec_set, 1u);
+                                    st_release_shared(&P.spec_set[pset], 1u);
                                 }
                                 st_release_shared(&P.boot_ready[slot], 1u);
                             }
@@ -2902,9 +2945,10 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
             // (and of the next call); no basis leaves it as it is
             const uint64_t t = next_prediction(sel, n, J.k, held);
             if (t != 0ull) {
-                P.spec = t;
+                const int pset = row_set<MODE>(J, row);
+                P.spec[pset] = t;
                 __threadfence_block();
-                st_release_shared(&P.spec_set, 1u);
+                st_release_shared(&P.spec_set[pset], 1u);
             }
         }
         if (!held) {
@@ -2939,10 +2983,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_cons
             mbar_init(&P.slot_empty[s], 1);
             slot_reset(P, s);
         }
-        // the prediction this CTA left at the end of the previous call
-        const uint64_t h = J.hint != nullptr ? J.hint[blockIdx.x] : 0ull;
-        P.spec = h;
-        P.spec_set = h != 0ull ? 1u : 0u;
+        // the predictions this CTA left at the end of the previous call
+        for (int t = 0; t < 2; ++t) {
+            const uint64_t h = J.hint != nullptr ? J.hint[(size_t)t * kPipeMaxGrid + blockIdx.x] : 0ull;
+            P.spec[t] = h;
+            P.spec_set[t] = h != 0ull ? 1u : 0u;
+        }
         P.fin_done = 0;
         P.redo_n = 0;
         P.redo_ready = 0u;
@@ -2961,7 +3007,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_cons
     // carry this CTA's latest prediction to the next call (a hint only: the
     // rows it predicts are checked exactly)
     __syncthreads();
-    if (threadIdx.x == 0 && J.hint != nullptr && P.spec_set != 0u && P.abort == 0) J.hint[blockIdx.x] = P.spec;
+    if (threadIdx.x < 2 && J.hint != nullptr && P.spec_set[threadIdx.x] != 0u && P.abort == 0)
+        J.hint[(size_t)threadIdx.x * kPipeMaxGrid + blockIdx.x] = P.spec[threadIdx.x];
 }
 
 // ---------------------------------------------------------------------------
@@ -3221,6 +3268,32 @@ static WsLayout ws_layout(int64_t rows, int32_t k, bool compact) {
     return L;
 }
 
+// A cycle's workspace: the verifier layout over all its rows, then the draft
+// rows' compact arrays (ids and probs [nq][ks], count, flags, drafts [nq]).
+struct CycleLayout {
+    WsLayout w;
+    size_t q_ids, q_probs, q_count, q_flags, q_draft, total;
+};
+static CycleLayout cycle_layout(int32_t R, int32_t B, int32_t k, int32_t layout) {
+    CycleLayout C{};
+    const int64_t nq = (int64_t)R * B, np = (int64_t)R * (B + 1 - layout);
+    C.w = ws_layout(nq + np, k, true);
+    const size_t ks = (size_t)((k + 3) & ~3);
+    size_t off = C.w.total;
+    C.q_ids = off;
+    off = align_up(off + (size_t)nq * ks * 4, 256);
+    C.q_probs = off;
+    off = align_up(off + (size_t)nq * ks * 4, 256);
+    C.q_count = off;
+    off = align_up(off + (size_t)nq * 4, 256);
+    C.q_flags = off;
+    off = align_up(off + (size_t)nq * 4, 256);
+    C.q_draft = off;
+    off = align_up(off + (size_t)nq * 4, 256);
+    C.total = off;
+    return C;
+}
+
 static bool params_ok(const uno_sampling_params& sp) {
     if (!(sp.temperature >= 0.0f) || std::isinf(sp.temperature)) return false;
     if (sp.top_k < 1) return false;
@@ -3265,11 +3338,11 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
         if (g < grid) grid = g;
     }
     J.S = 1;
-    if (J.hint != nullptr) J.hint += (size_t)MODE * kPipeMaxGrid;  // each entry point keeps its own
+    if (J.hint != nullptr) J.hint += (size_t)MODE * 2 * kPipeMaxGrid;  // each entry point keeps its own
     // shared memory: ring | candidate slots | per finisher: sel, wd, tail
     const size_t slot_bytes = (size_t)kPipeSlots * kPipeConsumers * J.cap_w * 8;
     size_t tail = 0;
-    if (MODE == kModeLinear)
+    if (MODE == kModeLinear || MODE == kModeCycle)
         tail = 16 + (size_t)(J.B + 1) * J.ks * 8 + 2 * ((size_t)J.B * 64 * 4 + 16) + (size_t)(4 * J.B + 2) * 4;
     else if (MODE == kModeTree)
         tail = 16 + (size_t)J.V * J.ks * 8 + (size_t)J.V * 12 + (size_t)(J.B + 1) * 8;
@@ -3298,7 +3371,7 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     RowJob TJ = J;
     TJ.tail_bytes = tail <= 48 * 1024 ? (int32_t)tail : 0;
     TJ.fin_stride = (int32_t)align_up((size_t)kPipeMaxK * 8 + (size_t)TJ.tail_bytes, 128);
-    const int64_t nreq = J.rows / J.rpr;
+    const int64_t nreq = MODE == kModeCycle ? J.nq2 / J.B : J.rows / J.rpr;
     const size_t tsm = (size_t)kTailWarps * TJ.fin_stride;
     auto tkern = tail_kernel<MODE>;
     if (tsm > 48 * 1024 &&
@@ -3493,6 +3566,97 @@ uno_status uno_linear_verify(const void* target_logits, uno_dtype dt, int32_t R,
     bind_workspace(J, workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeLinear>(J, s) : launch_rows<float, kModeLinear>(J, s);
+}
+
+size_t uno_linear_cycle_workspace_bytes(int32_t R, int32_t B, int64_t vocab, int32_t top_k, int32_t layout) {
+    if (R <= 0 || B <= 0 || vocab <= 0 || top_k < 1 || (layout != UNO_LAYOUT_GENERIC && layout != UNO_LAYOUT_TWO_PASS))
+        return 0;
+    const int32_t k = (int32_t)(top_k < vocab ? top_k : vocab);
+    return cycle_layout(R, B, k, layout).total;
+}
+
+uno_status uno_linear_cycle(const void* draft_logits, const void* target_logits, uno_dtype dt, int32_t R, int32_t B,
+                            int64_t vocab, int32_t layout, uno_sampling_params sp, uno_rng rng, int32_t* out_tokens,
+                            int32_t* out_num_accepted, int32_t* out_num_tokens, uint32_t* out_flags,
+                            int32_t* out_draft_ids, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!draft_logits || !target_logits || !out_tokens || !out_num_accepted || !out_num_tokens || !out_flags)
+        return UNO_ERR_INVALID_ARG;
+    if (R <= 0 || B <= 0 || vocab <= 0 || vocab > INT32_MAX) return UNO_ERR_INVALID_ARG;
+    if (layout != UNO_LAYOUT_GENERIC && layout != UNO_LAYOUT_TWO_PASS) return UNO_ERR_INVALID_ARG;
+    if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
+    if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    const size_t esz = dt == UNO_F32 ? 4 : 2;
+    if (!aligned_to(draft_logits, esz) || !aligned_to(target_logits, esz)) return UNO_ERR_INVALID_ARG;
+    if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
+    if ((int64_t)R > kCounterWords - kRowCounterWords) return UNO_ERR_UNSUPPORTED;
+    const int32_t k = (int32_t)(sp.top_k < vocab ? sp.top_k : vocab);
+    const int64_t nq = (int64_t)R * B, np = (int64_t)R * (B + 1 - layout);
+    const CycleLayout C = cycle_layout(R, B, k, layout);
+    if (!workspace || workspace_bytes < C.total || !aligned_to(workspace, 16)) return UNO_ERR_WORKSPACE;
+    unsigned char* wb = static_cast<unsigned char*>(workspace);
+    int32_t* q_ids = reinterpret_cast<int32_t*>(wb + C.q_ids);
+    float* q_probs = reinterpret_cast<float*>(wb + C.q_probs);
+    int32_t* q_count = reinterpret_cast<int32_t*>(wb + C.q_count);
+    uint32_t* q_flags = reinterpret_cast<uint32_t*>(wb + C.q_flags);
+    int32_t* drafts = out_draft_ids != nullptr ? out_draft_ids : reinterpret_cast<int32_t*>(wb + C.q_draft);
+    const int32_t ks = (k + 3) & ~3;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    RowJob J{};
+    J.vocab = vocab;
+    J.row_stride = vocab;
+    J.temperature = sp.temperature;
+    J.top_p = sp.top_p;
+    J.k = k;
+    J.seed = rng.seed;
+    J.cycle = rng.cycle;
+    J.first_request = rng.first_request;
+    // the draft rows' outputs: compact rows, flags and one proposal each
+    J.out_ids = q_ids;
+    J.out_probs = q_probs;
+    J.out_count = q_count;
+    J.out_flags = q_flags;
+    J.cap = ks;
+    J.has_rng = 1;
+    J.out_sample = drafts;
+    // the verification
+    J.B = B;
+    J.sh = layout;
+    J.draft_ids = drafts;
+    J.q_ids = q_ids;
+    J.q_probs = q_probs;
+    J.q_count = q_count;
+    J.q_cap = ks;
+    J.q_flags = q_flags;
+    J.out_tokens = out_tokens;
+    J.out_accept_len = out_num_accepted;
+    J.out_num_tokens = out_num_tokens;
+    J.out_req_flags = out_flags;
+    bind_workspace(J, workspace, C.w);
+    if (k <= kPipeMaxK) {
+        // one launch over the cycle's draft and target rows, then the request tails
+        J.logits = static_cast<const unsigned char*>(draft_logits);
+        J.logits2 = static_cast<const unsigned char*>(target_logits);
+        J.nq2 = nq;
+        J.rows = nq + np;
+        J.rpr = B;
+        const uno_status st = dt == UNO_BF16 ? launch_pipe<__nv_bfloat16, kModeCycle>(J, s)
+                                             : launch_pipe<float, kModeCycle>(J, s);
+        if (st != UNO_ERR_UNSUPPORTED) return st;
+    }
+    // the draft rows, then the target rows with the request tails
+    RowJob Q = J;
+    Q.logits = static_cast<const unsigned char*>(draft_logits);
+    Q.rows = nq;
+    Q.rpr = B;
+    uno_status st = dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeFilter>(Q, s) : launch_rows<float, kModeFilter>(Q, s);
+    if (st != UNO_OK) return st;
+    RowJob V = J;
+    V.logits = static_cast<const unsigned char*>(target_logits);
+    V.rows = np;
+    V.rpr = B + 1 - layout;
+    V.has_rng = 0;
+    return dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeLinear>(V, s) : launch_rows<float, kModeLinear>(V, s);
 }
 
 uno_status uno_tree_topk_expand(const int32_t* q_ids, const float* q_probs, const int32_t* q_count, int32_t q_cap,

@@ -65,7 +65,7 @@ def compare_filter(gpu: dict, ref: dict, events: Events, rows=None, sample=False
 
 def compare_requests(gpu: dict, ref: dict, events: Events, keys, reqs=None):
     g = {k: np_of(v) for k, v in gpu.items()}
-    n = ref["accept_len"].shape[0]
+    n = ref["margin"].shape[0]
     idx = np.arange(n) if reqs is None else np.asarray(reqs)
     for i in range(n):
         gi = idx[i]
