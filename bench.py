@@ -174,7 +174,7 @@ def kernel_source_hash():
 
 
 def committed_traffic():
-    """DRAM bytes (read + write) per launch of the filter kernel from the
+    """DRAM bytes (read + write) per launch of the cycle's row kernel from the
     committed ncu summary, if it was taken on the current kernel source."""
     p = ROOT / "profiles" / "traffic.json"
     try:
@@ -183,7 +183,7 @@ def committed_traffic():
         return None
     if d.get("kernel_source_sha") != kernel_source_hash():
         return None
-    return d.get("filter_dram_bytes_per_launch")
+    return d.get("cycle_dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------------------
