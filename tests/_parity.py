@@ -26,14 +26,23 @@ def np_of(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy()
 
 
+# (name, decisions, boundary events) of every named check in this session;
+# conftest prints them after the run and, when UNO_PARITY_EVENTS names a
+# file, writes them there as JSON
+RECORDS: list = []
+
+
 class Events:
     """Counts decisions and excused boundary events."""
 
-    def __init__(self):
+    def __init__(self, name=None):
+        self.name = name
         self.decisions = 0
         self.boundary = 0
 
     def check(self, max_rate=1e-5):
+        if self.name is not None:
+            RECORDS.append(dict(check=self.name, decisions=self.decisions, boundary_events=self.boundary))
         if self.decisions:
             assert self.boundary <= max(0, int(max_rate * self.decisions)), (self.boundary, self.decisions)
 

@@ -1,3 +1,5 @@
+import json
+import os
 import sys
 from pathlib import Path
 
@@ -25,3 +27,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Decision and boundary-event counts of the named parity checks."""
+    mod = sys.modules.get("_parity")
+    recs = getattr(mod, "RECORDS", None)
+    if not recs:
+        return
+    terminalreporter.write_sep("-", "parity decisions and boundary events")
+    for r in recs:
+        terminalreporter.write_line(f"{r['check']}: {r['decisions']} decisions, {r['boundary_events']} boundary events")
+    out = os.environ.get("UNO_PARITY_EVENTS")
+    if out:
+        Path(out).write_text(json.dumps(recs, indent=1) + "\n")
