@@ -290,6 +290,24 @@ def replay_ms(g, stream, reps, flush=None):
     return statistics.fmean(a.elapsed_time(b) for a, b in ev)
 
 
+def eager_ms(fn, stream, reps, flush=None):
+    """Mean CUDA-event time of fn(stream) issued from Python on `stream`;
+    `flush` runs between calls, outside the events."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            fn(stream)
+        for a, b in ev:
+            if flush is not None:
+                flush()
+            a.record(stream)
+            fn(stream)
+            b.record(stream)
+    stream.synchronize()
+    return statistics.fmean(a.elapsed_time(b) for a, b in ev)
+
+
 def oracle_rate(fn, budget_s):
     """Requests per second of fn(i) (one request each) over about budget_s."""
     done, spent = 0, 0.0
@@ -329,13 +347,18 @@ def tree_leg(index, device, first, stream, peak, reps, cpu_budget):
     depth, nn = to["node_depth"].cpu().numpy(), to["num_nodes"].cpu().numpy()
     p_np = tree_target(w, depth, nn, reqs)
     p = dev(p_np)
-    rng = (w.seed, 0, first)
+    # the cycle word lives on the device: every replay of the graph draws the
+    # next cycle's uniforms (the graph ends by advancing it)
+    cyc = torch.zeros(1, dtype=torch.int32, device=device)
+    rng = (w.seed, cyc, first)
 
     def cycle(st):
         f = uno_filter_softmax(q, rows_per_request=w.B, **sp)
         t = uno_tree_topk_expand(f["ids"], f["probs"], f["count"], R=w.R, B=w.B, K=w.K, V=w.V)
-        return uno_tree_verify(p, t["node_token"], t["node_parent"], t["num_nodes"], R=w.R, B=w.B, V=w.V, rng=rng,
-                               **sp)
+        v = uno_tree_verify(p, t["node_token"], t["node_parent"], t["num_nodes"], R=w.R, B=w.B, V=w.V, rng=rng,
+                            **sp)
+        cyc.add_(1)
+        return v
 
     g = graph_of(cycle, stream)
     flush = None
@@ -343,6 +366,7 @@ def tree_leg(index, device, first, stream, peak, reps, cpu_budget):
         junk = torch.empty(256 << 20, dtype=torch.uint8, device=device)
         flush = lambda: junk.fill_(1)  # noqa: E731
     ms = replay_ms(g, stream, reps, flush)
+    calls = eager_ms(cycle, stream, reps, flush)
     nbytes = (w.R * w.B + int(nn.sum())) * w.vocab * w.elem_bytes
 
     import oracle
@@ -361,7 +385,10 @@ def tree_leg(index, device, first, stream, peak, reps, cpu_budget):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "bytes_per_cycle": nbytes},
             "l2": "256 MB buffer rewritten between replays" if flush else "inputs larger than L2",
-            "timing": f"CUDA events around {reps} replays of one graph (filter, expand, verify: 4 kernels)",
+            "timing": f"CUDA events around {reps} replays of one graph (filter, expand, verify: 4 kernels, "
+                      "then the cycle word advanced on the device)",
+            "calls": {"ms_per_cycle": calls, "value": w.R / (calls / 1e3),
+                      "note": "the same cycle as three Python calls per cycle (no graph), CUDA events around each"},
             "cpu_baseline": {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"{done} requests, {spent:.1f} s, single-threaded C oracle"}}
 

@@ -92,11 +92,21 @@ typedef struct {
 /* Counter-based RNG state of one decode cycle.  first_request is the global
  * index of the call's first request: the counter's request word is
  * first_request + local request index, so a batch split across calls or GPUs
- * draws the same uniforms as one call over the whole batch. */
+ * draws the same uniforms as one call over the whole batch.
+ *
+ * cycle_word is NULL or a 4-byte aligned device address of a uint32_t.  When
+ * it is set, the kernels read the cycle word there when they run and ignore
+ * `cycle`.  A CUDA graph captured around a call replays the call's arguments
+ * unchanged; with cycle_word set, writing the next cycle's number to that
+ * word (on the graph's stream, before the replay) makes each replay draw that
+ * cycle's uniforms.  The word must stay valid, and unchanged while a call
+ * that reads it runs, until the call (or graph replay) completes.  A
+ * misaligned address returns UNO_ERR_INVALID_ARG. */
 typedef struct {
     uint64_t seed;
     uint32_t cycle;
     uint32_t first_request;
+    const uint32_t* cycle_word;
 } uno_rng;
 
 #define UNO_MAX_TOP_K 1024
@@ -269,13 +279,18 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
  * Arguments, results and errors are those of uno_linear_verify, minus the
  * workspace.  Sizes whose uno_linear_verify_workspace_bytes exceeds
  * UNO_NOALLOC_SCRATCH_BYTES return UNO_ERR_UNSUPPORTED before anything is
- * enqueued: the 8 MiB hold R*(B+1) * k4 up to about 880,000, k4 being
+ * enqueued: the 8 MiB hold R*(B+1) * k4 up to about 800,000, k4 being
  * min(top_k, vocab) rounded up to a multiple of 4 (512 requests with B = 16
- * at top_k 50 fit; at top_k 200 they do not).  The first call on a device
- * looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture.  The call
- * itself allocates nothing: it enqueues cudaMemsetAsync of the counters it
- * uses, then its kernels.  Every call
+ * at top_k 50 fit; at top_k 200 they do not).  Each CUDA context that loads
+ * the library has its own copy of the array at its own address.  A call made
+ * while `stream` is not being captured looks that address up
+ * (cudaGetSymbolAddress) in the current context and remembers it for that
+ * context; a call made during stream capture uses the remembered address, so
+ * make one uncaptured call in a context before capturing one there (a
+ * captured call in a context never seen returns UNO_ERR_CUDA if the lookup
+ * is refused during capture).  The call itself allocates nothing: it
+ * enqueues cudaMemsetAsync of the counters it may use, then its kernels.
+ * Every call
  * shares the one array, so calls that overlap on the GPU (other streams,
  * other host threads) race; serialise them.
  * ---------------------------------------------------------------------- */

@@ -48,14 +48,21 @@ class _Params(ctypes.Structure):
 
 
 class _Rng(ctypes.Structure):
-    _fields_ = [("seed", ctypes.c_uint64), ("cycle", ctypes.c_uint32), ("first_request", ctypes.c_uint32)]
+    _fields_ = [("seed", ctypes.c_uint64), ("cycle", ctypes.c_uint32), ("first_request", ctypes.c_uint32),
+                ("cycle_word", ctypes.c_void_p)]
 
 
 def _rng(rng):
-    """(seed, cycle) or (seed, cycle, first_request) -> _Rng."""
-    seed, cycle = int(rng[0]), int(rng[1])
+    """(seed, cycle) or (seed, cycle, first_request) -> _Rng.  cycle is an
+    int, or a one-element int32 CUDA tensor whose value the kernels read when
+    they run (what a captured graph needs to draw a new cycle per replay)."""
+    seed, cycle = int(rng[0]), rng[1]
     first = int(rng[2]) if len(rng) > 2 else 0
-    return _Rng(seed, cycle, first)
+    if isinstance(cycle, torch.Tensor):
+        _need(cycle.is_cuda and cycle.dtype == torch.int32 and cycle.numel() == 1,
+              "a device cycle word must be a one-element int32 CUDA tensor")
+        return _Rng(seed, 0, first, ctypes.c_void_p(cycle.data_ptr()))
+    return _Rng(seed, int(cycle), first, None)
 
 
 _lib = None

@@ -17,6 +17,7 @@
 // the verification rules follow its "Motivation" and "Modifications"
 // sections (see include/uno_filter.h for the full statement).
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -60,6 +61,7 @@ struct RowJob {
     int32_t has_rng;
     uint64_t seed;
     uint32_t cycle;
+    const uint32_t* cycle_word;  // nullable: the cycle word, read from device memory at run time
     uint32_t first_request;  // global index of request 0 of this call
     // workspace
     uint32_t* row_ticket;
@@ -100,6 +102,13 @@ struct RowJob {
     const int32_t* num_nodes;
     int32_t* out_path_nodes;
 };
+
+// The cycle word of the counter-based RNG: the by-value one, or the one in
+// device memory when the call gave its address (a captured CUDA graph replays
+// the same arguments every cycle; the word it reads there changes).
+__device__ __forceinline__ uint32_t cycle_of(const RowJob& J) {
+    return J.cycle_word != nullptr ? __ldg(J.cycle_word) : J.cycle;
+}
 
 // ---------------------------------------------------------------------------
 // Element traits.  A lane examines 16-byte units (8 bf16 or 4 fp32), four
@@ -665,7 +674,7 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
         const double px = xin ? lookup_sorted(pid, ppr, pc, x) : 0.0;
         bool accept = false;
         if (a > 0.0) {
-            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)i, kDrawAccept, J.cycle);
+            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)i, kDrawAccept, cycle_of(J));
             accept = (u * a < px);
         } else {
             flags |= kFlagDraftNotInSupport;
@@ -688,7 +697,7 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
                 flags |= kFlagResidualEmpty;
                 for (int j = 0; j < pc; ++j) wd[j] = (double)__ldcg(ppr + j);
             }
-            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)i, kDrawResidual, J.cycle);
+            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)i, kDrawResidual, cycle_of(J));
             pick = inv_cdf_serial(wd, pc, u);
             toks[i] = pick >= 0 ? __ldcg(pid + pick) : -1;
         }
@@ -706,7 +715,7 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
             const int32_t* pid = J.c_ids + (size_t)(base + B - sh) * J.ks;
             const float* ppr = J.c_probs + (size_t)(base + B - sh) * J.ks;
             for (int j = 0; j < pc; ++j) wd[j] = (double)__ldcg(ppr + j);
-            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)B, kDrawTarget, J.cycle);
+            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)B, kDrawTarget, cycle_of(J));
             const int pick = inv_cdf_serial(wd, pc, u);
             toks[B] = pick >= 0 ? __ldcg(pid + pick) : -1;
         }
@@ -749,7 +758,7 @@ __device__ __noinline__ void tree_tail(const RowJob& J, int32_t r, double* wd, i
             const int32_t* pid = J.c_ids + (size_t)(base + j) * J.ks;
             const float* ppr = J.c_probs + (size_t)(base + j) * J.ks;
             for (int q = 0; q < pc; ++q) wd[q] = (double)__ldcg(ppr + q);
-            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)j, kDrawTarget, J.cycle);
+            const double u = uniform53(J.seed, J.first_request + (uint32_t)r, (uint32_t)j, kDrawTarget, cycle_of(J));
             const int pick = inv_cdf_serial(wd, pc, u);
             y = pick >= 0 ? __ldcg(pid + pick) : -1;
             toks[t] = y;
@@ -1021,10 +1030,10 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     // the decisions' uniforms, one position per lane
     double ua = 0.0, ur = 0.0;
     if (lane < B) {
-        ua = uniform53(J.seed, req, (uint32_t)lane, kDrawAccept, J.cycle);
-        ur = uniform53(J.seed, req, (uint32_t)lane, kDrawResidual, J.cycle);
+        ua = uniform53(J.seed, req, (uint32_t)lane, kDrawAccept, cycle_of(J));
+        ur = uniform53(J.seed, req, (uint32_t)lane, kDrawResidual, cycle_of(J));
     } else if (lane == B) {
-        ur = uniform53(J.seed, req, (uint32_t)B, kDrawTarget, J.cycle);
+        ur = uniform53(J.seed, req, (uint32_t)B, kDrawTarget, cycle_of(J));
     }
     const bool copied = tail_copies_wait(bar, lane);
     if (!copied) {
@@ -1182,7 +1191,7 @@ __device__ __noinline__ bool tree_tail_fast(const RowJob& J, int32_t r, unsigned
         }
         const float* pp = npr + j * ks;
         const double wa = lane < pc ? (double)pp[lane] : 0.0, wb = lane + 32 < pc ? (double)pp[lane + 32] : 0.0;
-        const double u = uniform53(J.seed, req, (uint32_t)j, kDrawTarget, J.cycle);
+        const double u = uniform53(J.seed, req, (uint32_t)j, kDrawTarget, cycle_of(J));
         const int pick = warp_inv_cdf(wa, wb, u, lane);
         const int32_t y = pick >= 0 ? nid[j * ks + pick] : -1;
         if (lane == 0) {
@@ -1362,7 +1371,7 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
         int32_t tok = -1;
         if (J.has_rng && kept > 0) {
             const double u = uniform53(J.seed, J.first_request + (uint32_t)(row / J.rpr), (uint32_t)(row % J.rpr),
-                                       kDrawProposal, J.cycle);
+                                       kDrawProposal, cycle_of(J));
             const double wa = lane < kept ? (double)__uint_as_float((uint32_t)oa) : 0.0;
             const double wb = lane + 32 < kept ? (double)__uint_as_float((uint32_t)ob) : 0.0;
             const int pick = warp_inv_cdf(wa, wb, u, lane);
@@ -1504,7 +1513,7 @@ __device__ void finish_row(const RowJob& J, int64_t row, int32_t req, int n, uin
                 if (kept > 0) {
                     for (int j = 0; j < kept; ++j) wd[j] = (double)__uint_as_float((uint32_t)outk[j]);
                     const double u = uniform53(J.seed, J.first_request + (uint32_t)(row / J.rpr),
-                                               (uint32_t)(row % J.rpr), kDrawProposal, J.cycle);
+                                               (uint32_t)(row % J.rpr), kDrawProposal, cycle_of(J));
                     const int pick = inv_cdf_serial(wd, kept, u);
                     tok = pick >= 0 ? (int32_t)(outk[pick] >> 32) : -1;
                 }
@@ -3478,6 +3487,8 @@ size_t uno_tree_verify_workspace_bytes(int32_t R, int32_t V, int64_t vocab, int3
 }
 
 static bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+// a device cycle word, when given, is a 4-byte aligned uint32_t
+static bool rng_ok(const uno_rng& r) { return r.cycle_word == nullptr || aligned_to(r.cycle_word, 4); }
 
 uno_status uno_filter_softmax(const void* logits, uno_dtype dt, int64_t rows, int64_t vocab, int64_t row_stride,
                               int32_t rows_per_request, uno_sampling_params sp, int32_t cap, int32_t* out_ids,
@@ -3489,6 +3500,7 @@ uno_status uno_filter_softmax(const void* logits, uno_dtype dt, int64_t rows, in
         return UNO_ERR_INVALID_ARG;
     if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
     if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    if (rng && !rng_ok(*rng)) return UNO_ERR_INVALID_ARG;
     if (rng && !out_sample) return UNO_ERR_INVALID_ARG;
     if (!aligned_to(logits, dt == UNO_F32 ? 4 : 2)) return UNO_ERR_INVALID_ARG;
     if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
@@ -3516,6 +3528,7 @@ uno_status uno_filter_softmax(const void* logits, uno_dtype dt, int64_t rows, in
     J.has_rng = rng ? 1 : 0;
     J.seed = rng ? rng->seed : 0;
     J.cycle = rng ? rng->cycle : 0;
+    J.cycle_word = rng ? rng->cycle_word : nullptr;
     J.first_request = rng ? rng->first_request : 0;
     bind_workspace(J, workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -3533,6 +3546,7 @@ uno_status uno_linear_verify(const void* target_logits, uno_dtype dt, int32_t R,
     if (R <= 0 || B <= 0 || vocab <= 0 || vocab > INT32_MAX || q_cap < 1) return UNO_ERR_INVALID_ARG;
     if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
     if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    if (!rng_ok(rng)) return UNO_ERR_INVALID_ARG;
     if (!aligned_to(target_logits, dt == UNO_F32 ? 4 : 2)) return UNO_ERR_INVALID_ARG;
     if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
     const int32_t k = (int32_t)(sp.top_k < vocab ? sp.top_k : vocab);
@@ -3552,6 +3566,7 @@ uno_status uno_linear_verify(const void* target_logits, uno_dtype dt, int32_t R,
     J.k = k;
     J.seed = rng.seed;
     J.cycle = rng.cycle;
+    J.cycle_word = rng.cycle_word;
     J.first_request = rng.first_request;
     J.B = B;
     J.draft_ids = draft_ids;
@@ -3585,6 +3600,7 @@ uno_status uno_linear_cycle(const void* draft_logits, const void* target_logits,
     if (layout != UNO_LAYOUT_GENERIC && layout != UNO_LAYOUT_TWO_PASS) return UNO_ERR_INVALID_ARG;
     if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
     if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    if (!rng_ok(rng)) return UNO_ERR_INVALID_ARG;
     const size_t esz = dt == UNO_F32 ? 4 : 2;
     if (!aligned_to(draft_logits, esz) || !aligned_to(target_logits, esz)) return UNO_ERR_INVALID_ARG;
     if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
@@ -3610,6 +3626,7 @@ uno_status uno_linear_cycle(const void* draft_logits, const void* target_logits,
     J.k = k;
     J.seed = rng.seed;
     J.cycle = rng.cycle;
+    J.cycle_word = rng.cycle_word;
     J.first_request = rng.first_request;
     // the draft rows' outputs: compact rows, flags and one proposal each
     J.out_ids = q_ids;
@@ -3707,6 +3724,7 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
     if (V < B || V > UNO_MAX_TREE_NODES) return UNO_ERR_INVALID_ARG;
     if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
     if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    if (!rng_ok(rng)) return UNO_ERR_INVALID_ARG;
     if (!aligned_to(target_logits, dt == UNO_F32 ? 4 : 2)) return UNO_ERR_INVALID_ARG;
     if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
     const int32_t k = (int32_t)(sp.top_k < vocab ? sp.top_k : vocab);
@@ -3726,6 +3744,7 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
     J.k = k;
     J.seed = rng.seed;
     J.cycle = rng.cycle;
+    J.cycle_word = rng.cycle_word;
     J.first_request = rng.first_request;
     J.B = B;
     J.V = V;
@@ -3753,21 +3772,57 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_noalloc_scratch[UNO_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch on the current device.  In host code
-// the array's name is only a stand-in, so the address is looked up once per
-// device, with that device current, on the first call there.
-static uno_status noalloc_scratch(unsigned char** out) {
+// Device address of g_noalloc_scratch in the current context.  In host code
+// the array's name is only a stand-in: each context that loads the library's
+// module (a device's primary context, a driver-API context of a plugin host,
+// the primary context again after cudaDeviceReset) holds its own copy at its
+// own address.  Outside stream capture the address is looked up on every call
+// (cudaGetSymbolAddress, cheap once the module is loaded), so a stale address
+// is never used; the result is remembered per CUcontext for calls made while
+// `s` is being captured, where a context cannot be reset.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+static CUcontext current_context() {
+    static CtxGetCurrentFn fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<CtxGetCurrentFn>(f);
+    }();
+    CUcontext c = nullptr;
+    if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+static uno_status noalloc_scratch(cudaStream_t s, unsigned char** out) {
     static std::mutex mu;
-    static unsigned char* addr[64] = {nullptr};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return UNO_ERR_CUDA;
+    constexpr int kSlots = 64;
+    static CUcontext ctx[kSlots] = {nullptr};
+    static unsigned char* addr[kSlots] = {nullptr};
+    static int next = 0;
+    const CUcontext c = current_context();
+    if (c == nullptr) return UNO_ERR_CUDA;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return UNO_ERR_CUDA;
     std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return UNO_ERR_CUDA;
-        addr[dev] = static_cast<unsigned char*>(p);
+    int at = -1;
+    for (int i = 0; i < kSlots; ++i)
+        if (ctx[i] == c) at = i;
+    if (cs != cudaStreamCaptureStatusNone && at >= 0) {
+        *out = addr[at];
+        return UNO_OK;
     }
-    *out = addr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return UNO_ERR_CUDA;
+    if (at < 0) {
+        at = next;
+        next = (next + 1) % kSlots;
+        ctx[at] = c;
+    }
+    addr[at] = static_cast<unsigned char*>(p);
+    *out = addr[at];
     return UNO_OK;
 }
 
@@ -3782,6 +3837,7 @@ uno_status uno_linear_verify_noalloc(const void* target_logits, uno_dtype dt, in
     if (R <= 0 || B <= 0 || vocab <= 0 || vocab > INT32_MAX || q_cap < 1) return UNO_ERR_INVALID_ARG;
     if (dt != UNO_F32 && dt != UNO_BF16) return UNO_ERR_INVALID_ARG;
     if (!params_ok(sp)) return UNO_ERR_INVALID_ARG;
+    if (!rng_ok(rng)) return UNO_ERR_INVALID_ARG;
     if (!aligned_to(target_logits, dt == UNO_F32 ? 4 : 2)) return UNO_ERR_INVALID_ARG;
     if (sp.top_k > UNO_MAX_TOP_K) return UNO_ERR_UNSUPPORTED;
     if ((int64_t)R > kCounterWords - kRowCounterWords) return UNO_ERR_UNSUPPORTED;
@@ -3789,15 +3845,18 @@ uno_status uno_linear_verify_noalloc(const void* target_logits, uno_dtype dt, in
     const int64_t rows = (int64_t)R * (B + 1);
     const WsLayout L = ws_layout(rows, k, true);
     if (L.total > (size_t)UNO_NOALLOC_SCRATCH_BYTES) return UNO_ERR_UNSUPPORTED;  // beyond the fixed scratch
-    unsigned char* scratch = nullptr;
-    const uno_status st = noalloc_scratch(&scratch);
-    if (st != UNO_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned char* scratch = nullptr;
+    const uno_status st = noalloc_scratch(s, &scratch);
+    if (st != UNO_OK) return st;
     // the array keeps the last call's contents: clear the counters this call
-    // uses (row counters only matter for split rows, which need rows < 4096)
+    // may use: request tickets, and the tickets of split rows, which the
+    // general kernel keys by row (rows <= kRowCounterWords only) and the
+    // pipelined kernel by the row's first CTA (below kPipeMaxGrid)
     if (cudaMemsetAsync(scratch + L.req_ticket, 0, (size_t)R * 4, s) != cudaSuccess) return UNO_ERR_CUDA;
-    if (rows < 4096 && cudaMemsetAsync(scratch + L.row_ticket, 0, (size_t)rows * 4, s) != cudaSuccess)
-        return UNO_ERR_CUDA;
+    int64_t nrow_words = rows > kPipeMaxGrid ? rows : kPipeMaxGrid;
+    if (nrow_words > kRowCounterWords) nrow_words = kRowCounterWords;
+    if (cudaMemsetAsync(scratch + L.row_ticket, 0, (size_t)nrow_words * 4, s) != cudaSuccess) return UNO_ERR_CUDA;
 
     RowJob J{};
     J.logits = static_cast<const unsigned char*>(target_logits);
@@ -3810,6 +3869,7 @@ uno_status uno_linear_verify_noalloc(const void* target_logits, uno_dtype dt, in
     J.k = k;
     J.seed = rng.seed;
     J.cycle = rng.cycle;
+    J.cycle_word = rng.cycle_word;
     J.first_request = rng.first_request;
     J.B = B;
     J.draft_ids = draft_ids;

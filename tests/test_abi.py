@@ -105,3 +105,19 @@ def test_suffix_attention_rejects_bad_arguments_on_the_host(bad, status):
     st = lib.uno_tree_suffix_attention_merge(q, fake, fake, a["dt"], a["R"], a["V"], a["H"], a["Hkv"], a["d"],
                                              a["scale"], fake, fake, fake, fake, fake, fake, None, None)
     assert st == status
+
+
+def test_misaligned_cycle_word_rejected_on_the_host():
+    """A device cycle word must be 4-byte aligned; a misaligned address is an
+    argument error returned before any device work."""
+    from speculative_decoding_verification_filter_b200 import _binding as b
+    lib = b.load_library()
+    fake = ctypes.c_void_p(0x1000)
+    rng = b._Rng(1, 0, 0, ctypes.c_void_p(0x1002))
+    sp = b._Params(1.0, 5, 0.9)
+    st = lib.uno_filter_softmax(fake, 0, 4, 10, 10, 1, sp, 8, fake, fake, fake, None, ctypes.byref(rng), fake, fake,
+                                fake, 1 << 20, None)
+    assert st == 1
+    st = lib.uno_tree_verify(fake, 1, 1, 4, 8, 1000, b._Params(1.0, 50, 0.95), fake, fake, fake, rng, fake, fake,
+                             fake, fake, fake, fake, 1 << 24, None)
+    assert st == 1
