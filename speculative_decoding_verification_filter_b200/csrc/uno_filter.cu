@@ -3046,7 +3046,8 @@ __global__ void __launch_bounds__(32 * kTailWarps) tail_kernel(const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
-// Tree expansion: one warp per request.
+// Tree expansion: one CTA per request.  Its warps extract the top-K of the B
+// marginals side by side; warp 0 then expands the tree.
 // ---------------------------------------------------------------------------
 struct TreeJob {
     const int32_t* q_ids;
@@ -3060,28 +3061,35 @@ struct TreeJob {
     int32_t* num_nodes;
 };
 
-__global__ void __launch_bounds__(32) tree_expand_kernel(const __grid_constant__ TreeJob J) {
+constexpr int kTreeMaxWarps = 8;
+constexpr int kTreeRankMax = 256;  // rows up to this many entries are ranked, longer ones sorted
+
+__global__ void __launch_bounds__(32 * kTreeMaxWarps) tree_expand_kernel(const __grid_constant__ TreeJob J) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int B = J.B, K = J.K, V = J.V;
-    uint64_t* sortbuf = reinterpret_cast<uint64_t*>(smem);            // [sort_cap]
-    double* nscore = reinterpret_cast<double*>(sortbuf + J.sort_cap);  // [V]
+    const int nwarps = blockDim.x >> 5;
+    double* nscore = reinterpret_cast<double*>(smem);                  // [V]
     double* fscore = nscore + V;                                       // [V + 1]
-    int32_t* cand_id = reinterpret_cast<int32_t*>(fscore + V + 1);     // [B*K]
+    uint64_t* sortbufs = reinterpret_cast<uint64_t*>(fscore + V + 1);  // [nwarps][sort_cap]
+    int32_t* cand_id = reinterpret_cast<int32_t*>(sortbufs + (size_t)nwarps * J.sort_cap);  // [B*K]
     float* cand_p = reinterpret_cast<float*>(cand_id + B * K);         // [B*K]
     int32_t* ncand = reinterpret_cast<int32_t*>(cand_p + B * K);       // [B]
     int32_t* fdep = ncand + B;                                         // [V + 1]
     int32_t* fpar = fdep + V + 1;                                      // [V + 1]
     int32_t* frank = fpar + V + 1;                                     // [V + 1]
 
-    const int lane = threadIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.x;
 
-    // 1. top-K of each marginal by (prob desc, id asc)
-    for (int d = 0; d < B; ++d) {
+    // 1. top-K of each marginal by (prob desc, id asc), one row per warp at a
+    // time.  Keys are distinct (ids are), so an entry's place is the number
+    // of larger keys in its row.
+    uint64_t* sortbuf = sortbufs + (size_t)warp * J.sort_cap;
+    for (int d = warp; d < B; d += nwarps) {
         const int64_t row = (int64_t)r * B + d;
         int c = J.q_count[row];
         c = c < 0 ? 0 : (c > J.q_cap ? J.q_cap : c);
-        const int np2 = next_pow2(c < 1 ? 1 : c);
+        const int np2 = c <= kTreeRankMax ? c : next_pow2(c);
         for (int i = lane; i < np2; i += 32) {
             uint64_t key = 0ull;
             if (i < c) {
@@ -3092,15 +3100,29 @@ __global__ void __launch_bounds__(32) tree_expand_kernel(const __grid_constant__
             sortbuf[i] = key;
         }
         __syncwarp();
-        warp_bitonic_sort(sortbuf, np2, true, lane);
         const int nk = c < K ? c : K;
-        for (int i = lane; i < nk; i += 32) {
-            cand_id[d * K + i] = key_id(sortbuf[i]);
-            cand_p[d * K + i] = float_of_ord((uint32_t)(sortbuf[i] >> 32));
+        if (c <= kTreeRankMax) {
+            for (int i = lane; i < c; i += 32) {
+                const uint64_t key = sortbuf[i];
+                int rank = 0;
+                for (int j = 0; j < c; ++j) rank += sortbuf[j] > key ? 1 : 0;
+                if (rank < nk) {
+                    cand_id[d * K + rank] = key_id(key);
+                    cand_p[d * K + rank] = float_of_ord((uint32_t)(key >> 32));
+                }
+            }
+        } else {
+            warp_bitonic_sort(sortbuf, np2, true, lane);
+            for (int i = lane; i < nk; i += 32) {
+                cand_id[d * K + i] = key_id(sortbuf[i]);
+                cand_p[d * K + i] = float_of_ord((uint32_t)(sortbuf[i] >> 32));
+            }
         }
         if (lane == 0) ncand[d] = nk;
         __syncwarp();
     }
+    __syncthreads();
+    if (warp != 0) return;
 
     int32_t* tok = J.node_token + (size_t)r * V;
     int32_t* par = J.node_parent + (size_t)r * V;
@@ -3694,21 +3716,25 @@ uno_status uno_tree_topk_expand(const int32_t* q_ids, const float* q_probs, cons
     J.B = B;
     J.K = K;
     J.V = V;
-    J.sort_cap = next_pow2(q_cap);
+    J.sort_cap = q_cap <= kTreeRankMax ? q_cap : next_pow2(q_cap);
     J.node_token = node_token;
     J.node_parent = node_parent;
     J.node_depth = node_depth;
     J.node_score = node_score;
     J.num_nodes = num_nodes;
-    const size_t smem = (size_t)J.sort_cap * 8 + (size_t)(2 * V + 1) * 8 + (size_t)B * K * 8 + (size_t)B * 4 +
-                        (size_t)3 * (V + 1) * 4;
+    const size_t fixed = (size_t)(2 * V + 1) * 8 + (size_t)B * K * 8 + (size_t)B * 4 + (size_t)3 * (V + 1) * 4;
+    const size_t per_warp = align_up((size_t)J.sort_cap * 8, 8);
+    // warps: one per marginal up to kTreeMaxWarps, as many as fit 200 KB
+    int nw = B < kTreeMaxWarps ? B : kTreeMaxWarps;
+    while (nw > 1 && fixed + (size_t)nw * per_warp > 200 * 1024) --nw;
+    const size_t smem = fixed + (size_t)nw * per_warp;
     if (smem > 227 * 1024) return UNO_ERR_UNSUPPORTED;
     if (smem > 48 * 1024) {
         if (cudaFuncSetAttribute(tree_expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)
             return UNO_ERR_CUDA;
     }
-    tree_expand_kernel<<<(unsigned)R, 32, smem, static_cast<cudaStream_t>(stream)>>>(J);
+    tree_expand_kernel<<<(unsigned)R, 32 * nw, smem, static_cast<cudaStream_t>(stream)>>>(J);
     return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
 }
 
