@@ -122,6 +122,9 @@ typedef struct {
 #define UNO_FLAG_TIMEOUT 8u              /* a bounded wait for the row's own     */
                                          /* asynchronous copies gave up; the row */
                                          /* result is not valid                  */
+#define UNO_FLAG_BAD_PARAMS 32u          /* *_params entry points: the request's */
+                                         /* parameter entries are out of range;  */
+                                         /* the row has no support               */
 
 /* ------------------------------------------------------------------------
  * uno_filter_softmax -- filter each row and optionally draw from it.
@@ -265,6 +268,74 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
                            const int32_t* num_nodes, uno_rng rng, int32_t* out_tokens, int32_t* out_accept_len,
                            int32_t* out_num_tokens, int32_t* out_path_nodes, uint32_t* out_flags, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Per-request sampling parameters and the filter order.
+ * [eval guide, run_math_eval 全参数详解]: temperature, top_p and top_k are
+ * set per run (temperature >= 0, 0 greedy; top_p in (0, 1]; top_k > 0); a
+ * serving batch mixes requests that carry different ones.  [UNO PR, review
+ * thread on the filter order]: UNO takes top-k first, renormalises over the
+ * kept tokens and applies top-p to that distribution (UNO_ORDER_TOPK_FIRST,
+ * what the entry points above do); the regular sampler uses the "joint"
+ * order, where the top-p cut is taken on the full-vocabulary softmax
+ * (UNO_ORDER_JOINT): the cumulative mass of the top-k tokens, in descending
+ * order, is divided by the sum of exp((l - l_max) / T) over every finite
+ * logit of the row instead of over the top k.  Top-k still bounds the kept
+ * set, and the kept probabilities are still renormalised among themselves.
+ *
+ * temperature, top_k, top_p  device arrays of one entry per request
+ *             (4-byte aligned); a row reads the entries of its request
+ *             (filter: row / rows_per_request; verifiers: the request whose
+ *             target row it is).  Each call reads them when it runs, so they
+ *             may change between replays of a captured graph.
+ * top_k_max   host value, 1 .. UNO_MAX_TOP_K: an upper bound of the top_k
+ *             entries after clamping to the vocabulary.  It sizes the
+ *             selection and the workspace (pass it as top_k to the
+ *             *_workspace_bytes functions) and `cap` must hold
+ *             min(top_k_max, vocab).
+ * order       UNO_ORDER_TOPK_FIRST or UNO_ORDER_JOINT.  The joint order adds
+ *             one read of each row (its normaliser) before the row kernels.
+ * A request whose entries are out of range (temperature negative, NaN or
+ * infinite; top_k < 1 or, clamped to the vocabulary, above top_k_max; top_p
+ * outside (0, 1]) is not an error of the call: its rows get
+ * UNO_FLAG_BAD_PARAMS and no support, and a verifier treats them like
+ * non-finite target rows.  Host-side errors (UNO_ERR_INVALID_ARG): rp NULL,
+ * a NULL or misaligned array, top_k_max < 1, an unknown order.
+ *
+ * The four entry points take the same arguments as the ones above, with rp
+ * in place of the sampling parameters.
+ * ---------------------------------------------------------------------- */
+#define UNO_ORDER_TOPK_FIRST 0
+#define UNO_ORDER_JOINT 1
+typedef struct {
+    const float* temperature;
+    const int32_t* top_k;
+    const float* top_p;
+    int32_t top_k_max;
+    int32_t order;
+} uno_request_params;
+
+uno_status uno_filter_softmax_params(const void* logits, uno_dtype dt, int64_t rows, int64_t vocab,
+                                     int64_t row_stride, int32_t rows_per_request, const uno_request_params* rp,
+                                     int32_t cap, int32_t* out_ids, float* out_probs, int32_t* out_count,
+                                     float* out_dense, const uno_rng* rng, int32_t* out_sample, uint32_t* out_flags,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+uno_status uno_linear_verify_params(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int64_t vocab,
+                                    const uno_request_params* rp, const int32_t* draft_ids, const int32_t* q_ids,
+                                    const float* q_probs, const int32_t* q_count, int32_t q_cap, uno_rng rng,
+                                    int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                                    uint32_t* out_flags, void* workspace, size_t workspace_bytes, void* stream);
+uno_status uno_linear_cycle_params(const void* draft_logits, const void* target_logits, uno_dtype dt, int32_t R,
+                                   int32_t B, int64_t vocab, int32_t layout, const uno_request_params* rp,
+                                   uno_rng rng, int32_t* out_tokens, int32_t* out_num_accepted,
+                                   int32_t* out_num_tokens, uint32_t* out_flags, int32_t* out_draft_ids,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+uno_status uno_tree_verify_params(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int32_t V,
+                                  int64_t vocab, const uno_request_params* rp, const int32_t* node_token,
+                                  const int32_t* node_parent, const int32_t* num_nodes, uno_rng rng,
+                                  int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                                  int32_t* out_path_nodes, uint32_t* out_flags, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * uno_linear_verify_noalloc -- uno_linear_verify without a caller workspace.

@@ -8,6 +8,7 @@ from ._binding import (  # noqa: F401
     EXPORTED,
     LAYOUT_GENERIC,
     LAYOUT_TWO_PASS,
+    FLAG_BAD_PARAMS,
     FLAG_BAD_TREE,
     FLAG_DRAFT_NOT_IN_SUPPORT,
     FLAG_NONFINITE_ROW,
@@ -16,10 +17,14 @@ from ._binding import (  # noqa: F401
     UnoError,
     load_library,
     uno_filter_softmax,
+    uno_filter_softmax_params,
     uno_linear_cycle,
+    uno_linear_cycle_params,
     uno_linear_verify,
+    uno_linear_verify_params,
     uno_linear_verify_noalloc,
     uno_tree_suffix_attention_merge,
     uno_tree_topk_expand,
     uno_tree_verify,
+    uno_tree_verify_params,
 )

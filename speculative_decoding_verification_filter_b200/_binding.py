@@ -14,6 +14,7 @@ import ctypes
 import threading
 from pathlib import Path
 
+import numpy as np
 import torch
 
 _PKG = Path(__file__).resolve().parent
@@ -22,6 +23,7 @@ LIB_PATH = _PKG / "libuno_filter.so"
 UNO_F32, UNO_BF16 = 0, 1
 FLAG_NONFINITE_ROW, FLAG_DRAFT_NOT_IN_SUPPORT, FLAG_RESIDUAL_EMPTY = 1, 2, 4
 FLAG_BAD_TREE = 16
+FLAG_BAD_PARAMS = 32
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported argument", 3: "CUDA launch error",
           4: "workspace missing or too small"}
 
@@ -31,6 +33,7 @@ EXPORTED = (
     "uno_linear_cycle_workspace_bytes", "uno_linear_cycle",
     "uno_tree_topk_expand",
     "uno_tree_verify_workspace_bytes", "uno_tree_verify",
+    "uno_filter_softmax_params", "uno_linear_verify_params", "uno_linear_cycle_params", "uno_tree_verify_params",
     "uno_linear_verify_noalloc",
     "uno_tree_suffix_attention_merge",
     "uno_status_string",
@@ -50,6 +53,48 @@ class _Params(ctypes.Structure):
 class _Rng(ctypes.Structure):
     _fields_ = [("seed", ctypes.c_uint64), ("cycle", ctypes.c_uint32), ("first_request", ctypes.c_uint32),
                 ("cycle_word", ctypes.c_void_p)]
+
+
+class _ReqParams(ctypes.Structure):
+    _fields_ = [("temperature", ctypes.c_void_p), ("top_k", ctypes.c_void_p), ("top_p", ctypes.c_void_p),
+                ("top_k_max", ctypes.c_int32), ("order", ctypes.c_int32)]
+
+
+ORDERS = {"topk_first": 0, "joint": 1}
+
+
+class _PerRequest:
+    """Per-request parameter arrays on the device (kept alive for the call)
+    and the struct that points at them."""
+
+    def __init__(self, temperature, top_k, top_p, order, nreq, device, top_k_max):
+        _need(order in ORDERS, f"order must be one of {sorted(ORDERS)}")
+
+        def arr(x, dt):
+            t = torch.as_tensor(x, dtype=dt)
+            t = t.reshape(-1) if t.dim() else t.reshape(1).expand(nreq)
+            _need(t.numel() == nreq, f"per-request parameters need {nreq} entries")
+            return t.to(device, non_blocking=True).contiguous()
+
+        self.T = arr(temperature, torch.float32)
+        self.k = arr(top_k, torch.int32)
+        self.p = arr(top_p, torch.float32)
+        if top_k_max is None:
+            # the bound from the values themselves (a device array is read back)
+            top_k_max = int(torch.as_tensor(top_k).max().item())
+        self.top_k_max = max(1, int(top_k_max))
+        self.c = _ReqParams(ctypes.c_void_p(self.T.data_ptr()), ctypes.c_void_p(self.k.data_ptr()),
+                            ctypes.c_void_p(self.p.data_ptr()), self.top_k_max, ORDERS[order])
+
+
+def _per_request(temperature, top_k, top_p, order, nreq, device, top_k_max, force=False):
+    """None for scalar parameters in the top-k-first order (the plain entry
+    points) unless `force`, else a _PerRequest for the *_params entry points."""
+    scalar = not force and all(isinstance(x, (int, float, np.generic)) or (isinstance(x, (torch.Tensor, np.ndarray)) and x.ndim == 0)
+                 for x in (temperature, top_k, top_p))
+    if scalar and order == "topk_first":
+        return None
+    return _PerRequest(temperature, top_k, top_p, order, nreq, device, top_k_max)
 
 
 def _rng(rng):
@@ -102,6 +147,19 @@ def load_library():
         lib.uno_tree_verify.argtypes = [P, ctypes.c_int, i32, i32, i32, i64, _Params, P, P, P, _Rng,
                                         P, P, P, P, P, P, sz, P]
         lib.uno_tree_verify.restype = ctypes.c_int
+        RP = ctypes.POINTER(_ReqParams)
+        lib.uno_filter_softmax_params.argtypes = [P, ctypes.c_int, i64, i64, i64, i32, RP, i32, P, P, P, P,
+                                                  ctypes.POINTER(_Rng), P, P, P, sz, P]
+        lib.uno_filter_softmax_params.restype = ctypes.c_int
+        lib.uno_linear_verify_params.argtypes = [P, ctypes.c_int, i32, i32, i64, RP, P, P, P, P, i32, _Rng,
+                                                 P, P, P, P, P, sz, P]
+        lib.uno_linear_verify_params.restype = ctypes.c_int
+        lib.uno_linear_cycle_params.argtypes = [P, P, ctypes.c_int, i32, i32, i64, i32, RP, _Rng, P, P, P, P, P, P,
+                                                sz, P]
+        lib.uno_linear_cycle_params.restype = ctypes.c_int
+        lib.uno_tree_verify_params.argtypes = [P, ctypes.c_int, i32, i32, i32, i64, RP, P, P, P, _Rng,
+                                               P, P, P, P, P, P, sz, P]
+        lib.uno_tree_verify_params.restype = ctypes.c_int
         lib.uno_linear_verify_noalloc.argtypes = [P, ctypes.c_int, i32, i32, i64, _Params, P, P, P, P, i32, _Rng,
                                                   P, P, P, P, P]
         lib.uno_linear_verify_noalloc.restype = ctypes.c_int
@@ -195,7 +253,7 @@ def _host_back(out: dict, host: bool) -> dict:
 # entry points
 # ---------------------------------------------------------------------------
 def uno_filter_softmax(logits, *, temperature, top_k, top_p, rows_per_request=1, cap=None, rng=None,
-                       dense=False):
+                       dense=False, order="topk_first", top_k_max=None, per_request=False):
     """Filter each row of logits [rows, vocab] (top-k, then top-p, softmax).
 
     Returns dict(ids [rows, cap] int32, probs [rows, cap] float32, count [rows],
@@ -207,8 +265,12 @@ def uno_filter_softmax(logits, *, temperature, top_k, top_p, rows_per_request=1,
     device = _device_of(logits)
     x = _dev(logits, device)
     rows, vocab = x.shape
+    rpr = int(rows_per_request)
+    pr = _per_request(temperature, top_k, top_p, order, (rows + rpr - 1) // max(rpr, 1), device, top_k_max,
+                      per_request)
+    kb = pr.top_k_max if pr is not None else int(top_k)
     if cap is None:
-        cap = min(int(top_k), vocab)
+        cap = min(kb, vocab)
     stream = torch.cuda.current_stream(device)
     kw = dict(dtype=torch.int32, device=device)
     ids = torch.empty((rows, cap), **kw)
@@ -218,13 +280,20 @@ def uno_filter_softmax(logits, *, temperature, top_k, top_p, rows_per_request=1,
     dn = torch.empty((rows, vocab), dtype=torch.float32, device=device) if dense else None
     sample = torch.empty(rows, **kw) if rng is not None else None
     rng_c = ctypes.byref(_rng(rng)) if rng is not None else None
-    nbytes = lib.uno_filter_softmax_workspace_bytes(rows, vocab, int(top_k))
+    nbytes = lib.uno_filter_softmax_workspace_bytes(rows, vocab, kb)
     ws = workspace(nbytes, device, stream)
-    st = lib.uno_filter_softmax(_ptr(x), _dtype_code(x), rows, vocab, x.stride(0), int(rows_per_request),
-                                _Params(float(temperature), int(top_k), float(top_p)), int(cap), _ptr(ids),
-                                _ptr(probs), _ptr(count), _ptr(dn), rng_c, _ptr(sample), _ptr(flags),
-                                _ptr(ws), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
-    _check("uno_filter_softmax", st)
+    if pr is None:
+        st = lib.uno_filter_softmax(_ptr(x), _dtype_code(x), rows, vocab, x.stride(0), rpr,
+                                    _Params(float(temperature), int(top_k), float(top_p)), int(cap), _ptr(ids),
+                                    _ptr(probs), _ptr(count), _ptr(dn), rng_c, _ptr(sample), _ptr(flags),
+                                    _ptr(ws), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
+        _check("uno_filter_softmax", st)
+    else:
+        st = lib.uno_filter_softmax_params(_ptr(x), _dtype_code(x), rows, vocab, x.stride(0), rpr,
+                                           ctypes.byref(pr.c), int(cap), _ptr(ids), _ptr(probs), _ptr(count),
+                                           _ptr(dn), rng_c, _ptr(sample), _ptr(flags), _ptr(ws), ws.numel(),
+                                           ctypes.c_void_p(stream.cuda_stream))
+        _check("uno_filter_softmax_params", st)
     out = dict(ids=ids, probs=probs, count=count, flags=flags)
     if dense:
         out["dense"] = dn
@@ -234,7 +303,7 @@ def uno_filter_softmax(logits, *, temperature, top_k, top_p, rows_per_request=1,
 
 
 def uno_linear_verify(target_logits, draft_ids, q_ids, q_probs, q_count, *, R, B, temperature, top_k, top_p,
-                      rng):
+                      rng, order="topk_first", top_k_max=None, per_request=False):
     """Linear rejection sampling.  target_logits [R*(B+1), vocab] (or
     [R, B+1, vocab]); draft_ids [R, B]; q_* as returned by uno_filter_softmax
     for the R*B draft rows.  Returns dict(tokens [R, B+1], accept_len,
@@ -255,21 +324,31 @@ def uno_linear_verify(target_logits, draft_ids, q_ids, q_probs, q_count, *, R, B
     acc = torch.empty(R, **kw)
     ntok = torch.empty(R, **kw)
     flags = torch.empty(R, **kw)
-    nbytes = lib.uno_linear_verify_workspace_bytes(R, B, vocab, int(top_k))
+    pr = _per_request(temperature, top_k, top_p, order, R, device, top_k_max, per_request)
+    kb = pr.top_k_max if pr is not None else int(top_k)
+    nbytes = lib.uno_linear_verify_workspace_bytes(R, B, vocab, kb)
     ws = workspace(nbytes, device, stream)
-    st = lib.uno_linear_verify(_ptr(x), _dtype_code(x), R, B, vocab,
-                               _Params(float(temperature), int(top_k), float(top_p)), _ptr(d), _ptr(qi),
-                               _ptr(qp), _ptr(qc), qi.shape[1], _rng(rng), _ptr(toks),
-                               _ptr(acc), _ptr(ntok), _ptr(flags), _ptr(ws), ws.numel(),
-                               ctypes.c_void_p(stream.cuda_stream))
-    _check("uno_linear_verify", st)
+    if pr is None:
+        st = lib.uno_linear_verify(_ptr(x), _dtype_code(x), R, B, vocab,
+                                   _Params(float(temperature), int(top_k), float(top_p)), _ptr(d), _ptr(qi),
+                                   _ptr(qp), _ptr(qc), qi.shape[1], _rng(rng), _ptr(toks),
+                                   _ptr(acc), _ptr(ntok), _ptr(flags), _ptr(ws), ws.numel(),
+                                   ctypes.c_void_p(stream.cuda_stream))
+        _check("uno_linear_verify", st)
+    else:
+        st = lib.uno_linear_verify_params(_ptr(x), _dtype_code(x), R, B, vocab, ctypes.byref(pr.c), _ptr(d),
+                                          _ptr(qi), _ptr(qp), _ptr(qc), qi.shape[1], _rng(rng), _ptr(toks),
+                                          _ptr(acc), _ptr(ntok), _ptr(flags), _ptr(ws), ws.numel(),
+                                          ctypes.c_void_p(stream.cuda_stream))
+        _check("uno_linear_verify_params", st)
     return _host_back(dict(tokens=toks, accept_len=acc, num_tokens=ntok, flags=flags), host)
 
 
 LAYOUT_GENERIC, LAYOUT_TWO_PASS = 0, 1
 
 
-def uno_linear_cycle(draft_logits, target_logits, *, R, B, temperature, top_k, top_p, rng, layout=LAYOUT_GENERIC):
+def uno_linear_cycle(draft_logits, target_logits, *, R, B, temperature, top_k, top_p, rng, layout=LAYOUT_GENERIC,
+                     order="topk_first", top_k_max=None, per_request=False):
     """One linear cycle in one call: draft_logits [R*B, vocab] (or [R, B,
     vocab]); target_logits [R*(B+1), vocab] for layout LAYOUT_GENERIC, [R*B,
     vocab] for LAYOUT_TWO_PASS (x_0 untested, target row i-1 tests x_i).
@@ -292,13 +371,22 @@ def uno_linear_cycle(draft_logits, target_logits, *, R, B, temperature, top_k, t
     ntok = torch.empty(R, **kw)
     flags = torch.empty(R, **kw)
     drafts = torch.empty((R, B), **kw)
-    nbytes = lib.uno_linear_cycle_workspace_bytes(R, B, vocab, int(top_k), int(layout))
+    pr = _per_request(temperature, top_k, top_p, order, R, device, top_k_max, per_request)
+    kb = pr.top_k_max if pr is not None else int(top_k)
+    nbytes = lib.uno_linear_cycle_workspace_bytes(R, B, vocab, kb, int(layout))
     ws = workspace(nbytes, device, stream)
-    st = lib.uno_linear_cycle(_ptr(d), _ptr(t), _dtype_code(d), R, B, vocab, int(layout),
-                              _Params(float(temperature), int(top_k), float(top_p)), _rng(rng), _ptr(toks),
-                              _ptr(nacc), _ptr(ntok), _ptr(flags), _ptr(drafts), _ptr(ws), ws.numel(),
-                              ctypes.c_void_p(stream.cuda_stream))
-    _check("uno_linear_cycle", st)
+    if pr is None:
+        st = lib.uno_linear_cycle(_ptr(d), _ptr(t), _dtype_code(d), R, B, vocab, int(layout),
+                                  _Params(float(temperature), int(top_k), float(top_p)), _rng(rng), _ptr(toks),
+                                  _ptr(nacc), _ptr(ntok), _ptr(flags), _ptr(drafts), _ptr(ws), ws.numel(),
+                                  ctypes.c_void_p(stream.cuda_stream))
+        _check("uno_linear_cycle", st)
+    else:
+        st = lib.uno_linear_cycle_params(_ptr(d), _ptr(t), _dtype_code(d), R, B, vocab, int(layout),
+                                         ctypes.byref(pr.c), _rng(rng), _ptr(toks), _ptr(nacc), _ptr(ntok),
+                                         _ptr(flags), _ptr(drafts), _ptr(ws), ws.numel(),
+                                         ctypes.c_void_p(stream.cuda_stream))
+        _check("uno_linear_cycle_params", st)
     return _host_back(dict(tokens=toks, num_accepted=nacc, num_tokens=ntok, flags=flags, drafts=drafts), host)
 
 
@@ -328,7 +416,7 @@ def uno_tree_topk_expand(q_ids, q_probs, q_count, *, R, B, K, V):
 
 
 def uno_tree_verify(target_logits, node_token, node_parent, num_nodes, *, R, B, V, temperature, top_k, top_p,
-                    rng):
+                    rng, order="topk_first", top_k_max=None, per_request=False):
     """Target-only tree verification.  target_logits [R*V, vocab] (one row
     per node).  Returns dict(tokens [R, B+1], accept_len, num_tokens,
     path_nodes [R, B+1], flags)."""
@@ -353,14 +441,48 @@ def uno_tree_verify(target_logits, node_token, node_parent, num_nodes, *, R, B, 
     acc = torch.empty(R, **kw)
     ntok = torch.empty(R, **kw)
     flags = torch.empty(R, **kw)
-    nbytes = lib.uno_tree_verify_workspace_bytes(R, V, vocab, int(top_k))
+    pr = _per_request(temperature, top_k, top_p, order, R, device, top_k_max, per_request)
+    kb = pr.top_k_max if pr is not None else int(top_k)
+    nbytes = lib.uno_tree_verify_workspace_bytes(R, V, vocab, kb)
     ws = workspace(nbytes, device, stream)
-    st = lib.uno_tree_verify(_ptr(x), _dtype_code(x), R, B, V, vocab,
-                             _Params(float(temperature), int(top_k), float(top_p)), _ptr(tk), _ptr(pa), _ptr(nn),
-                             _rng(rng), _ptr(toks), _ptr(acc), _ptr(ntok), _ptr(path),
-                             _ptr(flags), _ptr(ws), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
-    _check("uno_tree_verify", st)
+    if pr is None:
+        st = lib.uno_tree_verify(_ptr(x), _dtype_code(x), R, B, V, vocab,
+                                 _Params(float(temperature), int(top_k), float(top_p)), _ptr(tk), _ptr(pa),
+                                 _ptr(nn), _rng(rng), _ptr(toks), _ptr(acc), _ptr(ntok), _ptr(path),
+                                 _ptr(flags), _ptr(ws), ws.numel(), ctypes.c_void_p(stream.cuda_stream))
+        _check("uno_tree_verify", st)
+    else:
+        st = lib.uno_tree_verify_params(_ptr(x), _dtype_code(x), R, B, V, vocab, ctypes.byref(pr.c), _ptr(tk),
+                                        _ptr(pa), _ptr(nn), _rng(rng), _ptr(toks), _ptr(acc), _ptr(ntok),
+                                        _ptr(path), _ptr(flags), _ptr(ws), ws.numel(),
+                                        ctypes.c_void_p(stream.cuda_stream))
+        _check("uno_tree_verify_params", st)
     return _host_back(dict(tokens=toks, accept_len=acc, num_tokens=ntok, path_nodes=path, flags=flags), host)
+
+
+def uno_filter_softmax_params(logits, *, temperature, top_k, top_p, order="topk_first", top_k_max=None, **kw):
+    """uno_filter_softmax through the per-request entry point: temperature,
+    top_k and top_p hold one entry per request (scalars are repeated)."""
+    return uno_filter_softmax(logits, temperature=temperature, top_k=top_k, top_p=top_p, order=order,
+                              top_k_max=top_k_max, per_request=True, **kw)
+
+
+def uno_linear_verify_params(*args, temperature, top_k, top_p, order="topk_first", top_k_max=None, **kw):
+    """uno_linear_verify through the per-request entry point."""
+    return uno_linear_verify(*args, temperature=temperature, top_k=top_k, top_p=top_p, order=order,
+                             top_k_max=top_k_max, per_request=True, **kw)
+
+
+def uno_linear_cycle_params(*args, temperature, top_k, top_p, order="topk_first", top_k_max=None, **kw):
+    """uno_linear_cycle through the per-request entry point."""
+    return uno_linear_cycle(*args, temperature=temperature, top_k=top_k, top_p=top_p, order=order,
+                            top_k_max=top_k_max, per_request=True, **kw)
+
+
+def uno_tree_verify_params(*args, temperature, top_k, top_p, order="topk_first", top_k_max=None, **kw):
+    """uno_tree_verify through the per-request entry point."""
+    return uno_tree_verify(*args, temperature=temperature, top_k=top_k, top_p=top_p, order=order,
+                           top_k_max=top_k_max, per_request=True, **kw)
 
 
 def uno_linear_verify_noalloc(target_logits, draft_ids, q_ids, q_probs, q_count, *, R, B, temperature, top_k,

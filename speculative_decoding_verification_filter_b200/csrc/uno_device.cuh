@@ -18,7 +18,8 @@ constexpr int kMaxSplits = 16;             // CTAs that may share one row
 constexpr uint32_t kDrawProposal = 0, kDrawAccept = 1, kDrawResidual = 2, kDrawTarget = 3;
 
 // Flag bits, as in the public header.
-constexpr uint32_t kFlagNonfinite = 1u, kFlagDraftNotInSupport = 2u, kFlagResidualEmpty = 4u, kFlagTimeout = 8u;
+constexpr uint32_t kFlagNonfinite = 1u, kFlagDraftNotInSupport = 2u, kFlagResidualEmpty = 4u, kFlagTimeout = 8u,
+                   kFlagBadParams = 32u;
 
 // ---------------------------------------------------------------------------
 // Sortable 64-bit keys.  High word: the logit's binary32 bits mapped so that

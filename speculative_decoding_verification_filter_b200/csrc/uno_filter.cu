@@ -43,7 +43,13 @@ struct RowJob {
     int32_t S;                        // CTAs per row
     // sampling parameters
     float temperature, top_p;
-    int32_t k;                        // min(top_k, vocab)
+    int32_t k;                        // min(top_k, vocab); with per-request parameters, min(top_k_max, vocab)
+    // per-request sampling parameters (nullable: the scalars above apply)
+    const float* rq_T;
+    const int32_t* rq_k;
+    const float* rq_p;
+    int32_t joint;                    // 1: the top-p cut on the full-vocabulary softmax
+    double2* row_ms;                  // joint order: per row, (largest finite logit, sum of exp)
     int32_t hw, cap_w;                // warp buffer high-water mark / capacity
     int32_t merge_cap;                // entries of the merge area
     int32_t fin_off;                  // shared-memory offset of the finishing area (0: the ring)
@@ -108,6 +114,39 @@ struct RowJob {
 // the same arguments every cycle; the word it reads there changes).
 __device__ __forceinline__ uint32_t cycle_of(const RowJob& J) {
     return J.cycle_word != nullptr ? __ldg(J.cycle_word) : J.cycle;
+}
+
+// The request a row belongs to: a cycle's draft rows come B per request,
+// its target rows B + 1 (generic layout) or B (two-pass layout) per request.
+template <int MODE>
+__device__ __forceinline__ int32_t request_of(const RowJob& J, int64_t row) {
+    if (MODE == kModeCycle)
+        return (int32_t)(row < J.nq2 ? row / J.B : (row - J.nq2) / (J.B + 1 - J.sh));
+    return (int32_t)(row / J.rpr);
+}
+
+// A row's sampling parameters: the call's scalars, or its request's entries
+// of the per-request arrays.  Entries outside the valid ranges (or a top_k
+// above the call's bound) make `ok` false.
+struct RowParams {
+    float T, p;
+    int k;
+    bool ok;
+};
+template <int MODE>
+__device__ __forceinline__ RowParams row_params(const RowJob& J, int64_t row) {
+    RowParams r{J.temperature, J.top_p, J.k, true};
+    if (J.rq_T != nullptr) {
+        const int32_t q = request_of<MODE>(J, row);
+        r.T = J.rq_T[q];
+        r.p = J.rq_p[q];
+        const int32_t kq = J.rq_k[q];
+        const int64_t kv = (int64_t)kq < J.vocab ? (int64_t)kq : J.vocab;
+        r.ok = r.T >= 0.0f && r.T < __int_as_float(0x7f800000) && kq >= 1 && r.p > 0.0f && r.p <= 1.0f &&
+               kv <= (int64_t)J.k;
+        r.k = kv < 1 ? 1 : (kv > J.k ? J.k : (int)kv);
+    }
+    return r;
 }
 
 // ---------------------------------------------------------------------------
@@ -1283,28 +1322,46 @@ __device__ __forceinline__ void cta_rank_topk(const uint64_t* uni, int U, int k,
     }
 }
 
+// The joint order's normaliser of a row whose largest value is v0:
+// sum over every finite logit of exp((l - v0) / T), from the row's pair.
+__device__ __forceinline__ double joint_sum(const RowJob& J, int64_t row, double v0, double inv_t) {
+    const double2 ms = J.row_ms[row];
+    return ms.y * exp((ms.x - v0) * inv_t);
+}
+
+// A row's flags: bit 0 of rowbad: NaN / +inf (or no finite logit); bit 1: a
+// wait gave up; badp: its request's parameters are out of range.
+__device__ __forceinline__ uint32_t row_flags(bool bad, uint32_t rowbad, bool badp) {
+    if (!bad) return 0u;
+    if (badp) return kFlagBadParams | ((rowbad & 1u) ? kFlagNonfinite : 0u) | ((rowbad & 2u) ? kFlagTimeout : 0u);
+    return (rowbad & 2u) ? (kFlagTimeout | ((rowbad & 1u) ? kFlagNonfinite : 0u)) : kFlagNonfinite;
+}
+
 template <int MODE>
 __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n, uint32_t rowbad,
                                 const uint64_t* sel, double* wd, unsigned char* tail_smem, FinishShared& fs, int lane,
                                 uint64_t* pairs) {
-    const bool bad = rowbad != 0u || n == 0;
+    const RowParams rp = row_params<MODE>(J, row);
+    if (n > rp.k) n = rp.k;  // sel[] holds the best min(top_k_max, vocab), descending
+    const bool bad = rowbad != 0u || n == 0 || !rp.ok;
     int kept = 0;
     uint64_t oa = ~0ull, ob = ~0ull;  // (id, prob) pairs, ascending id after the sort
     if (!bad) {
         const uint64_t ka = lane < n ? sel[lane] : 0ull, kb = lane + 32 < n ? sel[lane + 32] : 0ull;
         double wa = 0.0, wb = 0.0;
-        if (J.temperature == 0.0f) {
+        if (rp.T == 0.0f) {
             kept = 1;
             wa = lane == 0 ? 1.0 : 0.0;
         } else {
             const double v0 = (double)key_value(sel[0]);
-            const double inv_t = 1.0 / (double)J.temperature;
+            const double inv_t = 1.0 / (double)rp.T;
             if (lane < n) wa = exp(((double)key_value(ka) - v0) * inv_t);
             if (lane + 32 < n) wb = exp(((double)key_value(kb) - v0) * inv_t);
-            if (J.top_p >= 1.0f) {
+            if (rp.p >= 1.0f) {
                 kept = n;
             } else {
-                const double inv_s = 1.0 / warp_sum_d(wa + wb);
+                const double S = J.joint ? joint_sum(J, row, v0, inv_t) : warp_sum_d(wa + wb);
+                const double inv_s = 1.0 / S;
                 const double pa = wa * inv_s, pb = wb * inv_s;
                 // mass before rank j
                 const double ia = warp_incl_scan_d(pa, lane);
@@ -1315,7 +1372,7 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
                     ea = 0.0;
                     eb = ta;
                 }
-                const double tp = (double)J.top_p;
+                const double tp = (double)rp.p;
                 const bool keepa = lane < n && (lane == 0 || ea < tp);
                 const bool keepb = lane + 32 < n && eb < tp;
                 kept = __popc(__ballot_sync(kFull, keepa)) + __popc(__ballot_sync(kFull, keepb));
@@ -1344,9 +1401,7 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
         oa = lane < kept ? pairs[lane] : ~0ull;
         ob = lane + 32 < kept ? pairs[lane + 32] : ~0ull;
     }
-    // bit 0 of rowbad: NaN / +inf (or no finite logit); bit 1: a wait gave up
-    const uint32_t rflags = !bad ? 0u : (rowbad & 2u) ? (kFlagTimeout | ((rowbad & 1u) ? kFlagNonfinite : 0u))
-                                                       : kFlagNonfinite;
+    const uint32_t rflags = row_flags(bad, rowbad, !rp.ok);
     if (MODE == kModeFilter || (MODE == kModeCycle && row < J.nq2)) {
         int32_t* ids = J.out_ids + (size_t)row * J.cap;
         float* pr = J.out_probs + (size_t)row * J.cap;
@@ -1409,29 +1464,33 @@ __device__ void finish_row(const RowJob& J, int64_t row, int32_t req, int n, uin
                            uint64_t* outk, double* wd, double* pd, unsigned char* tail_smem, FinishShared& fs, int warp,
                            int lane) {
     const int tid = threadIdx.x;
-    const bool bad = rowbad != 0u || n == 0;
+    const RowParams rp = row_params<MODE>(J, row);
+    if (n > rp.k) n = rp.k;  // sel[] holds the best min(top_k_max, vocab), descending
+    const bool bad = rowbad != 0u || n == 0 || !rp.ok;
     int kept = 0;
     if (!bad) {
         const double v0 = (double)key_value(sel[0]);
-        if (J.temperature == 0.0f) {
+        if (rp.T == 0.0f) {
             kept = 1;
             if (tid == 0) fs.W = 1.0;
             if (tid == 0) wd[0] = 1.0;
         } else {
-            const double temp = (double)J.temperature;
+            const double temp = (double)rp.T;
             for (int j = tid; j < n; j += kThreads) wd[j] = exp(((double)key_value(sel[j]) - v0) / temp);
             __syncthreads();
-            if (tid == 0) fs.S = serial_sum(wd, n);  // the defined (descending) order
+            // the defined (descending) order; the joint order's normaliser
+            // covers the whole row
+            if (tid == 0) fs.S = J.joint ? joint_sum(J, row, v0, 1.0 / temp) : serial_sum(wd, n);
             __syncthreads();
             const double S = fs.S;
             for (int j = tid; j < n; j += kThreads) pd[j] = wd[j] / S;
             __syncthreads();
             if (tid == 0) {
                 int kk = 0;
-                if (J.top_p >= 1.0f) {
+                if (rp.p >= 1.0f) {
                     kk = n;
                 } else {
-                    const double tp = (double)J.top_p;
+                    const double tp = (double)rp.p;
                     double m = 0.0;
                     int j = 0;
                     for (; j + 8 <= n; j += 8) {  // loads ahead of the dependent walk
@@ -1465,7 +1524,7 @@ __device__ void finish_row(const RowJob& J, int64_t row, int32_t req, int n, uin
             }
         }
         __syncthreads();
-        if (J.temperature != 0.0f) kept = fs.kept;
+        if (rp.T != 0.0f) kept = fs.kept;
         const double W = fs.W;
         // (id, prob) pairs in ascending id order
         for (int j = tid; j < kept; j += kThreads) {
@@ -1485,9 +1544,7 @@ __device__ void finish_row(const RowJob& J, int64_t row, int32_t req, int n, uin
         }
         __syncthreads();
     }
-    // bit 0 of rowbad: NaN / +inf (or no finite logit); bit 1: a wait gave up
-    const uint32_t rflags = !bad ? 0u : (rowbad & 2u) ? (kFlagTimeout | ((rowbad & 1u) ? kFlagNonfinite : 0u))
-                                                       : kFlagNonfinite;
+    const uint32_t rflags = row_flags(bad, rowbad, !rp.ok);
 
     if (MODE == kModeFilter) {
         int32_t* ids = J.out_ids + (size_t)row * J.cap;
@@ -3046,6 +3103,103 @@ __global__ void __launch_bounds__(32 * kTailWarps) tail_kernel(const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
+// The joint filter order's normaliser, one CTA per row, before the row
+// kernels: the row's largest finite logit m and sum_j exp((l_j - m) / T) over
+// its finite logits, in one read of the row.  Each thread keeps a running
+// maximum and rescales its sum when the maximum rises.  The exponent
+// (l - m) / T is formed as (l - m) * c with c = log2(e) / T split into two
+// floats (hi + lo), so that the rounding of c does not bias every term alike;
+// a unit's terms are added in float, units in double.
+// ---------------------------------------------------------------------------
+constexpr int kJointThreads = 256;
+
+struct JointScale {
+    float hi, lo;
+};
+__device__ __forceinline__ JointScale joint_scale(float T) {
+    const double c = 1.4426950408889634 / (double)T;  // log2(e) / T
+    JointScale k;
+    k.hi = (float)c;
+    k.lo = (float)(c - (double)k.hi);
+    return k;
+}
+__device__ __forceinline__ float joint_term(float v, float m, JointScale c) {
+    const float d = v - m;
+    return exp2f(fmaf(d, c.hi, d * c.lo));
+}
+// (m, s) with s relative to m: raise m to at least x, rescaling s
+__device__ __forceinline__ void joint_raise(float& m, double& s, float x, JointScale c) {
+    if (x > m) {
+        const double d = (double)m - (double)x;
+        s *= exp2(d * ((double)c.hi + (double)c.lo));
+        m = x;
+    }
+}
+__device__ __forceinline__ void joint_merge(float& m, double& s, float m2, double s2, JointScale c) {
+    const float M = m > m2 ? m : m2;
+    const double cc = (double)c.hi + (double)c.lo;
+    s = s * exp2(((double)m - (double)M) * cc) + s2 * exp2(((double)m2 - (double)M) * cc);
+    m = M;
+}
+
+template <typename T, int MODE>
+__global__ void __launch_bounds__(kJointThreads) joint_norm_kernel(const __grid_constant__ RowJob J) {
+    const int64_t row = blockIdx.x;
+    if (!item_active<MODE>(J, row)) return;
+    const RowParams rp = row_params<MODE>(J, row);
+    if (!(rp.T > 0.0f) || !rp.ok) {  // greedy rows and rows with bad parameters need no normaliser
+        if (threadIdx.x == 0) J.row_ms[row] = make_double2(0.0, 0.0);
+        return;
+    }
+    const JointScale c = joint_scale(rp.T);
+    const RowGeom g = row_geom<T>(J, row);
+    constexpr int KPU = Elem<T>::kPerUnit;
+    float m = -3.402823466e38f;  // lowest finite float
+    double s = 0.0;
+    const uint4* units = reinterpret_cast<const uint4*>(g.base + (size_t)g.head * Elem<T>::kBytes);
+    for (int64_t i = threadIdx.x; i < g.nunit; i += kJointThreads) {
+        const uint4 r = __ldg(units + i);
+        float um = m;
+#pragma unroll
+        for (int e = 0; e < KPU; ++e) {
+            const float v = Elem<T>::get(r, e);
+            um = v > um ? v : um;
+        }
+        joint_raise(m, s, um, c);
+        float t = 0.0f;
+#pragma unroll
+        for (int e = 0; e < KPU; ++e) t += joint_term(Elem<T>::get(r, e), m, c);
+        s += (double)t;
+    }
+    // the head and tail scalars (fewer than one unit each)
+    const int64_t ntail = J.vocab - g.tail_begin;
+    if (threadIdx.x < g.head + ntail) {
+        const int64_t id = threadIdx.x < g.head ? (int64_t)threadIdx.x : g.tail_begin + (threadIdx.x - g.head);
+        const float v = Elem<T>::load_scalar(g.base + (size_t)id * Elem<T>::kBytes);
+        joint_raise(m, s, v, c);
+        s += (double)joint_term(v, m, c);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(kFull, m, o);
+        const double s2 = __shfl_xor_sync(kFull, s, o);
+        joint_merge(m, s, m2, s2, c);
+    }
+    __shared__ float wm[kJointThreads / 32];
+    __shared__ double wsum[kJointThreads / 32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        wm[warp] = m;
+        wsum[warp] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kJointThreads / 32; ++w) joint_merge(m, s, wm[w], wsum[w], c);
+        J.row_ms[row] = make_double2((double)m, s);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Tree expansion: one CTA per request.  Its warps extract the top-K of the B
 // marginals side by side; warp 0 then expands the tree.
 // ---------------------------------------------------------------------------
@@ -3261,8 +3415,8 @@ constexpr int64_t kCounterWords = UNO_WORKSPACE_COUNTER_BYTES / 4;
 constexpr int64_t kRowCounterWords = kCounterWords / 2;
 
 struct WsLayout {
-    size_t row_ticket, req_ticket, part_keys, part_count, part_flags, part_spec, redo, c_ids, c_probs, c_count,
-        c_flags, total;
+    size_t row_ticket, req_ticket, part_keys, part_count, part_flags, part_spec, redo, row_ms, c_ids, c_probs,
+        c_count, c_flags, total;
 };
 
 static WsLayout ws_layout(int64_t rows, int32_t k, bool compact) {
@@ -3285,6 +3439,8 @@ static WsLayout ws_layout(int64_t rows, int32_t k, bool compact) {
     off = align_up(off + nslot * 8, 256);
     L.redo = off;
     off = align_up(off + ((size_t)rows + kPipeMaxGrid) * 4, 256);
+    L.row_ms = off;
+    off = align_up(off + (size_t)rows * 16, 256);
     L.c_ids = off;
     const size_t crow = compact ? (size_t)rows : 0;
     const size_t ks = (size_t)((k + 3) & ~3);
@@ -3354,6 +3510,14 @@ static size_t row_smem_bytes(RowJob& J) {
 
 // The pipelined kernel: grid (balanced pieces), ring depth and shared memory.
 // Returns UNO_ERR_UNSUPPORTED (nothing launched) when it does not fit.
+// The joint order's per-row normalisers, ahead of the row kernels.
+template <typename T, int MODE>
+static uno_status launch_joint(const RowJob& J, cudaStream_t stream) {
+    if (!J.joint || J.rows <= 0) return UNO_OK;
+    joint_norm_kernel<T, MODE><<<(unsigned)J.rows, kJointThreads, 0, stream>>>(J);
+    return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
+}
+
 template <typename T, int MODE>
 static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     J.hw = J.k + 16 > 64 ? J.k + 16 : 64;
@@ -3414,6 +3578,8 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
 
 template <typename T, int MODE>
 static uno_status launch_rows(RowJob J, cudaStream_t stream) {
+    const uno_status sj = launch_joint<T, MODE>(J, stream);
+    if (sj != UNO_OK) return sj;
     if (J.k <= kPipeMaxK && J.out_dense == nullptr) {
         const uno_status st = launch_pipe<T, MODE>(J, stream);
         if (st != UNO_ERR_UNSUPPORTED) return st;
@@ -3465,12 +3631,38 @@ static void bind_workspace(RowJob& J, void* ws, const WsLayout& L) {
     J.part_flags = reinterpret_cast<uint32_t*>(b + L.part_flags);
     J.part_spec = reinterpret_cast<uint64_t*>(b + L.part_spec);
     J.redo = reinterpret_cast<int32_t*>(b + L.redo);
+    J.row_ms = reinterpret_cast<double2*>(b + L.row_ms);
     J.hint = reinterpret_cast<uint64_t*>(b + UNO_WORKSPACE_COUNTER_BYTES);
     J.c_ids = reinterpret_cast<int32_t*>(b + L.c_ids);
     J.ks = (J.k + 3) & ~3;
     J.c_probs = reinterpret_cast<float*>(b + L.c_probs);
     J.c_count = reinterpret_cast<int32_t*>(b + L.c_count);
     J.c_flags = reinterpret_cast<uint32_t*>(b + L.c_flags);
+}
+
+// Per-request parameters: the call's sampling parameters for its checks and
+// sizes (top_k = the bound), the arrays for the rows.
+static bool request_params_ok(const uno_request_params* rp) {
+    if (rp == nullptr || !rp->temperature || !rp->top_k || !rp->top_p) return false;
+    if ((reinterpret_cast<uintptr_t>(rp->temperature) | reinterpret_cast<uintptr_t>(rp->top_k) |
+         reinterpret_cast<uintptr_t>(rp->top_p)) % 4 != 0)
+        return false;
+    if (rp->top_k_max < 1) return false;
+    return rp->order == UNO_ORDER_TOPK_FIRST || rp->order == UNO_ORDER_JOINT;
+}
+static uno_sampling_params bound_params(const uno_request_params* rp) {
+    uno_sampling_params sp;
+    sp.temperature = 1.0f;
+    sp.top_k = rp->top_k_max;
+    sp.top_p = 1.0f;
+    return sp;
+}
+static void apply_request_params(RowJob& J, const uno_request_params* rp) {
+    if (rp == nullptr) return;
+    J.rq_T = rp->temperature;
+    J.rq_k = rp->top_k;
+    J.rq_p = rp->top_p;
+    J.joint = rp->order == UNO_ORDER_JOINT ? 1 : 0;
 }
 
 }  // namespace uno
@@ -3512,8 +3704,8 @@ static bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintp
 // a device cycle word, when given, is a 4-byte aligned uint32_t
 static bool rng_ok(const uno_rng& r) { return r.cycle_word == nullptr || aligned_to(r.cycle_word, 4); }
 
-uno_status uno_filter_softmax(const void* logits, uno_dtype dt, int64_t rows, int64_t vocab, int64_t row_stride,
-                              int32_t rows_per_request, uno_sampling_params sp, int32_t cap, int32_t* out_ids,
+static uno_status filter_softmax_impl(const void* logits, uno_dtype dt, int64_t rows, int64_t vocab, int64_t row_stride,
+                              int32_t rows_per_request, uno_sampling_params sp, const uno_request_params* rp, int32_t cap, int32_t* out_ids,
                               float* out_probs, int32_t* out_count, float* out_dense, const uno_rng* rng,
                               int32_t* out_sample, uint32_t* out_flags, void* workspace, size_t workspace_bytes,
                               void* stream) {
@@ -3540,6 +3732,7 @@ uno_status uno_filter_softmax(const void* logits, uno_dtype dt, int64_t rows, in
     J.temperature = sp.temperature;
     J.top_p = sp.top_p;
     J.k = k;
+    apply_request_params(J, rp);
     J.out_ids = out_ids;
     J.out_probs = out_probs;
     J.out_count = out_count;
@@ -3557,8 +3750,8 @@ uno_status uno_filter_softmax(const void* logits, uno_dtype dt, int64_t rows, in
     return dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeFilter>(J, s) : launch_rows<float, kModeFilter>(J, s);
 }
 
-uno_status uno_linear_verify(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int64_t vocab,
-                             uno_sampling_params sp, const int32_t* draft_ids, const int32_t* q_ids,
+static uno_status linear_verify_impl(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int64_t vocab,
+                             uno_sampling_params sp, const uno_request_params* rp, const int32_t* draft_ids, const int32_t* q_ids,
                              const float* q_probs, const int32_t* q_count, int32_t q_cap, uno_rng rng,
                              int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
                              uint32_t* out_flags, void* workspace, size_t workspace_bytes, void* stream) {
@@ -3586,6 +3779,7 @@ uno_status uno_linear_verify(const void* target_logits, uno_dtype dt, int32_t R,
     J.temperature = sp.temperature;
     J.top_p = sp.top_p;
     J.k = k;
+    apply_request_params(J, rp);
     J.seed = rng.seed;
     J.cycle = rng.cycle;
     J.cycle_word = rng.cycle_word;
@@ -3612,8 +3806,8 @@ size_t uno_linear_cycle_workspace_bytes(int32_t R, int32_t B, int64_t vocab, int
     return cycle_layout(R, B, k, layout).total;
 }
 
-uno_status uno_linear_cycle(const void* draft_logits, const void* target_logits, uno_dtype dt, int32_t R, int32_t B,
-                            int64_t vocab, int32_t layout, uno_sampling_params sp, uno_rng rng, int32_t* out_tokens,
+static uno_status linear_cycle_impl(const void* draft_logits, const void* target_logits, uno_dtype dt, int32_t R, int32_t B,
+                            int64_t vocab, int32_t layout, uno_sampling_params sp, const uno_request_params* rp, uno_rng rng, int32_t* out_tokens,
                             int32_t* out_num_accepted, int32_t* out_num_tokens, uint32_t* out_flags,
                             int32_t* out_draft_ids, void* workspace, size_t workspace_bytes, void* stream) {
     if (!draft_logits || !target_logits || !out_tokens || !out_num_accepted || !out_num_tokens || !out_flags)
@@ -3646,6 +3840,7 @@ uno_status uno_linear_cycle(const void* draft_logits, const void* target_logits,
     J.temperature = sp.temperature;
     J.top_p = sp.top_p;
     J.k = k;
+    apply_request_params(J, rp);
     J.seed = rng.seed;
     J.cycle = rng.cycle;
     J.cycle_word = rng.cycle_word;
@@ -3679,8 +3874,10 @@ uno_status uno_linear_cycle(const void* draft_logits, const void* target_logits,
         J.nq2 = nq;
         J.rows = nq + np;
         J.rpr = B;
-        const uno_status st = dt == UNO_BF16 ? launch_pipe<__nv_bfloat16, kModeCycle>(J, s)
-                                             : launch_pipe<float, kModeCycle>(J, s);
+        uno_status st = dt == UNO_BF16 ? launch_joint<__nv_bfloat16, kModeCycle>(J, s)
+                                       : launch_joint<float, kModeCycle>(J, s);
+        if (st != UNO_OK) return st;
+        st = dt == UNO_BF16 ? launch_pipe<__nv_bfloat16, kModeCycle>(J, s) : launch_pipe<float, kModeCycle>(J, s);
         if (st != UNO_ERR_UNSUPPORTED) return st;
     }
     // the draft rows, then the target rows with the request tails
@@ -3738,8 +3935,8 @@ uno_status uno_tree_topk_expand(const int32_t* q_ids, const float* q_probs, cons
     return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
 }
 
-uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int32_t V, int64_t vocab,
-                           uno_sampling_params sp, const int32_t* node_token, const int32_t* node_parent,
+static uno_status tree_verify_impl(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int32_t V, int64_t vocab,
+                           uno_sampling_params sp, const uno_request_params* rp, const int32_t* node_token, const int32_t* node_parent,
                            const int32_t* num_nodes, uno_rng rng, int32_t* out_tokens, int32_t* out_accept_len,
                            int32_t* out_num_tokens, int32_t* out_path_nodes, uint32_t* out_flags, void* workspace,
                            size_t workspace_bytes, void* stream) {
@@ -3768,6 +3965,7 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
     J.temperature = sp.temperature;
     J.top_p = sp.top_p;
     J.k = k;
+    apply_request_params(J, rp);
     J.seed = rng.seed;
     J.cycle = rng.cycle;
     J.cycle_word = rng.cycle_word;
@@ -3785,6 +3983,94 @@ uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, i
     bind_workspace(J, workspace, L);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return dt == UNO_BF16 ? launch_rows<__nv_bfloat16, kModeTree>(J, s) : launch_rows<float, kModeTree>(J, s);
+}
+
+// ---------------------------------------------------------------------------
+// The entry points: one set with the call's sampling parameters, one with
+// per-request parameter arrays and a filter order.
+// ---------------------------------------------------------------------------
+uno_status uno_filter_softmax(const void* logits, uno_dtype dt, int64_t rows, int64_t vocab, int64_t row_stride,
+                              int32_t rows_per_request, uno_sampling_params sp, int32_t cap, int32_t* out_ids,
+                              float* out_probs, int32_t* out_count, float* out_dense, const uno_rng* rng,
+                              int32_t* out_sample, uint32_t* out_flags, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    return filter_softmax_impl(logits, dt, rows, vocab, row_stride, rows_per_request, sp, nullptr, cap, out_ids,
+                               out_probs, out_count, out_dense, rng, out_sample, out_flags, workspace,
+                               workspace_bytes, stream);
+}
+
+uno_status uno_filter_softmax_params(const void* logits, uno_dtype dt, int64_t rows, int64_t vocab,
+                                     int64_t row_stride, int32_t rows_per_request, const uno_request_params* rp,
+                                     int32_t cap, int32_t* out_ids, float* out_probs, int32_t* out_count,
+                                     float* out_dense, const uno_rng* rng, int32_t* out_sample, uint32_t* out_flags,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+    if (!request_params_ok(rp)) return UNO_ERR_INVALID_ARG;
+    return filter_softmax_impl(logits, dt, rows, vocab, row_stride, rows_per_request, bound_params(rp), rp, cap,
+                               out_ids, out_probs, out_count, out_dense, rng, out_sample, out_flags, workspace,
+                               workspace_bytes, stream);
+}
+
+uno_status uno_linear_verify(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int64_t vocab,
+                             uno_sampling_params sp, const int32_t* draft_ids, const int32_t* q_ids,
+                             const float* q_probs, const int32_t* q_count, int32_t q_cap, uno_rng rng,
+                             int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                             uint32_t* out_flags, void* workspace, size_t workspace_bytes, void* stream) {
+    return linear_verify_impl(target_logits, dt, R, B, vocab, sp, nullptr, draft_ids, q_ids, q_probs, q_count, q_cap,
+                              rng, out_tokens, out_accept_len, out_num_tokens, out_flags, workspace, workspace_bytes,
+                              stream);
+}
+
+uno_status uno_linear_verify_params(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int64_t vocab,
+                                    const uno_request_params* rp, const int32_t* draft_ids, const int32_t* q_ids,
+                                    const float* q_probs, const int32_t* q_count, int32_t q_cap, uno_rng rng,
+                                    int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                                    uint32_t* out_flags, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!request_params_ok(rp)) return UNO_ERR_INVALID_ARG;
+    return linear_verify_impl(target_logits, dt, R, B, vocab, bound_params(rp), rp, draft_ids, q_ids, q_probs,
+                              q_count, q_cap, rng, out_tokens, out_accept_len, out_num_tokens, out_flags, workspace,
+                              workspace_bytes, stream);
+}
+
+uno_status uno_linear_cycle(const void* draft_logits, const void* target_logits, uno_dtype dt, int32_t R, int32_t B,
+                            int64_t vocab, int32_t layout, uno_sampling_params sp, uno_rng rng, int32_t* out_tokens,
+                            int32_t* out_num_accepted, int32_t* out_num_tokens, uint32_t* out_flags,
+                            int32_t* out_draft_ids, void* workspace, size_t workspace_bytes, void* stream) {
+    return linear_cycle_impl(draft_logits, target_logits, dt, R, B, vocab, layout, sp, nullptr, rng, out_tokens,
+                             out_num_accepted, out_num_tokens, out_flags, out_draft_ids, workspace, workspace_bytes,
+                             stream);
+}
+
+uno_status uno_linear_cycle_params(const void* draft_logits, const void* target_logits, uno_dtype dt, int32_t R,
+                                   int32_t B, int64_t vocab, int32_t layout, const uno_request_params* rp,
+                                   uno_rng rng, int32_t* out_tokens, int32_t* out_num_accepted,
+                                   int32_t* out_num_tokens, uint32_t* out_flags, int32_t* out_draft_ids,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    if (!request_params_ok(rp)) return UNO_ERR_INVALID_ARG;
+    return linear_cycle_impl(draft_logits, target_logits, dt, R, B, vocab, layout, bound_params(rp), rp, rng,
+                             out_tokens, out_num_accepted, out_num_tokens, out_flags, out_draft_ids, workspace,
+                             workspace_bytes, stream);
+}
+
+uno_status uno_tree_verify(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int32_t V, int64_t vocab,
+                           uno_sampling_params sp, const int32_t* node_token, const int32_t* node_parent,
+                           const int32_t* num_nodes, uno_rng rng, int32_t* out_tokens, int32_t* out_accept_len,
+                           int32_t* out_num_tokens, int32_t* out_path_nodes, uint32_t* out_flags, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    return tree_verify_impl(target_logits, dt, R, B, V, vocab, sp, nullptr, node_token, node_parent, num_nodes, rng,
+                            out_tokens, out_accept_len, out_num_tokens, out_path_nodes, out_flags, workspace,
+                            workspace_bytes, stream);
+}
+
+uno_status uno_tree_verify_params(const void* target_logits, uno_dtype dt, int32_t R, int32_t B, int32_t V,
+                                  int64_t vocab, const uno_request_params* rp, const int32_t* node_token,
+                                  const int32_t* node_parent, const int32_t* num_nodes, uno_rng rng,
+                                  int32_t* out_tokens, int32_t* out_accept_len, int32_t* out_num_tokens,
+                                  int32_t* out_path_nodes, uint32_t* out_flags, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    if (!request_params_ok(rp)) return UNO_ERR_INVALID_ARG;
+    return tree_verify_impl(target_logits, dt, R, B, V, vocab, bound_params(rp), rp, node_token, node_parent,
+                            num_nodes, rng, out_tokens, out_accept_len, out_num_tokens, out_path_nodes, out_flags,
+                            workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -121,3 +121,30 @@ def test_misaligned_cycle_word_rejected_on_the_host():
     st = lib.uno_tree_verify(fake, 1, 1, 4, 8, 1000, b._Params(1.0, 50, 0.95), fake, fake, fake, rng, fake, fake,
                              fake, fake, fake, fake, 1 << 24, None)
     assert st == 1
+
+
+@pytest.mark.parametrize("bad", ["null", "order", "kmax", "misaligned", "null_array"])
+def test_request_params_rejected_on_the_host(bad):
+    """The per-request entry points check the parameter struct on the host
+    before any device work (the fake pointers are never dereferenced)."""
+    from speculative_decoding_verification_filter_b200 import _binding as b
+    lib = b.load_library()
+    fake = ctypes.c_void_p(0x1000)
+    a = dict(T=0x1000, k=0x2000, p=0x3000, kmax=5, order=0)
+    if bad == "order":
+        a["order"] = 7
+    elif bad == "kmax":
+        a["kmax"] = 0
+    elif bad == "misaligned":
+        a["k"] = 0x2002
+    elif bad == "null_array":
+        a["p"] = None
+    rp = None if bad == "null" else ctypes.byref(
+        b._ReqParams(ctypes.c_void_p(a["T"]), ctypes.c_void_p(a["k"]), ctypes.c_void_p(a["p"]) if a["p"] else None,
+                     a["kmax"], a["order"]))
+    st = lib.uno_filter_softmax_params(fake, 0, 4, 10, 10, 1, rp, 8, fake, fake, fake, None, None, None, fake, fake,
+                                       1 << 20, None)
+    assert st == 1
+    st = lib.uno_linear_verify_params(fake, 1, 1, 4, 1000, rp, fake, fake, fake, fake, 8, b._Rng(1, 0), fake, fake,
+                                      fake, fake, fake, 1 << 24, None)
+    assert st == 1
