@@ -76,6 +76,7 @@ struct RowJob {
     int32_t* part_count;   // [rows*S]
     uint32_t* part_flags;  // [rows*S]
     uint64_t* part_spec;   // pipelined kernel: the predicted threshold each piece used
+    double2* part_ms;      // pipelined kernel, joint order: each piece's pair (m, s)
     int32_t* redo;         // pipelined kernel: rows each CTA reads again (rows + grid entries)
     uint64_t* hint;        // pipelined kernel: per CTA, the prediction carried to the next call
     int32_t* c_ids;        // [rows][ks]  compact target rows (verifiers)
@@ -147,6 +148,49 @@ __device__ __forceinline__ RowParams row_params(const RowJob& J, int64_t row) {
         r.k = kv < 1 ? 1 : (kv > J.k ? J.k : (int)kv);
     }
     return r;
+}
+
+// The joint order's normaliser is carried as a pair (m, s): a running
+// maximum m of the row's finite logits and s = sum of 2^((l - m) * c) over
+// them, c = log2(e) / T.  The exponent (l - m) * c is formed with c split
+// into two floats (hi + lo), so that the rounding of c does not bias every
+// term alike.
+struct JointScale {
+    float hi, lo;
+};
+__device__ __forceinline__ JointScale joint_scale(float T) {
+    const double c = 1.4426950408889634 / (double)T;  // log2(e) / T
+    JointScale k;
+    k.hi = (float)c;
+    k.lo = (float)(c - (double)k.hi);
+    return k;
+}
+__device__ __forceinline__ float joint_term(float v, float m, JointScale c) {
+    const float d = v - m;
+    return exp2f(fmaf(d, c.hi, d * c.lo));
+}
+// The same term from the hardware base-2 exponential (PTX ex2.approx.ftz:
+// relative error about 2^-22; results below 2^-126 flush to zero, which
+// leaves a row's sum unchanged at float precision).
+__device__ __forceinline__ float joint_term_fast(float v, float m, JointScale c) {
+    const float d = v - m;
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(fmaf(d, c.hi, d * c.lo)));
+    return y;
+}
+// (m, s) with s relative to m: raise m to at least x, rescaling s
+__device__ __forceinline__ void joint_raise(float& m, double& s, float x, JointScale c) {
+    if (x > m) {
+        const double d = (double)m - (double)x;
+        s *= exp2(d * ((double)c.hi + (double)c.lo));
+        m = x;
+    }
+}
+__device__ __forceinline__ void joint_merge(float& m, double& s, float m2, double s2, JointScale c) {
+    const float M = m > m2 ? m : m2;
+    const double cc = (double)c.hi + (double)c.lo;
+    s = s * exp2(((double)m - (double)M) * cc) + s2 * exp2(((double)m2 - (double)M) * cc);
+    m = M;
 }
 
 // ---------------------------------------------------------------------------
@@ -1337,11 +1381,13 @@ __device__ __forceinline__ uint32_t row_flags(bool bad, uint32_t rowbad, bool ba
     return (rowbad & 2u) ? (kFlagTimeout | ((rowbad & 1u) ? kFlagNonfinite : 0u)) : kFlagNonfinite;
 }
 
-template <int MODE>
+// jms: the row's joint-order pair when the caller accumulated it (else the
+// normaliser pass left it in J.row_ms).
+template <int MODE, int PR>
 __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n, uint32_t rowbad,
                                 const uint64_t* sel, double* wd, unsigned char* tail_smem, FinishShared& fs, int lane,
-                                uint64_t* pairs) {
-    const RowParams rp = row_params<MODE>(J, row);
+                                uint64_t* pairs, const double2* jms) {
+    const RowParams rp = PR ? row_params<MODE>(J, row) : RowParams{J.temperature, J.top_p, J.k, true};
     if (n > rp.k) n = rp.k;  // sel[] holds the best min(top_k_max, vocab), descending
     const bool bad = rowbad != 0u || n == 0 || !rp.ok;
     int kept = 0;
@@ -1360,7 +1406,8 @@ __device__ void finish_row_warp(const RowJob& J, int64_t row, int32_t req, int n
             if (rp.p >= 1.0f) {
                 kept = n;
             } else {
-                const double S = J.joint ? joint_sum(J, row, v0, inv_t) : warp_sum_d(wa + wb);
+                const double S = !(PR && J.joint) ? warp_sum_d(wa + wb)
+                                 : jms != nullptr ? jms->y * exp((jms->x - v0) * inv_t) : joint_sum(J, row, v0, inv_t);
                 const double inv_s = 1.0 / S;
                 const double pa = wa * inv_s, pb = wb * inv_s;
                 // mass before rank j
@@ -1758,7 +1805,8 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const __grid_constant_
     }
 
     if (J.k <= 64) {
-        if (warp == 0) finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, smem + J.tail_off, fs, lane, outk);
+        if (warp == 0)
+            finish_row_warp<MODE, 1>(J, row, req, n, rowbad, sel, wd, smem + J.tail_off, fs, lane, outk, nullptr);
     } else {
         finish_row<MODE>(J, row, req, n, rowbad, sel, outk, wd, pd, smem + J.tail_off, fs, warp, lane);
     }
@@ -1847,6 +1895,8 @@ struct __align__(16) PipeShared {
     uint32_t boot_ready[kPipeSlots];        // the seed is in tau
     uint32_t mode[kPipeSlots];              // the piece's mode, set by its first consumer (1 predicted, 2 not)
     int cnt[kPipeSlots][kPipeConsumers];    // candidates per consumer warp of the slot's piece
+    float jm[kPipeSlots][kPipeConsumers];   // joint order: per consumer warp, its pair (m, s) for the piece
+    double js[kPipeSlots][kPipeConsumers];
     int wcnt[kPipeConsumers];               // candidate counts (compaction bookkeeping)
     uint32_t bad[kPipeSlots];               // NaN / +inf (bit 0) or gave-up (bit 1) of the slot's piece
     unsigned long long spec[2];             // the latest prediction (a threshold key), per row set
@@ -2518,7 +2568,39 @@ __device__ __forceinline__ uint32_t boot_threshold(const uint32_t* bv, int nA, i
 
 
 // Consumer warp c (0 .. kPipeConsumers-1): ring elements q with q % 8 == c.
-template <typename T, int MODE>
+// Joint order: add a stage's elements to the lane's pair (m, s).  lm is the
+// ordered key of the lane's largest finite element in the stage (0: none).
+// The stage's terms go to four float sums (independent chains of at most 64
+// terms each), then to s in double.
+template <typename T>
+__device__ __forceinline__ void joint_stage(const uint4* lsp, int left, uint32_t lm, JointScale c, float& m,
+                                            double& s) {
+    if (lm != 0u) joint_raise(m, s, float_of_ord(lm), c);
+    float t[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 4
+    for (int u = 0; u < kPLaneUnits; ++u) {
+        if (32 * u < left) {
+            const uint4 r = lsp[u * 32];
+#pragma unroll
+            for (int e = 0; e < Elem<T>::kPerUnit; ++e) t[e & 3] += joint_term_fast(Elem<T>::get(r, e), m, c);
+        }
+    }
+    s += (double)((t[0] + t[1]) + (t[2] + t[3]));
+}
+
+// A warp's pairs merged into every lane.
+__device__ __forceinline__ void joint_warp_merge(float& m, double& s, JointScale c) {
+#pragma unroll 1
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(kFull, m, o);
+        const double s2 = __shfl_xor_sync(kFull, s, o);
+        joint_merge(m, s, m2, s2, c);
+    }
+}
+
+constexpr float kLowestFloat = -3.402823466e38f;
+
+template <typename T, int MODE, int PR>
 __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char* ring, uint64_t* slots, int c,
                              int lane) {
     typedef StageScan<T> SS;
@@ -2538,6 +2620,16 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
         // the finisher is done with this slot's previous piece
         if ((used & sb) && !pipe_wait_warp(&P.slot_empty[slot], (par & sb) ? 0u : 1u, P)) fail = true;
         const Piece p = redo ? whole_row<T>(J, L.cr, row) : piece_of<T>(J, L.cr, row);
+        // joint order: the piece's pair (m, s) over every element it reads
+        bool jon = false;
+        JointScale jc{0.0f, 0.0f};
+        if (PR && J.joint) {
+            const RowParams rp = row_params<MODE>(J, row);
+            jon = rp.ok && rp.T > 0.0f;
+            if (jon) jc = joint_scale(rp.T);
+        }
+        float jm = kLowestFloat;
+        double js = 0.0;
         // a cycle's draft rows and target rows keep separate predictions
         const int pset = row_set<MODE>(J, row);
         // the first consumer warp to start the piece fixes its mode: predicted
@@ -2579,6 +2671,10 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
                 } else if (v != -__int_as_float(0x7f800000)) {
                     key = make_key(v, (uint32_t)id);
                     has = true;
+                    if (jon) {
+                        joint_raise(jm, js, v, jc);
+                        js += (double)joint_term(v, jm, jc);
+                    }
                 }
             }
             const unsigned bal = __ballot_sync(kFull, has);
@@ -2667,6 +2763,7 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
                 ub = SS::flags(lsp, left, SS::unit_cmp(tau_value(ws.tau)));
             }
             if (nonfin) ws.bad |= 1u;
+            if (jon) joint_stage<T>(lsp, left, lm, jc, jm, js);
             if (__any_sync(kFull, ub != 0u)) {
                 const uint32_t id0 = id_base + (uint32_t)(su + lane) * KPU;
                 const int nc = extract_fast<T>(ws.buf, ws.cnt, ub, lsp, ws.tau, id0, cap_w, lane);
@@ -2692,7 +2789,10 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
             ws.cnt = warp_keep_ge(ws.buf, ws.cnt, ws.tau, lane);
         }
         const uint32_t wb = __reduce_or_sync(kFull, ws.bad | (fail ? 2u : 0u));
+        if (jon) joint_warp_merge(jm, js, jc);
         if (lane == 0) {
+            P.jm[slot][c] = jm;
+            P.js[slot][c] = js;
             P.cnt[slot][c] = ws.cnt;
             if (wb) atomicOr(&P.bad[slot], wb);
             mbar_arrive(&P.slot_full[slot]);
@@ -2817,9 +2917,12 @@ struct Merged {
     int n;
     uint32_t rowbad;
     uint64_t spec;
+    float jm;  // joint order: the row's pair (m, s) from its pieces' pairs
+    double js;
 };
 __device__ __noinline__ Merged merge_pieces(const RowJob& J, int64_t T, int64_t G, int64_t nu, int64_t row,
-                                            int64_t first_cta, int np, uint64_t* sel, int lane) {
+                                            int64_t first_cta, int np, uint64_t* sel, int lane, bool jon,
+                                            JointScale jc) {
     CtaRange c;
     c.T = T;
     c.G = G;
@@ -2871,7 +2974,17 @@ __device__ __noinline__ Merged merge_pieces(const RowJob& J, int64_t T, int64_t 
     if (lane < n) sel[lane] = ~ra;
     if (lane + 32 < n) sel[lane + 32] = ~rb;
     __syncwarp();
-    return Merged{n, rowbad, sp};
+    float jm = kLowestFloat;
+    double js = 0.0;
+    if (jon) {
+        if (lane < np) {
+            const double2 v = __ldcg(J.part_ms + myslot);
+            jm = (float)v.x;
+            js = v.y;
+        }
+        joint_warp_merge(jm, js, jc);
+    }
+    return Merged{n, rowbad, sp, jm, js};
 }
 
 // The slot's per-piece state starts afresh for its next piece (one thread).
@@ -2885,7 +2998,7 @@ __device__ __forceinline__ void slot_reset(PipeShared& P, int slot) {
 }
 
 // Finishing warp f.
-template <typename T, int MODE>
+template <typename T, int MODE, int PR>
 __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slots, unsigned char* scratch, int f,
                             int lane) {
     uint64_t* sel = reinterpret_cast<uint64_t*>(scratch);            // [kPipeMaxK]
@@ -2916,6 +3029,15 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
         uint32_t rowbad = 2u;
         uint64_t spec = 0ull;
         int n = 0;
+        bool jon = false;  // joint order: the piece's and then the row's pair (m, s)
+        JointScale jc{0.0f, 0.0f};
+        if (PR && J.joint) {
+            const RowParams rp = row_params<MODE>(J, row);
+            jon = rp.ok && rp.T > 0.0f;
+            if (jon) jc = joint_scale(rp.T);
+        }
+        float jm = kLowestFloat;
+        double js = 0.0;
         const bool ok = pipe_wait_warp(&P.slot_full[slot], use & 1u, P);
         ++use;
         if (ok) {
@@ -2924,6 +3046,13 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
             const uint64_t tf = P.tau[slot];
             rowbad = P.bad[slot];
             spec = P.used[slot];
+            if (jon) {
+                if (lane < kPipeConsumers) {
+                    jm = P.jm[slot][lane];
+                    js = P.js[slot][lane];
+                }
+                joint_warp_merge(jm, js, jc);
+            }
             int U = 0;
             for (int w = 0; w < kPipeConsumers; ++w) {
                 const int cw = P.cnt[slot][w];
@@ -2987,6 +3116,7 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
                 J.part_count[ps] = n;
                 J.part_flags[ps] = rowbad;
                 J.part_spec[ps] = spec;
+                if (jon) J.part_ms[ps] = make_double2((double)jm, js);
                 __threadfence();
                 const uint32_t t = atomicAdd(J.row_ticket + p.first_cta, 1u);
                 last = (t == (uint32_t)(p.np - 1));
@@ -2997,10 +3127,12 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
             }
             last = __shfl_sync(kFull, last, 0);
             if (!last) continue;
-            const Merged m = merge_pieces(J, L.cr.T, L.cr.G, L.cr.nu, row, p.first_cta, p.np, sel, lane);
+            const Merged m = merge_pieces(J, L.cr.T, L.cr.G, L.cr.nu, row, p.first_cta, p.np, sel, lane, jon, jc);
             n = m.n;
             rowbad = m.rowbad;
             spec = m.spec;
+            jm = m.jm;
+            js = m.js;
         }
         // a predicted threshold holds when the row's k-th kept key reaches it:
         // then at least k elements of the row do, and none of the top k was
@@ -3026,11 +3158,14 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
             __syncwarp();
             continue;
         }
-        finish_row_warp<MODE>(J, row, req, n, rowbad, sel, wd, tail, unused_fs, lane, gat);
+        const double2 jms = make_double2((double)jm, js);
+        finish_row_warp<MODE, PR>(J, row, req, n, rowbad, sel, wd, tail, unused_fs, lane, gat, &jms);
     }
 }
 
-template <typename T, int MODE>
+// PR: 1 when the call has per-request parameters (and may use the joint
+// order), 0 for the call's scalar parameters, which compiles neither in.
+template <typename T, int MODE, int PR>
 __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_constant__ RowJob J) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ PipeShared P;
@@ -3065,10 +3200,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_cons
     if (warp == 0) {
         if (lane == 0) pipe_produce<T, MODE>(J, P, ring);
     } else if (warp <= kPipeConsumers) {
-        pipe_consume<T, MODE>(J, P, ring, slots, warp - 1, lane);
+        pipe_consume<T, MODE, PR>(J, P, ring, slots, warp - 1, lane);
     } else {
         const int f = warp - 1 - kPipeConsumers;
-        pipe_finish<T, MODE>(J, P, slots, fin + (size_t)f * J.fin_stride, f, lane);
+        pipe_finish<T, MODE, PR>(J, P, slots, fin + (size_t)f * J.fin_stride, f, lane);
     }
     // carry this CTA's latest prediction to the next call (a hint only: the
     // rows it predicts are checked exactly)
@@ -3112,35 +3247,6 @@ __global__ void __launch_bounds__(32 * kTailWarps) tail_kernel(const __grid_cons
 // a unit's terms are added in float, units in double.
 // ---------------------------------------------------------------------------
 constexpr int kJointThreads = 256;
-
-struct JointScale {
-    float hi, lo;
-};
-__device__ __forceinline__ JointScale joint_scale(float T) {
-    const double c = 1.4426950408889634 / (double)T;  // log2(e) / T
-    JointScale k;
-    k.hi = (float)c;
-    k.lo = (float)(c - (double)k.hi);
-    return k;
-}
-__device__ __forceinline__ float joint_term(float v, float m, JointScale c) {
-    const float d = v - m;
-    return exp2f(fmaf(d, c.hi, d * c.lo));
-}
-// (m, s) with s relative to m: raise m to at least x, rescaling s
-__device__ __forceinline__ void joint_raise(float& m, double& s, float x, JointScale c) {
-    if (x > m) {
-        const double d = (double)m - (double)x;
-        s *= exp2(d * ((double)c.hi + (double)c.lo));
-        m = x;
-    }
-}
-__device__ __forceinline__ void joint_merge(float& m, double& s, float m2, double s2, JointScale c) {
-    const float M = m > m2 ? m : m2;
-    const double cc = (double)c.hi + (double)c.lo;
-    s = s * exp2(((double)m - (double)M) * cc) + s2 * exp2(((double)m2 - (double)M) * cc);
-    m = M;
-}
 
 template <typename T, int MODE>
 __global__ void __launch_bounds__(kJointThreads) joint_norm_kernel(const __grid_constant__ RowJob J) {
@@ -3415,8 +3521,8 @@ constexpr int64_t kCounterWords = UNO_WORKSPACE_COUNTER_BYTES / 4;
 constexpr int64_t kRowCounterWords = kCounterWords / 2;
 
 struct WsLayout {
-    size_t row_ticket, req_ticket, part_keys, part_count, part_flags, part_spec, redo, row_ms, c_ids, c_probs,
-        c_count, c_flags, total;
+    size_t row_ticket, req_ticket, part_keys, part_count, part_flags, part_spec, part_ms, redo, row_ms, c_ids,
+        c_probs, c_count, c_flags, total;
 };
 
 static WsLayout ws_layout(int64_t rows, int32_t k, bool compact) {
@@ -3437,6 +3543,8 @@ static WsLayout ws_layout(int64_t rows, int32_t k, bool compact) {
     off = align_up(off + nslot * 4, 256);
     L.part_spec = off;
     off = align_up(off + nslot * 8, 256);
+    L.part_ms = off;
+    off = align_up(off + nslot * 16, 256);
     L.redo = off;
     off = align_up(off + ((size_t)rows + kPipeMaxGrid) * 4, 256);
     L.row_ms = off;
@@ -3555,7 +3663,7 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     J.fin_stride = (int32_t)stride_of(0);
     J.defer_tails = 1;
     const size_t dyn = (size_t)nst * kPStageBytes + slot_bytes + (size_t)kPipeFinishers * J.fin_stride;
-    auto kern = pipe_kernel<T, MODE>;
+    auto kern = J.rq_T != nullptr ? pipe_kernel<T, MODE, 1> : pipe_kernel<T, MODE, 0>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) != cudaSuccess)
         return UNO_ERR_CUDA;
     if (grid <= 0) return UNO_OK;
@@ -3578,12 +3686,14 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
 
 template <typename T, int MODE>
 static uno_status launch_rows(RowJob J, cudaStream_t stream) {
-    const uno_status sj = launch_joint<T, MODE>(J, stream);
-    if (sj != UNO_OK) return sj;
+    // the pipelined kernel forms the joint order's normalisers as it reads
+    // the rows; the general one takes them from a pass of their own
     if (J.k <= kPipeMaxK && J.out_dense == nullptr) {
         const uno_status st = launch_pipe<T, MODE>(J, stream);
         if (st != UNO_ERR_UNSUPPORTED) return st;
     }
+    const uno_status sj = launch_joint<T, MODE>(J, stream);
+    if (sj != UNO_OK) return sj;
     // warp buffer: high-water mark, plus room for one piece of appends from
     // every lane; it also holds the threshold seed (2 keys per thread)
     J.hw = J.k + 16 > 64 ? J.k + 16 : 64;
@@ -3630,6 +3740,7 @@ static void bind_workspace(RowJob& J, void* ws, const WsLayout& L) {
     J.part_count = reinterpret_cast<int32_t*>(b + L.part_count);
     J.part_flags = reinterpret_cast<uint32_t*>(b + L.part_flags);
     J.part_spec = reinterpret_cast<uint64_t*>(b + L.part_spec);
+    J.part_ms = reinterpret_cast<double2*>(b + L.part_ms);
     J.redo = reinterpret_cast<int32_t*>(b + L.redo);
     J.row_ms = reinterpret_cast<double2*>(b + L.row_ms);
     J.hint = reinterpret_cast<uint64_t*>(b + UNO_WORKSPACE_COUNTER_BYTES);
@@ -3874,10 +3985,8 @@ static uno_status linear_cycle_impl(const void* draft_logits, const void* target
         J.nq2 = nq;
         J.rows = nq + np;
         J.rpr = B;
-        uno_status st = dt == UNO_BF16 ? launch_joint<__nv_bfloat16, kModeCycle>(J, s)
-                                       : launch_joint<float, kModeCycle>(J, s);
-        if (st != UNO_OK) return st;
-        st = dt == UNO_BF16 ? launch_pipe<__nv_bfloat16, kModeCycle>(J, s) : launch_pipe<float, kModeCycle>(J, s);
+        const uno_status st = dt == UNO_BF16 ? launch_pipe<__nv_bfloat16, kModeCycle>(J, s)
+                                             : launch_pipe<float, kModeCycle>(J, s);
         if (st != UNO_ERR_UNSUPPORTED) return st;
     }
     // the draft rows, then the target rows with the request tails
