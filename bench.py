@@ -393,6 +393,33 @@ def tree_leg(index, device, first, stream, peak, reps, cpu_budget):
                              "sample": f"{done} requests, {spent:.1f} s, single-threaded C oracle"}}
 
 
+def params_leg(q, p, w, first, stream, peak, reps):
+    """uno_linear_cycle_params over the headline batch: per-request arrays
+    (each request's own entries, here the workload's values), in the
+    top-k-first and in the joint filter order, one graph replay per cycle."""
+    import torch
+    from speculative_decoding_verification_filter_b200 import uno_linear_cycle_params
+    dev = q.device
+    T = torch.full((w.R,), w.temperature, dtype=torch.float32, device=dev)
+    K = torch.full((w.R,), w.top_k, dtype=torch.int32, device=dev)
+    P = torch.full((w.R,), w.top_p, dtype=torch.float32, device=dev)
+    nbytes = (q.shape[0] + p.shape[0]) * w.vocab * w.elem_bytes
+    out = {}
+    for order in ("topk_first", "joint"):
+        g = graph_of(lambda st, order=order: uno_linear_cycle_params(
+            q, p, R=w.R, B=w.B, temperature=T, top_k=K, top_p=P, rng=(w.seed, 0, first), order=order,
+            top_k_max=w.top_k), stream)
+        ms = replay_ms(g, stream, reps)
+        del g
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[order] = {"ms_per_cycle": ms, "value": w.R / (ms / 1e3), "unit": UNIT,
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                                   "bytes_per_cycle": nbytes}}
+    out["note"] = ("uno_linear_cycle_params, CUDA events around graph replays; the joint order also forms every "
+                   "row's sum of exp over the full vocabulary while it reads the row")
+    return out
+
+
 def stress_leg(device, first, stream, peak, reps, cpu_budget):
     """The linear stress workload (512 requests, B = 16, fp32, T = 0.7): one
     uno_linear_cycle per replay.  Its 10.3 GB of logits are drawn on the GPU
@@ -598,6 +625,7 @@ def run_ours(args, w):
         "clocks": dict(clocks, note="NVML every 1 ms over the timed steps and 100 ms more of the same replays"),
     }
     if not args.no_tree:
+        line["per_request"] = params_leg(q, p, w, first, stream, peak, max(10, min(K, 100)))
         line["tree_16_32_32"] = tree_leg(2, device, first, stream, peak, 200, 3.0)
         line["tree_8_16_8"] = tree_leg(3, device, rank * 64, stream, peak, 100, 3.0)
         line["stress"] = stress_leg(device, first, stream, peak, 10, 4.0)

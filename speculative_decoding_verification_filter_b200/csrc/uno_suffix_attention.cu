@@ -175,6 +175,321 @@ __global__ void __launch_bounds__(32 * kWarps) suffix_attention_kernel(const __g
     }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core form: bf16 inputs, d a multiple of 16 up to 256.
+//
+// One CTA of four warps per (request, key/value head, tile of 128 stacked
+// rows).  The rows of a tile are (query head, node) pairs of the G query
+// heads that read this key/value head, row m = hl * V + j, so the G heads
+// share one K and one V and the contraction has M = 128 (G = 4 heads of a
+// V = 32 tree fill one tile exactly).
+// - Staging: the tile's Q rows, the head's K rows and V transposed go to
+//   shared memory in the tensor cores' K-major layout without swizzle: core
+//   matrices of 8 rows x 16 bytes, the 16-byte chunks of a core matrix's
+//   rows adjacent, core matrices along K 128 bytes apart (LBO) and groups of
+//   8 rows 16 K bytes apart (SBO).  Nodes are padded to Np = V rounded up
+//   to 16 with zeros.
+// - S = Q K^T: one thread issues tcgen05.mma (kind::f16, bf16 in, f32
+//   accumulate; M = 128, N = Np, d / 16 steps of K = 16) into TMEM columns
+//   [0, Np); tcgen05.commit signals an mbarrier.
+// - Thread t owns TMEM lane t, i.e. row t of the tile: it reads its row of S
+//   (tcgen05.ld), applies the ancestor mask, takes the maximum and the sum
+//   of exp, and writes its unnormalised weights P to shared memory as three
+//   bf16 parts (hi + mid + lo carry P to a relative 2^-24, so the second
+//   contraction is as accurate as one in binary32).
+// - O = P V: three accumulating chains of tcgen05.mma (M = 128, N = d,
+//   K = Np) into TMEM columns [128, 128 + d).
+// - Epilogue: each thread reads its row of O, divides by the sum and merges
+//   with the prefix state.
+// Every wait on the mbarrier is bounded; on expiry the request is flagged
+// UNO_FLAG_TIMEOUT, and the TMEM is freed after a second bounded wait.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+constexpr int kTcRows = 128;
+constexpr int kTcThreads = 128;
+constexpr uint32_t kTcColO = 128;  // TMEM column of O
+constexpr uint32_t kTcMaxTries = 1u << 22;
+
+// byte offset of bf16 element (row, k) of a K-major operand whose rows hold K elements
+__device__ __forceinline__ uint32_t kmajor_off(int row, int k, int K) {
+    return (uint32_t)((row >> 3) * (K * 16) + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
+}
+// shared-memory matrix descriptor of such an operand starting at `addr`:
+// start >> 4 in bits 0-13, LBO = 128 B in bits 16-29, SBO = 16 K bytes in
+// bits 32-45, descriptor version 1 in bits 46-47, no swizzle (bits 61-63 = 0)
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr, int K) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)(128u >> 4) << 16) |
+           ((uint64_t)(((uint32_t)K * 16u >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// instruction descriptor, kind::f16: f32 accumulator (bits 4-5 = 1), bf16 A
+// and B (bits 7-9 = 1, 10-12 = 1), both K-major, N >> 3 in bits 17-22,
+// M >> 4 in bits 24-28
+__device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+// 16 consecutive f32 columns of this thread's TMEM lane (warp-collective)
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t x[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7]),
+          "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]), "=r"(x[13]), "=r"(x[14]), "=r"(x[15])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(x[i]);
+}
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
+    for (uint32_t it = 0; it < kTcMaxTries; ++it)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+
+// shared-memory bytes of the tensor-core form (0: it does not apply)
+__host__ __device__ inline size_t tc_smem_bytes(int V, int d) {
+    const int Np = (V + 15) / 16 * 16;
+    return (size_t)kTcRows * d * 2 + (size_t)Np * d * 2 * 2 + (size_t)3 * kTcRows * Np * 2 +
+           (size_t)V * kMaskWords * 4;
+}
+
+__global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const __grid_constant__ Job J) {
+    extern __shared__ __align__(1024) unsigned char sm[];
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tmem_base;
+    __shared__ int s_bad;
+    const int r = blockIdx.x, g = blockIdx.y, m0 = blockIdx.z * kTcRows;
+    const int V = J.V, d = J.d, G = J.G, rows = G * V;
+    const int Np = (V + 15) / 16 * 16;
+    unsigned char* sQ = sm;                                   // [128][d]
+    unsigned char* sK = sQ + (size_t)kTcRows * d * 2;         // [Np][d]
+    unsigned char* sVt = sK + (size_t)Np * d * 2;             // [d][Np]
+    unsigned char* sP = sVt + (size_t)d * Np * 2;             // 3 x [128][Np]
+    uint32_t* anc = reinterpret_cast<uint32_t*>(sP + (size_t)3 * kTcRows * Np * 2);  // [V][kMaskWords]
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t ncols = kTcColO + (uint32_t)d <= 256u ? 256u : 512u;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&tmem_base)),
+                     "r"(ncols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    int n = J.num_nodes[r];
+    n = n < 1 ? 1 : (n > V ? V : n);
+
+    // staging: one 16-byte chunk (8 elements) per thread and step
+    const int cpr = d >> 3;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    for (int e = tid; e < kTcRows * cpr; e += kTcThreads) {
+        const int ml = e / cpr, c = e - ml * cpr, m = m0 + ml;
+        uint4 x = zero;
+        if (m < rows) {
+            const int hl = m / V, j = m - hl * V;
+            if (j < n) {
+                const size_t row = ((size_t)r * V + j) * J.H + (size_t)g * G + hl;
+                x = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.q) + row * d) + c);
+            }
+        }
+        *reinterpret_cast<uint4*>(sQ + kmajor_off(ml, c * 8, d)) = x;
+    }
+    for (int e = tid; e < Np * cpr; e += kTcThreads) {
+        const int i = e / cpr, c = e - i * cpr;
+        uint4 kx = zero, vx = zero;
+        if (i < n) {
+            const size_t src = (((size_t)r * V + i) * J.Hkv + g) * d;
+            kx = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.k) + src) + c);
+            vx = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.v) + src) + c);
+        }
+        *reinterpret_cast<uint4*>(sK + kmajor_off(i, c * 8, d)) = kx;
+        const uint32_t w[4] = {vx.x, vx.y, vx.z, vx.w};
+#pragma unroll
+        for (int q = 0; q < 8; ++q)  // V^T: element (column t of V, node i)
+            *reinterpret_cast<uint16_t*>(sVt + kmajor_off(c * 8 + q, i, Np)) =
+                (uint16_t)((q & 1) ? (w[q >> 1] >> 16) : (w[q >> 1] & 0xffffu));
+    }
+    if (tid == 0) {
+        const int32_t* par = J.parent + (size_t)r * V;
+        int bad = 0;
+        for (int j = 0; j < n; ++j) {
+            const int p = par[j];
+            const bool ok = j == 0 ? p == -1 : (p >= 0 && p < j);
+            uint32_t* a = anc + j * kMaskWords;
+            for (int w2 = 0; w2 < kMaskWords; ++w2) a[w2] = (ok && j > 0) ? anc[p * kMaskWords + w2] : 0u;
+            a[j >> 5] |= 1u << (j & 31);
+            bad |= ok ? 0 : 1;
+        }
+        s_bad = bad;
+    }
+    fence_proxy_async();  // the staged operands, for the tensor cores
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tb = tmem_base;
+
+    // S = Q K^T
+    if (tid == 0) {
+        const uint32_t id1 = idesc_bf16(kTcRows, Np), aq = smem_u32(sQ), ak = smem_u32(sK);
+        for (int s = 0; s < d / 16; ++s)
+            tc_mma(tb, kmajor_desc(aq + 256u * s, d), kmajor_desc(ak + 256u * s, d), id1, s > 0 ? 1u : 0u);
+        tc_commit(&bar);
+    }
+    bool ok = tc_wait(&bar, 0);
+    tc_fence_after();
+
+    // this thread's row: masked softmax statistics and the weights P
+    const int ml = tid, m = m0 + ml;
+    const int hl = m / V, j = m - hl * V;
+    const bool live = m < rows && j < n;
+    const uint32_t lane_addr = tb + ((uint32_t)(warp * 32) << 16);
+    const uint32_t* a = anc + (live ? j : 0) * kMaskWords;
+    float mx = -INFINITY;
+    for (int c0 = 0; c0 < Np; c0 += 16) {
+        float sv[16];
+        tc_ld16(lane_addr + (uint32_t)c0, sv);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const int i = c0 + q;
+            if (live && i < n && ((a[i >> 5] >> (i & 31)) & 1u)) mx = fmaxf(mx, sv[q] * J.scale);
+        }
+    }
+    float sum = 0.0f;
+    for (int c0 = 0; c0 < Np; c0 += 16) {
+        float sv[16];
+        tc_ld16(lane_addr + (uint32_t)c0, sv);
+        uint32_t part[3][8];
+#pragma unroll
+        for (int q = 0; q < 16; q += 2) {
+            float pr[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int i = c0 + q + h;
+                pr[h] = (live && i < n && ((a[i >> 5] >> (i & 31)) & 1u)) ? expf(sv[q + h] * J.scale - mx) : 0.0f;
+                sum += pr[h];
+            }
+            // three bf16 parts of each weight
+            float r0 = pr[0], r1 = pr[1];
+#pragma unroll
+            for (int t = 0; t < 3; ++t) {
+                const uint32_t b0 = bf16_bits(r0), b1 = bf16_bits(r1);
+                part[t][q >> 1] = b0 | (b1 << 16);
+                r0 -= __uint_as_float(b0 << 16);
+                r1 -= __uint_as_float(b1 << 16);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+            unsigned char* base = sP + (size_t)t * kTcRows * Np * 2;
+            *reinterpret_cast<uint4*>(base + kmajor_off(ml, c0, Np)) =
+                make_uint4(part[t][0], part[t][1], part[t][2], part[t][3]);
+            *reinterpret_cast<uint4*>(base + kmajor_off(ml, c0 + 8, Np)) =
+                make_uint4(part[t][4], part[t][5], part[t][6], part[t][7]);
+        }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // O = P V, three accumulating parts
+    if (tid == 0) {
+        const uint32_t id2 = idesc_bf16(kTcRows, d), av = smem_u32(sVt);
+        uint32_t acc = 0u;
+        for (int t = 0; t < 3; ++t) {
+            const uint32_t ap = smem_u32(sP + (size_t)t * kTcRows * Np * 2);
+            for (int s = 0; s < Np / 16; ++s) {
+                tc_mma(tb + kTcColO, kmajor_desc(ap + 256u * s, Np), kmajor_desc(av + 256u * s, Np), id2, acc);
+                acc = 1u;
+            }
+        }
+        tc_commit(&bar);
+    }
+    ok = tc_wait(&bar, 1) && ok;
+    tc_fence_after();
+
+    // epilogue: the suffix state merged with the prefix state
+    const size_t orow = live ? ((size_t)r * V + j) * J.H + (size_t)g * G + hl : 0;
+    const float lse_s = mx + logf(sum);
+    float w1 = 0.0f, w2 = 1.0f, M = lse_s;
+    if (live) {
+        const float lp = J.lse_prefix[orow];
+        const bool has_prefix = lp != -INFINITY;
+        M = has_prefix ? fmaxf(lp, lse_s) : lse_s;
+        w1 = has_prefix ? expf(lp - M) : 0.0f;
+        w2 = expf(lse_s - M);
+    }
+    const float inv = 1.0f / (w1 + w2), inv_sum = 1.0f / sum;
+    for (int c0 = 0; c0 < d; c0 += 16) {
+        float ov[16];
+        tc_ld16(lane_addr + kTcColO + (uint32_t)c0, ov);
+        if (live) {
+            const float4* op = reinterpret_cast<const float4*>(J.o_prefix + orow * d + c0);
+            float4* out = reinterpret_cast<float4*>(J.out_o + orow * d + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 pv = w1 != 0.0f ? op[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+                float4 o;
+                o.x = (w1 * pv.x + w2 * (ov[4 * q + 0] * inv_sum)) * inv;
+                o.y = (w1 * pv.y + w2 * (ov[4 * q + 1] * inv_sum)) * inv;
+                o.z = (w1 * pv.z + w2 * (ov[4 * q + 2] * inv_sum)) * inv;
+                o.w = (w1 * pv.w + w2 * (ov[4 * q + 3] * inv_sum)) * inv;
+                out[q] = o;
+            }
+        }
+    }
+    if (live) J.out_lse[orow] = M + logf(w1 + w2);
+    if (m < rows && !live) {  // nodes past num_nodes: o = 0, lse = -inf
+        const size_t prow = ((size_t)r * V + j) * J.H + (size_t)g * G + hl;
+        for (int t = 0; t < d; ++t) J.out_o[prow * d + t] = 0.0f;
+        J.out_lse[prow] = -INFINITY;
+    }
+    if (tid == 0 && g == 0 && blockIdx.z == 0 && J.out_flags != nullptr)
+        J.out_flags[r] = (s_bad ? UNO_FLAG_BAD_TREE : 0u) | (ok ? 0u : UNO_FLAG_TIMEOUT);
+    if (!ok) tc_wait(&bar, 1);  // a second bounded wait before the TMEM is freed
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tb), "r"(ncols) : "memory");
+}
+
 }  // namespace uno_sa
 
 extern "C" uno_status uno_tree_suffix_attention_merge(const void* q, const void* k, const void* v, uno_dtype dt,
@@ -197,8 +512,12 @@ extern "C" uno_status uno_tree_suffix_attention_merge(const void* q, const void*
         !aligned(node_parent, 4) || !aligned(num_nodes, 4) || (out_flags && !aligned(out_flags, 4)))
         return UNO_ERR_INVALID_ARG;
     if (d > kMaxD) return UNO_ERR_UNSUPPORTED;
+    // bf16 rows with d a multiple of 16 take the tensor cores; the rest the
+    // CUDA-core kernel
+    const size_t tc_smem = tc_smem_bytes(V, d);
+    const bool tc = dt == UNO_BF16 && d % 16 == 0 && tc_smem <= 200 * 1024;
     const size_t smem = ((size_t)2 * V * (d + 1) + (size_t)kWarps * d) * 4 + (size_t)V * kMaskWords * 4;
-    if (smem > 227 * 1024) return UNO_ERR_UNSUPPORTED;
+    if (!tc && smem > 227 * 1024) return UNO_ERR_UNSUPPORTED;
     Job J{};
     J.q = q;
     J.k = k;
@@ -218,6 +537,16 @@ extern "C" uno_status uno_tree_suffix_attention_merge(const void* q, const void*
     J.out_o = out_o;
     J.out_lse = out_lse;
     J.out_flags = out_flags;
+    if (tc) {
+        if (tc_smem > 48 * 1024 &&
+            cudaFuncSetAttribute(suffix_attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tc_smem) != cudaSuccess)
+            return UNO_ERR_CUDA;
+        const int tiles = (J.G * V + kTcRows - 1) / kTcRows;
+        suffix_attention_tc_kernel<<<dim3((unsigned)R, (unsigned)Hkv, (unsigned)tiles), kTcThreads, tc_smem,
+                                     static_cast<cudaStream_t>(stream)>>>(J);
+        return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
+    }
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(suffix_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess)

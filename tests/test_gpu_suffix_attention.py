@@ -99,3 +99,18 @@ def test_bad_tree_is_flagged_and_confined_to_its_request():
     dev["node_parent"] = parent
     _, _, flags = _check(dev, host, scale, skip=(1,))
     assert flags[1] == FLAG_BAD_TREE
+
+
+# bf16 rows with d a multiple of 16 take the tensor-core kernel: stacked rows
+# G * V spanning several 128-row tiles, V not a multiple of 16, head dims 32
+# to 256, the largest tree, and padding past num_nodes
+@pytest.mark.parametrize("R,V,H,Hkv,d,L,seed,kw", [
+    (2, 40, 16, 2, 32, 12, 11, {}),
+    (3, 20, 8, 1, 256, 30, 12, dict(num_nodes=[20, 7, 13])),
+    (2, 128, 4, 4, 64, 5, 13, dict(chain=True)),
+    (2, 128, 2, 1, 64, 9, 14, {}),
+    (5, 3, 4, 4, 16, 0, 15, dict(empty_prefix=(0, 1, 2, 3, 4))),
+])
+def test_tensor_core_shapes(R, V, H, Hkv, d, L, seed, kw):
+    dev, host, scale = _case(R, V, H, Hkv, d, L, seed, "bf16", **kw)
+    _check(dev, host, scale)
