@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-tree", action="store_true", help="skip the other workloads' timings")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle time budget of the cpu_baseline")
+    ap.add_argument("--only", choices=["suffix_attention"], default=None,
+                    help="run one side measurement alone and print its JSON")
     return ap.parse_args()
 
 
@@ -420,6 +422,48 @@ def params_leg(q, p, w, first, stream, peak, reps):
     return out
 
 
+def suffix_attention_leg(device, stream, peak, reps=50):
+    """uno_tree_suffix_attention_merge at the attention shape of an 8B model
+    (32 query heads over 8 key/value heads, head dim 128, a 32-node binary
+    tree, bf16 q/k/v, f32 prefix state), 1 and 64 requests; each launch timed
+    alone with CUDA events, the L2 rewritten (256 MB) before it."""
+    import torch
+    from speculative_decoding_verification_filter_b200 import uno_tree_suffix_attention_merge
+    V, H, Hkv, d = 32, 32, 8, 128
+    junk = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    out = {}
+    for R in (1, 64):
+        g = torch.Generator(device=device)
+        g.manual_seed(1000 + R)
+        q = torch.randn((R, V, H, d), generator=g, device=device).to(torch.bfloat16)
+        k = torch.randn((R, V, Hkv, d), generator=g, device=device).to(torch.bfloat16)
+        v = torch.randn((R, V, Hkv, d), generator=g, device=device).to(torch.bfloat16)
+        par = torch.tensor([-1] + [j // 2 for j in range(1, V)], dtype=torch.int32, device=device).repeat(R, 1)
+        nn = torch.full((R,), V, dtype=torch.int32, device=device)
+        op = torch.randn((R, V, H, d), generator=g, device=device)
+        lp = torch.randn((R, V, H), generator=g, device=device)
+        nbytes = q.numel() * 2 + 2 * k.numel() * 2 + 2 * (op.numel() + lp.numel()) * 4
+        ts = []
+        with torch.cuda.stream(stream):
+            for i in range(reps + 3):
+                junk.fill_(1)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                uno_tree_suffix_attention_merge(q, k, v, par, nn, op, lp, scale=d ** -0.5)
+                b.record(stream)
+                if i >= 3:
+                    ts.append((a, b))
+        stream.synchronize()
+        us = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e3
+        gbs = nbytes / us / 1e3
+        out[f"requests_{R}"] = {"us": us, "bytes": nbytes,
+                                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                                             "frac": gbs / peak}}
+    out["note"] = ("tcgen05 tensor-core kernel (bf16 rows, d a multiple of 16); bound by latency at these sizes; "
+                   "median of one-launch CUDA-event times, L2 rewritten before each launch")
+    return out
+
+
 def stress_leg(device, first, stream, peak, reps, cpu_budget):
     """The linear stress workload (512 requests, B = 16, fp32, T = 0.7): one
     uno_linear_cycle per replay.  Its 10.3 GB of logits are drawn on the GPU
@@ -629,6 +673,7 @@ def run_ours(args, w):
         line["tree_16_32_32"] = tree_leg(2, device, first, stream, peak, 200, 3.0)
         line["tree_8_16_8"] = tree_leg(3, device, rank * 64, stream, peak, 100, 3.0)
         line["stress"] = stress_leg(device, first, stream, peak, 10, 4.0)
+        line["suffix_attention_8b"] = suffix_attention_leg(device, stream, peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if rank == 0:
@@ -641,6 +686,12 @@ def run_ours(args, w):
 
 def main():
     args = parse()
+    if args.only == "suffix_attention":
+        import torch
+        device = torch.device("cuda", 0)
+        peak, _ = hbm_peak()
+        print(json.dumps(suffix_attention_leg(device, torch.cuda.Stream(device), peak, reps=10)), flush=True)
+        return
     from speculative_decoding_verification_filter_b200.inputs import WORKLOADS
     w = WORKLOADS[args.workload]
     if w.mode != "linear":
