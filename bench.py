@@ -167,11 +167,21 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(text):
+    """C/CUDA source without its comments and blank lines (a comment edit
+    leaves the kernels, and so their counters, unchanged)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash():
+    """Hash of the row kernels' code (comments and blank lines left out)."""
     h = hashlib.sha256()
     for rel in ("speculative_decoding_verification_filter_b200/csrc/uno_filter.cu",
                 "speculative_decoding_verification_filter_b200/csrc/uno_device.cuh"):
-        h.update((ROOT / rel).read_bytes())
+        h.update(_code_only((ROOT / rel).read_text()).encode())
     return h.hexdigest()[:16]
 
 

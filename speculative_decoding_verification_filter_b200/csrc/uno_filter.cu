@@ -1841,17 +1841,22 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const __grid_constant_
 //     The k-th largest of any set of disjoint group maxima of a row is at
 //     most the row's k-th largest element, so this loses nothing.  A CTA's
 //     first piece runs this way.
-//   * predicted: the piece is filtered by a threshold taken from an earlier
-//     piece of the same CTA (a value that about 2k elements of that piece
-//     reached, from the maxima of its 1024-element groups), with no waiting.
-//     Decoding cycles give rows of one distribution, so the prediction holds
-//     almost always; it is checked exactly: the row's k-th kept key must be
-//     at or above every threshold its pieces used, which means at least k
-//     elements of the row reach them and nothing of the top k was dropped.
-//     A row that fails the check is re-read whole, in boot mode, at the end
-//     of the CTA's list (the redo pass), before the kernel exits.
-// At the end of a piece its final threshold, the k-th largest of its group
-// maxima, is what the finisher gathers by, so the finisher sorts about k keys.
+//   * predicted: the piece is filtered by the CTA's latest prediction, with
+//     no waiting: a value that about 2.5 k elements of a row reach,
+//     extrapolated from the k/2-th and k-th values of the last finished row
+//     of the same row set (or, at the start, the prediction the CTA left in
+//     the workspace at the end of the previous call).  The first consumer to
+//     start a piece fixes its mode.  Decoding cycles give rows of one
+//     distribution, so the prediction holds almost always; it is checked
+//     exactly: the row's k-th kept key must be at or above every threshold
+//     its pieces used, which means at least k elements of the row reach them
+//     and nothing of the top k was dropped.  A row that fails the check is
+//     re-read whole, in boot mode, at the end of the CTA's list (the redo
+//     pass), before the kernel exits.
+// Consumers raise the piece's threshold as their candidate buffers fill (a
+// buffer over its high-water mark is cut to its k best), and the finisher
+// gathers by the highest threshold any of them posted, so it sorts about k
+// keys.
 //
 // Every wait is bounded; a wait that gives up sets the CTA's abort word,
 // every role stops at its next check, and rows that were not finished are

@@ -224,6 +224,7 @@ constexpr int kTcRows = 128;
 constexpr int kTcThreads = 128;
 constexpr uint32_t kTcColO = 128;  // TMEM column of O
 constexpr uint32_t kTcMaxTries = 1u << 22;
+constexpr int kTcBatch = 8;  // staging loads in flight per thread
 
 // byte offset of bf16 element (row, k) of a K-major operand whose rows hold K elements
 __device__ __forceinline__ uint32_t kmajor_off(int row, int k, int K) {
@@ -280,10 +281,15 @@ __device__ __forceinline__ uint32_t bf16_bits(float x) {
 }
 
 // shared-memory bytes of the tensor-core form (0: it does not apply)
+// (the epilogue's O blocks of 128 x (cb + 4) floats reuse the operand area
+// and the ancestor masks)
 __host__ __device__ inline size_t tc_smem_bytes(int V, int d) {
     const int Np = (V + 15) / 16 * 16;
-    return (size_t)kTcRows * d * 2 + (size_t)Np * d * 2 * 2 + (size_t)3 * kTcRows * Np * 2 +
-           (size_t)V * kMaskWords * 4;
+    const size_t ops = (size_t)kTcRows * d * 2 + (size_t)Np * d * 2 * 2 + (size_t)3 * kTcRows * Np * 2 +
+                       (size_t)V * kMaskWords * 4;
+    const int cb = d < 64 ? d : 64;
+    const size_t out = (size_t)kTcRows * (cb + 4) * 4;
+    return ops > out ? ops : out;
 }
 
 __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const __grid_constant__ Job J) {
@@ -316,35 +322,53 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
     int n = J.num_nodes[r];
     n = n < 1 ? 1 : (n > V ? V : n);
 
-    // staging: one 16-byte chunk (8 elements) per thread and step
+    // staging: 16-byte chunks (8 elements), kTcBatch loads in flight per thread
     const int cpr = d >> 3;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    for (int e = tid; e < kTcRows * cpr; e += kTcThreads) {
-        const int ml = e / cpr, c = e - ml * cpr, m = m0 + ml;
-        uint4 x = zero;
-        if (m < rows) {
-            const int hl = m / V, j = m - hl * V;
-            if (j < n) {
-                const size_t row = ((size_t)r * V + j) * J.H + (size_t)g * G + hl;
-                x = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.q) + row * d) + c);
+    for (int e0 = tid; e0 < kTcRows * cpr; e0 += kTcThreads * kTcBatch) {
+        uint4 x[kTcBatch];
+#pragma unroll
+        for (int u = 0; u < kTcBatch; ++u) {
+            const int e = e0 + u * kTcThreads, ml = e / cpr, c = e - ml * cpr, m = m0 + ml;
+            x[u] = zero;
+            if (e < kTcRows * cpr && m < rows) {
+                const int hl = m / V, j = m - hl * V;
+                if (j < n) {
+                    const size_t row = ((size_t)r * V + j) * J.H + (size_t)g * G + hl;
+                    x[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.q) + row * d) + c);
+                }
             }
         }
-        *reinterpret_cast<uint4*>(sQ + kmajor_off(ml, c * 8, d)) = x;
-    }
-    for (int e = tid; e < Np * cpr; e += kTcThreads) {
-        const int i = e / cpr, c = e - i * cpr;
-        uint4 kx = zero, vx = zero;
-        if (i < n) {
-            const size_t src = (((size_t)r * V + i) * J.Hkv + g) * d;
-            kx = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.k) + src) + c);
-            vx = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.v) + src) + c);
-        }
-        *reinterpret_cast<uint4*>(sK + kmajor_off(i, c * 8, d)) = kx;
-        const uint32_t w[4] = {vx.x, vx.y, vx.z, vx.w};
 #pragma unroll
-        for (int q = 0; q < 8; ++q)  // V^T: element (column t of V, node i)
-            *reinterpret_cast<uint16_t*>(sVt + kmajor_off(c * 8 + q, i, Np)) =
-                (uint16_t)((q & 1) ? (w[q >> 1] >> 16) : (w[q >> 1] & 0xffffu));
+        for (int u = 0; u < kTcBatch; ++u) {
+            const int e = e0 + u * kTcThreads, ml = e / cpr, c = e - ml * cpr;
+            if (e < kTcRows * cpr) *reinterpret_cast<uint4*>(sQ + kmajor_off(ml, c * 8, d)) = x[u];
+        }
+    }
+    for (int e0 = tid; e0 < Np * cpr; e0 += kTcThreads * (kTcBatch / 2)) {
+        uint4 kx[kTcBatch / 2], vx[kTcBatch / 2];
+#pragma unroll
+        for (int u = 0; u < kTcBatch / 2; ++u) {
+            const int e = e0 + u * kTcThreads, i = e / cpr, c = e - i * cpr;
+            kx[u] = zero;
+            vx[u] = zero;
+            if (e < Np * cpr && i < n) {
+                const size_t src = (((size_t)r * V + i) * J.Hkv + g) * d;
+                kx[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.k) + src) + c);
+                vx[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.v) + src) + c);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kTcBatch / 2; ++u) {
+            const int e = e0 + u * kTcThreads, i = e / cpr, c = e - i * cpr;
+            if (e >= Np * cpr) continue;
+            *reinterpret_cast<uint4*>(sK + kmajor_off(i, c * 8, d)) = kx[u];
+            const uint32_t w[4] = {vx[u].x, vx[u].y, vx[u].z, vx[u].w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q)  // V^T: element (column t of V, node i)
+                *reinterpret_cast<uint16_t*>(sVt + kmajor_off(c * 8 + q, i, Np)) =
+                    (uint16_t)((q & 1) ? (w[q >> 1] >> 16) : (w[q >> 1] & 0xffffu));
+        }
     }
     if (tid == 0) {
         const int32_t* par = J.parent + (size_t)r * V;
@@ -445,41 +469,75 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
     ok = tc_wait(&bar, 1) && ok;
     tc_fence_after();
 
-    // epilogue: the suffix state merged with the prefix state
-    const size_t orow = live ? ((size_t)r * V + j) * J.H + (size_t)g * G + hl : 0;
-    const float lse_s = mx + logf(sum);
-    float w1 = 0.0f, w2 = 1.0f, M = lse_s;
-    if (live) {
-        const float lp = J.lse_prefix[orow];
-        const bool has_prefix = lp != -INFINITY;
-        M = has_prefix ? fmaxf(lp, lse_s) : lse_s;
-        w1 = has_prefix ? expf(lp - M) : 0.0f;
-        w2 = expf(lse_s - M);
-    }
-    const float inv = 1.0f / (w1 + w2), inv_sum = 1.0f / sum;
-    for (int c0 = 0; c0 < d; c0 += 16) {
-        float ov[16];
-        tc_ld16(lane_addr + kTcColO + (uint32_t)c0, ov);
+    // epilogue: the suffix state merged with the prefix state.  The operand
+    // area is free now; O goes through it in blocks of cb columns so that the
+    // prefix reads and the output writes are whole rows per warp.
+    __shared__ float s_c1[kTcRows], s_c2[kTcRows];
+    __shared__ long long s_row[kTcRows];  // output row, -1: none; -2 - row: a node past num_nodes
+    {
+        const size_t orow = ((size_t)r * V + j) * J.H + (size_t)g * G + hl;
+        float c1 = 0.0f, c2 = 0.0f;
         if (live) {
-            const float4* op = reinterpret_cast<const float4*>(J.o_prefix + orow * d + c0);
-            float4* out = reinterpret_cast<float4*>(J.out_o + orow * d + c0);
+            const float lse_s = mx + logf(sum);
+            const float lp = J.lse_prefix[orow];
+            const bool has_prefix = lp != -INFINITY;
+            const float M = has_prefix ? fmaxf(lp, lse_s) : lse_s;
+            const float w1 = has_prefix ? expf(lp - M) : 0.0f;
+            const float w2 = expf(lse_s - M);
+            const float inv = 1.0f / (w1 + w2);
+            c1 = w1 * inv;
+            c2 = w2 * inv / sum;
+            J.out_lse[orow] = M + logf(w1 + w2);
+        } else if (m < rows) {
+            J.out_lse[orow] = -INFINITY;  // a node past num_nodes
+        }
+        s_c1[ml] = c1;
+        s_c2[ml] = c2;
+        s_row[ml] = live ? (long long)orow : (m < rows ? -2 - (long long)orow : -1);
+    }
+    const int cb = d < 64 ? d : 64, ld = cb + 4;
+    float* sO = reinterpret_cast<float*>(sm);  // [128][cb + 4]
+    for (int b0 = 0; b0 < d; b0 += cb) {
+        tc_fence_before();
+        __syncthreads();  // the operands (first block) or the previous block are consumed
+        for (int c0 = 0; c0 < cb; c0 += 16) {
+            float ov[16];
+            tc_ld16(lane_addr + kTcColO + (uint32_t)(b0 + c0), ov);
+            const float c2 = s_c2[ml];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float4 pv = w1 != 0.0f ? op[q] : make_float4(0.f, 0.f, 0.f, 0.f);
-                float4 o;
-                o.x = (w1 * pv.x + w2 * (ov[4 * q + 0] * inv_sum)) * inv;
-                o.y = (w1 * pv.y + w2 * (ov[4 * q + 1] * inv_sum)) * inv;
-                o.z = (w1 * pv.z + w2 * (ov[4 * q + 2] * inv_sum)) * inv;
-                o.w = (w1 * pv.w + w2 * (ov[4 * q + 3] * inv_sum)) * inv;
-                out[q] = o;
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<float4*>(sO + (size_t)ml * ld + c0 + 4 * q) =
+                    make_float4(ov[4 * q] * c2, ov[4 * q + 1] * c2, ov[4 * q + 2] * c2, ov[4 * q + 3] * c2);
+        }
+        __syncthreads();
+        const int f4 = cb >> 2;
+        for (int e0 = tid; e0 < kTcRows * f4; e0 += kTcThreads * 4) {
+            float4 pv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kTcThreads, row = e / f4, c4 = e - row * f4;
+                pv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (e < kTcRows * f4 && s_row[row] >= 0 && s_c1[row] != 0.0f)
+                    pv[u] = __ldg(reinterpret_cast<const float4*>(J.o_prefix + (size_t)s_row[row] * d + b0) + c4);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * kTcThreads, row = e / f4, c4 = e - row * f4;
+                if (e >= kTcRows * f4 || s_row[row] == -1) continue;
+                float4* out;
+                float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (s_row[row] >= 0) {
+                    const float c1 = s_c1[row];
+                    const float4 sv = *reinterpret_cast<const float4*>(sO + (size_t)row * ld + 4 * c4);
+                    o = make_float4(c1 * pv[u].x + sv.x, c1 * pv[u].y + sv.y, c1 * pv[u].z + sv.z,
+                                    c1 * pv[u].w + sv.w);
+                    out = reinterpret_cast<float4*>(J.out_o + (size_t)s_row[row] * d + b0) + c4;
+                } else {
+                    out = reinterpret_cast<float4*>(J.out_o + (size_t)(-2 - s_row[row]) * d + b0) + c4;
+                }
+                *out = o;
             }
         }
-    }
-    if (live) J.out_lse[orow] = M + logf(w1 + w2);
-    if (m < rows && !live) {  // nodes past num_nodes: o = 0, lse = -inf
-        const size_t prow = ((size_t)r * V + j) * J.H + (size_t)g * G + hl;
-        for (int t = 0; t < d; ++t) J.out_o[prow * d + t] = 0.0f;
-        J.out_lse[prow] = -INFINITY;
     }
     if (tid == 0 && g == 0 && blockIdx.z == 0 && J.out_flags != nullptr)
         J.out_flags[r] = (s_bad ? UNO_FLAG_BAD_TREE : 0u) | (ok ? 0u : UNO_FLAG_TIMEOUT);
