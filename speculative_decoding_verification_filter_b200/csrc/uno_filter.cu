@@ -78,6 +78,7 @@ struct RowJob {
     uint64_t* part_spec;   // pipelined kernel: the predicted threshold each piece used
     double2* part_ms;      // pipelined kernel, joint order: each piece's pair (m, s)
     int32_t* redo;         // pipelined kernel: rows each CTA reads again (rows + grid entries)
+    uint32_t* dyn;         // pipelined kernel: rows handed out at run time (nullable; see kDyn*)
     uint64_t* hint;        // pipelined kernel: per CTA, the prediction carried to the next call
     int32_t* c_ids;        // [rows][ks]  compact target rows (verifiers)
     float* c_probs;        // [rows][ks]
@@ -708,6 +709,10 @@ __device__ __forceinline__ double lookup_sorted(const int32_t* ids, const float*
     return 0.0;
 }
 
+// A compact row's count as the request tails use it: a value outside [0, k]
+// (only a row that was never written holds one) reads as an empty row.
+__device__ __forceinline__ int clamp_count(int c, int k) { return (c < 0 || c > k) ? 0 : c; }
+
 // Linear verification of request r from global memory (one warp): any k, any
 // B.  Generic layout (sh = 0): target row i tests proposal x_i, row B gives
 // the bonus.  Two-pass layout (sh = 1): x_0 is emitted untested, row i - 1
@@ -737,7 +742,7 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
         }
     }
     for (int i = sh; i < B && !stopped; ++i) {
-        const int pc = __ldcg(J.c_count + base + i - sh);
+        const int pc = clamp_count(__ldcg(J.c_count + base + i - sh), J.k);
         const int32_t* pid = J.c_ids + (size_t)(base + i - sh) * J.ks;
         const float* ppr = J.c_probs + (size_t)(base + i - sh) * J.ks;
         if (pc == 0) {
@@ -791,7 +796,7 @@ __device__ __noinline__ void linear_tail(const RowJob& J, int32_t r, double* wd,
         stopped = true;
     }
     if (!stopped) {
-        const int pc = __ldcg(J.c_count + base + B - sh);
+        const int pc = clamp_count(__ldcg(J.c_count + base + B - sh), J.k);
         if (pc == 0) {
             ntok = B;
         } else if (lane == 0) {
@@ -829,7 +834,7 @@ __device__ __noinline__ void tree_tail(const RowJob& J, int32_t r, double* wd, i
     __syncwarp();
     int32_t j = 0, t = 0, acc = 0, ntok = 0;
     for (;;) {
-        const int pc = __ldcg(J.c_count + base + j);
+        const int pc = clamp_count(__ldcg(J.c_count + base + j), J.k);
         if (pc == 0) {
             if (lane == 0) path[t] = j;
             ntok = t;
@@ -1099,7 +1104,7 @@ __device__ __noinline__ bool linear_tail_fast(const RowJob& J, int32_t r, unsign
     int pc_l = 0, qc_l = 0, d_l = 0;
     uint32_t f_l = 0;
     if (lane < P) {
-        pc_l = __ldcg(J.c_count + base + lane);
+        pc_l = clamp_count(__ldcg(J.c_count + base + lane), J.k);
         f_l = __ldcg(J.c_flags + base + lane);
     }
     if (lane < B) {
@@ -1246,7 +1251,7 @@ __device__ __noinline__ bool tree_tail_fast(const RowJob& J, int32_t r, unsigned
     }
     uint32_t flags = 0;
     for (int j = lane; j < n; j += 32) {
-        ncnt[j] = __ldcg(J.c_count + base + j);
+        ncnt[j] = clamp_count(__ldcg(J.c_count + base + j), J.k);
         flags |= __ldcg(J.c_flags + base + j);
         tk[j] = J.node_token[(size_t)r * V + j];
         pa[j] = J.node_parent[(size_t)r * V + j];
@@ -1864,6 +1869,17 @@ __global__ void __launch_bounds__(kThreads, 4) row_kernel(const __grid_constant_
 // ---------------------------------------------------------------------------
 constexpr int kPipeConsumers = 8;
 constexpr int kPipeFinishers = 2;
+// Rows handed out at run time: the producer of each CTA takes the next row
+// from a counter in the workspace and posts it in a queue that the CTA's
+// consumers and finishers read in order.  Counter words (zero between calls):
+constexpr int kDynNext = 0;      // next row
+constexpr int kDynDone = 1;      // CTAs that have exited
+constexpr int kDynRetryPut = 2;  // rows posted for a second read
+constexpr int kDynRetryGet = 3;  // of those, taken
+constexpr int kDynFinished = 4;  // rows finished
+constexpr int kDynWords = 8;     // then one word per posted retry (row + 1; 0 = not yet written)
+constexpr int kDynOffset = 1024; // counter words start here in the row-ticket area
+constexpr int kDynQ = 64;        // queue entries (the producer runs at most a few rows ahead)
 constexpr int kPipeSlots = kPipeFinishers;
 constexpr int kPipeWarps = 1 + kPipeConsumers + kPipeFinishers;
 constexpr int kPipeThreads = 32 * kPipeWarps;
@@ -1906,6 +1922,8 @@ struct __align__(16) PipeShared {
     uint32_t bad[kPipeSlots];               // NaN / +inf (bit 0) or gave-up (bit 1) of the slot's piece
     unsigned long long spec[2];             // the latest prediction (a threshold key), per row set
     uint32_t spec_set[2];                   // a prediction exists
+    long long qrow[kDynQ];                  // run-time rows: the row (bit 62: a second read), -1 at the end
+    uint32_t qseq[kDynQ];                   // entry i % kDynQ holds item i when it reads i + 1
     int fin_done;                           // finishers done with the CTA's list
     int redo_n;                             // rows of the redo pass
     uint32_t redo_ready;                    // redo_n is final
@@ -2458,6 +2476,7 @@ struct PipeList {
     int64_t nredo;         // known after the main items (-1 before)
     int64_t full_units;    // units of a whole row (for "big" pieces)
     bool spec_ok;          // rows are long enough for predictions
+    bool dyn;              // rows handed out at run time (whole rows; nmain known at the end)
 };
 
 template <typename T>
@@ -2475,7 +2494,19 @@ __device__ __forceinline__ PipeList pipe_list(const RowJob& J) {
     // predictions read the spacing of a row's k best values; rows must hold
     // several times k elements
     L.spec_ok = J.k >= 8 && L.cr.nu * Elem<T>::kPerUnit >= (int64_t)16 * J.k;
+    L.dyn = J.dyn != nullptr;
+    if (L.dyn) {
+        L.nmain = -1;
+        L.rot = false;
+    }
     return L;
+}
+
+// The piece of an item: a whole row when it is read again or rows are
+// handed out at run time, else the CTA's share of it.
+template <typename T>
+__device__ __forceinline__ Piece item_piece(const RowJob& J, const PipeList& L, int64_t row, bool redo) {
+    return (redo || L.dyn) ? whole_row<T>(J, L.cr, row) : piece_of<T>(J, L.cr, row);
 }
 
 // Row of main item i.
@@ -2516,6 +2547,62 @@ __device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring
             ++q;
         }
     };
+    if (L.dyn) {
+        // take rows until none is left: first the counter's, then rows that a
+        // finisher posted for a second read; a row is done once some finisher
+        // has finished it, so the producers stop when every row is
+        auto post = [&](int64_t i, long long e) {
+            P.qrow[i % kDynQ] = e;
+            st_release_shared(&P.qseq[i % kDynQ], (uint32_t)(i + 1));
+        };
+        uint32_t* dc = J.dyn;
+        int64_t i = 0;
+        for (; ok; ++i) {
+            const uint32_t r = atomicAdd(dc + kDynNext, 1u);
+            if ((int64_t)r < J.rows) {
+                post(i, (long long)r);
+                issue(whole_row<T>(J, L.cr, (int64_t)r));
+                continue;
+            }
+            long long e = -1;
+            bool found = false;
+            for (uint32_t it = 0; it < kMaxWaitTries && !pipe_aborted(P); ++it) {
+                // claim the next posted retry: the taken count only moves from t
+                // to t + 1 while t is below the posted count (which only grows)
+                uint32_t t = *reinterpret_cast<volatile uint32_t*>(dc + kDynRetryGet);
+                bool claimed = false;
+                while (t < *reinterpret_cast<volatile uint32_t*>(dc + kDynRetryPut)) {
+                    const uint32_t seen = atomicCAS(dc + kDynRetryGet, t, t + 1u);
+                    if (seen == t) {
+                        claimed = true;
+                        break;
+                    }
+                    t = seen;
+                }
+                if (claimed) {
+                    // the poster writes the entry after taking its index: wait for it
+                    volatile uint32_t* slot = dc + kDynWords + t;
+                    uint32_t v = 0;
+                    for (uint32_t w = 0; w < kMaxWaitTries && (v = *slot) == 0u; ++w) __nanosleep(32);
+                    if (v != 0u) {
+                        *slot = 0u;  // back to zero for the next call
+                        e = (long long)(v - 1u) | (1ll << 62);
+                        found = true;
+                    }
+                    break;
+                }
+                if (*reinterpret_cast<volatile uint32_t*>(dc + kDynFinished) >= (uint32_t)J.rows) break;
+                __nanosleep(256);
+            }
+            if (!found) break;
+            post(i, e);
+            issue(whole_row<T>(J, L.cr, (int64_t)(e & ((1ll << 62) - 1))));
+        }
+        post(i, -1);
+        if (!ok) atomicExch(&P.abort, 1);
+        for (uint32_t d = q > nst ? q - nst : 0u; d < q; ++d) (void)mbar_wait_bounded(&P.full[d % nst], (d / nst) & 1u);
+        return;
+    }
     for (int64_t i = 0; ok && i < L.nmain; ++i) {
         const int64_t row = main_row(L, i);
         if (item_active<MODE>(J, row)) issue(piece_of<T>(J, L.cr, row));
@@ -2538,6 +2625,29 @@ __device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring
 template <typename T>
 __device__ __forceinline__ bool pipe_item(const RowJob& J, PipeShared& P, PipeList& L, int64_t i, int64_t& row,
                                           bool& redo) {
+    if (L.dyn) {
+        // run-time rows: entry i of the queue (the producer posts -1 at the end)
+        const uint32_t* seq = &P.qseq[i % kDynQ];
+        bool ok = true;
+        if (__shfl_sync(kFull, ld_acquire_shared(seq), 0) != (uint32_t)(i + 1)) {
+            ok = false;
+            for (uint32_t it = 0; it < kMaxWaitTries; ++it) {
+                if (ld_acquire_shared(seq) == (uint32_t)(i + 1)) {
+                    ok = true;
+                    break;
+                }
+                if ((it & 15u) == 15u && pipe_aborted(P)) break;
+                __nanosleep(64);
+            }
+            ok = __all_sync(kFull, ok);
+        }
+        if (!ok) return false;
+        const long long e = *reinterpret_cast<const volatile long long*>(&P.qrow[i % kDynQ]);
+        if (e < 0) return false;
+        row = (int64_t)(e & ((1ll << 62) - 1));
+        redo = (e >> 62) != 0;
+        return true;
+    }
     if (i < L.nmain) {
         row = main_row(L, i);
         redo = false;
@@ -2624,7 +2734,7 @@ __device__ void pipe_consume(const RowJob& J, PipeShared& P, const unsigned char
         const uint32_t sb = 1u << slot;
         // the finisher is done with this slot's previous piece
         if ((used & sb) && !pipe_wait_warp(&P.slot_empty[slot], (par & sb) ? 0u : 1u, P)) fail = true;
-        const Piece p = redo ? whole_row<T>(J, L.cr, row) : piece_of<T>(J, L.cr, row);
+        const Piece p = item_piece<T>(J, L, row, redo);
         // joint order: the piece's pair (m, s) over every element it reads
         bool jon = false;
         JointScale jc{0.0f, 0.0f};
@@ -3108,7 +3218,7 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
         } else if (lane == 0) {
             atomicExch(&P.abort, 1);
         }
-        const Piece p = redo ? whole_row<T>(J, L.cr, row) : piece_of<T>(J, L.cr, row);
+        const Piece p = item_piece<T>(J, L, row, redo);
         if (p.np > 1) {
             // publish this piece's best; the last piece of the row merges
             const int64_t ps = part_slot(L.cr, L.cr.b, row);
@@ -3145,7 +3255,10 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
         const bool held = !(spec != 0ull && rowbad == 0u && (n < J.k || sel[J.k - 1] < spec));
         if (L.spec_ok && rowbad == 0u && lane == 0) {
             // the row's best values set the prediction of the pieces that follow
-            // (and of the next call); no basis leaves it as it is
+            // (and of the next call).  A prediction that failed is dropped (it
+            // may come from rows of another scale, carried over from an earlier
+            // call): the pieces that follow seed themselves, exactly, until a
+            // row finished with its own seed sets a new one.
             const uint64_t t = next_prediction(sel, n, J.k, held);
             if (t != 0ull) {
                 const int pset = row_set<MODE>(J, row);
@@ -3156,8 +3269,14 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
         }
         if (!held) {
             if (lane == 0) {
-                const int at = atomicAdd(&P.redo_n, 1);
-                J.redo[L.rbase + at] = (int32_t)row;
+                if (L.dyn) {
+                    // post the row for a second read, by whichever producer takes it
+                    const uint32_t at = atomicAdd(J.dyn + kDynRetryPut, 1u);
+                    atomicExch(J.dyn + kDynWords + at, (uint32_t)row + 1u);
+                } else {
+                    const int at = atomicAdd(&P.redo_n, 1);
+                    J.redo[L.rbase + at] = (int32_t)row;
+                }
                 __threadfence();
             }
             __syncwarp();
@@ -3165,6 +3284,10 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
         }
         const double2 jms = make_double2((double)jm, js);
         finish_row_warp<MODE, PR>(J, row, req, n, rowbad, sel, wd, tail, unused_fs, lane, gat, &jms);
+        if (L.dyn && lane == 0) {
+            __threadfence();
+            atomicAdd(J.dyn + kDynFinished, 1u);
+        }
     }
 }
 
@@ -3195,6 +3318,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_cons
             P.spec[t] = h;
             P.spec_set[t] = h != 0ull ? 1u : 0u;
         }
+        for (int e = 0; e < kDynQ; ++e) P.qseq[e] = 0u;
         P.fin_done = 0;
         P.redo_n = 0;
         P.redo_ready = 0u;
@@ -3215,6 +3339,15 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_cons
     __syncthreads();
     if (threadIdx.x < 2 && J.hint != nullptr && P.spec_set[threadIdx.x] != 0u && P.abort == 0)
         J.hint[(size_t)threadIdx.x * kPipeMaxGrid + blockIdx.x] = P.spec[threadIdx.x];
+    // run-time rows: the last CTA to exit puts the counters back to zero
+    // (every other CTA has stopped touching them)
+    if (J.dyn != nullptr && threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(J.dyn + kDynDone, 1u) == gridDim.x - 1) {
+            for (int w = 0; w < kDynWords; ++w) atomicExch(J.dyn + w, 0u);
+            __threadfence();
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -3646,6 +3779,12 @@ static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
         if (g < grid) grid = g;
     }
     J.S = 1;
+    // With several rows per CTA, rows are handed out at run time (whole rows,
+    // one counter), so that CTAs whose stream runs slower take fewer; tree
+    // mode keeps the fixed pieces (its inactive node rows are skipped).
+    J.dyn = nullptr;
+    if (MODE != kModeTree && J.rows >= 4 * grid && J.rows + kDynOffset + kDynWords <= kRowCounterWords)
+        J.dyn = J.row_ticket + kDynOffset;
     if (J.hint != nullptr) J.hint += (size_t)MODE * 2 * kPipeMaxGrid;  // each entry point keeps its own
     // shared memory: ring | candidate slots | per finisher: sel, wd, tail
     const size_t slot_bytes = (size_t)kPipeSlots * kPipeConsumers * J.cap_w * 8;
@@ -4278,9 +4417,10 @@ uno_status uno_linear_verify_noalloc(const void* target_logits, uno_dtype dt, in
     // the array keeps the last call's contents: clear the counters this call
     // may use: request tickets, and the tickets of split rows, which the
     // general kernel keys by row (rows <= kRowCounterWords only) and the
-    // pipelined kernel by the row's first CTA (below kPipeMaxGrid)
+    // pipelined kernel by the row's first CTA (below kPipeMaxGrid), and the
+    // pipelined kernel's run-time row counters (kDynOffset on)
     if (cudaMemsetAsync(scratch + L.req_ticket, 0, (size_t)R * 4, s) != cudaSuccess) return UNO_ERR_CUDA;
-    int64_t nrow_words = rows > kPipeMaxGrid ? rows : kPipeMaxGrid;
+    int64_t nrow_words = kDynOffset + kDynWords + (rows > kPipeMaxGrid ? rows : kPipeMaxGrid);
     if (nrow_words > kRowCounterWords) nrow_words = kRowCounterWords;
     if (cudaMemsetAsync(scratch + L.row_ticket, 0, (size_t)nrow_words * 4, s) != cudaSuccess) return UNO_ERR_CUDA;
 
