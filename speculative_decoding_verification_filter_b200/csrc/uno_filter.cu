@@ -3538,89 +3538,105 @@ __global__ void __launch_bounds__(32 * kTreeMaxWarps) tree_expand_kernel(const _
     // best unexpanded child in the frontier; popping a child brings in its own
     // first child and its next sibling.  Scores never rise along those links
     // and the tie order never falls, so this pops nodes in the same order as
-    // a frontier that holds every child.
-    int nf = 0;
+    // a frontier that holds every child.  The frontier holds at most as many
+    // entries as the tree has nodes (V <= 128): entry j lives in registers of
+    // lane j % 32, slot j / 32, as its score and its tie key (depth << 24 |
+    // parent << 12 | rank; lower ranks first at equal scores).
+    constexpr int kSlots = (UNO_MAX_TREE_NODES + 31) / 32;
+    double fs[kSlots];
+    uint32_t ft[kSlots];
+    fs[0] = fs[1] = fs[2] = fs[3] = -1.0;  // empty (scores are positive)
+    ft[0] = ft[1] = ft[2] = ft[3] = 0xffffffffu;
+    auto tie_of = [](int d, int p, int rk) -> uint32_t {
+        return ((uint32_t)d << 24) | ((uint32_t)p << 12) | (uint32_t)rk;
+    };
+    // entry j := (score, tie), by its owner lane (unrolled, so that the
+    // slots stay in registers)
+#define UNO_TREE_SLOT(t_)                                     \
+    fs[t_] = (own_ && (pj_ >> 5) == (t_)) ? psc_ : fs[t_];    \
+    ft[t_] = (own_ && (pj_ >> 5) == (t_)) ? ptk_ : ft[t_];
+#define UNO_TREE_PUT(j_, sc_, tk_)                            \
+    do {                                                      \
+        const int pj_ = (j_);                                 \
+        const double psc_ = (sc_);                            \
+        const uint32_t ptk_ = (tk_);                          \
+        const bool own_ = lane == (pj_ & 31);                 \
+        UNO_TREE_SLOT(0) UNO_TREE_SLOT(1) UNO_TREE_SLOT(2) UNO_TREE_SLOT(3) \
+    } while (0)
+    static_assert(kSlots == 4, "four frontier slots per lane");
     if (lane == 0) {
         nscore[0] = 1.0;
         tok[0] = -1;
         par[0] = -1;
         dep[0] = 0;
         sco[0] = 1.0f;
-        if (ncand[0] > 0) {
-            fscore[0] = 1.0 * (double)cand_p[0];
-            fdep[0] = 1;
-            fpar[0] = 0;
-            frank[0] = 0;
-            nf = 1;
-        }
     }
-    nf = __shfl_sync(kFull, nf, 0);
     __syncwarp();
+    int nf = 0;
+    if (ncand[0] > 0) {
+        UNO_TREE_PUT(0, 1.0 * (double)cand_p[0], tie_of(1, 0, 0));
+        nf = 1;
+    }
     int n = 1;
     while (n < V && nf > 0) {
-        // lane-local best over entries lane, lane+32, ...
-        int best = -1;
-        double bs = 0.0;
-        uint32_t btie = 0xffffffffu;
-        for (int f = lane; f < nf; f += 32) {
-            const double s = fscore[f];
-            const uint32_t tie = ((uint32_t)fdep[f] << 24) | ((uint32_t)fpar[f] << 12) | (uint32_t)frank[f];
-            if (best < 0 || s > bs || (s == bs && tie < btie)) {
-                best = f;
-                bs = s;
-                btie = tie;
-            }
+        // the lane's best entry, then the warp's: the highest score, and among
+        // equal scores the smallest tie key
+        double bs = fs[0];
+        uint32_t bt = ft[0];
+        int bslot = 0;
+#define UNO_TREE_BEST(t_)                                          \
+        if (fs[t_] > bs || (fs[t_] == bs && ft[t_] < bt)) {        \
+            bs = fs[t_];                                           \
+            bt = ft[t_];                                           \
+            bslot = t_;                                            \
         }
-        // warp maximum of the score, then the smallest tie key among lanes
-        // holding it (depth < 256, parent < 4096, rank < 4096)
-        double ms = best >= 0 ? bs : -1.0;
+        UNO_TREE_BEST(1) UNO_TREE_BEST(2) UNO_TREE_BEST(3)
+#undef UNO_TREE_BEST
+        double ms = bs;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const double other = __shfl_xor_sync(kFull, ms, o);
             ms = other > ms ? other : ms;
         }
-        const uint32_t mytie = (best >= 0 && bs == ms) ? btie : 0xffffffffu;
-        const uint32_t mtie = __reduce_min_sync(kFull, mytie);
-        const unsigned owner_bal = __ballot_sync(kFull, best >= 0 && bs == ms && btie == mtie);
-        const int owner = __ffs(owner_bal) - 1;
-        const int f = __shfl_sync(kFull, best, owner);
+        const uint32_t mt = __reduce_min_sync(kFull, bs == ms ? bt : 0xffffffffu);
+        const unsigned own = __ballot_sync(kFull, bs == ms && bt == mt);
+        const int owner = __ffs(own) - 1;
+        const int jo = owner + 32 * __shfl_sync(kFull, bslot, owner);
+        const double sp = ms;
+        const int d = (int)(mt >> 24), pp = (int)((mt >> 12) & 0xfffu), rk = (int)(mt & 0xfffu);
+        // remove it: the last entry moves into its place
+        const int jl = nf - 1;
+        const int jt = jl >> 5;
+        double ls = jt == 0 ? fs[0] : jt == 1 ? fs[1] : jt == 2 ? fs[2] : fs[3];
+        uint32_t lt = jt == 0 ? ft[0] : jt == 1 ? ft[1] : jt == 2 ? ft[2] : ft[3];
+        ls = __shfl_sync(kFull, ls, jl & 31);
+        lt = __shfl_sync(kFull, lt, jl & 31);
+        UNO_TREE_PUT(jl, -1.0, 0xffffffffu);
+        if (jo != jl) UNO_TREE_PUT(jo, ls, lt);
+        nf = jl;
+        // the popped entry becomes node n
+        const int idx = n;
         if (lane == 0) {
-            const double s = fscore[f];
-            const int32_t d = fdep[f], p = fpar[f], rk = frank[f];
-            // remove f (move the last entry into its slot)
-            const int lastf = nf - 1;
-            fscore[f] = fscore[lastf];
-            fdep[f] = fdep[lastf];
-            fpar[f] = fpar[lastf];
-            frank[f] = frank[lastf];
-            int m = lastf;
-            const int idx = n;
-            nscore[idx] = s;
+            nscore[idx] = sp;
             tok[idx] = cand_id[(d - 1) * K + rk];
-            par[idx] = p;
+            par[idx] = pp;
             dep[idx] = d;
-            sco[idx] = (float)s;
-            if (d < B && ncand[d] > 0) {  // first child of the new node
-                fscore[m] = s * (double)cand_p[d * K + 0];
-                fdep[m] = d + 1;
-                fpar[m] = idx;
-                frank[m] = 0;
-                ++m;
-            }
-            if (rk + 1 < ncand[d - 1]) {  // next sibling
-                fscore[m] = nscore[p] * (double)cand_p[(d - 1) * K + rk + 1];
-                fdep[m] = d;
-                fpar[m] = p;
-                frank[m] = rk + 1;
-                ++m;
-            }
-            nf = m;
+            sco[idx] = (float)sp;
         }
-        nf = __shfl_sync(kFull, nf, 0);
-        ++n;
         __syncwarp();
+        if (d < B && ncand[d] > 0) {  // its first child
+            UNO_TREE_PUT(nf, sp * (double)cand_p[d * K + 0], tie_of(d + 1, idx, 0));
+            ++nf;
+        }
+        if (rk + 1 < ncand[d - 1]) {  // its next sibling
+            UNO_TREE_PUT(nf, nscore[pp] * (double)cand_p[(d - 1) * K + rk + 1], tie_of(d, pp, rk + 1));
+            ++nf;
+        }
+        ++n;
     }
     if (lane == 0) J.num_nodes[r] = n;
+#undef UNO_TREE_PUT
+#undef UNO_TREE_SLOT
 }
 
 // ---------------------------------------------------------------------------
