@@ -3467,14 +3467,10 @@ __global__ void __launch_bounds__(32 * kTreeMaxWarps) tree_expand_kernel(const _
     const int B = J.B, K = J.K, V = J.V;
     const int nwarps = blockDim.x >> 5;
     double* nscore = reinterpret_cast<double*>(smem);                  // [V]
-    double* fscore = nscore + V;                                       // [V + 1]
-    uint64_t* sortbufs = reinterpret_cast<uint64_t*>(fscore + V + 1);  // [nwarps][sort_cap]
+    uint64_t* sortbufs = reinterpret_cast<uint64_t*>(nscore + V);      // [nwarps][sort_cap]
     int32_t* cand_id = reinterpret_cast<int32_t*>(sortbufs + (size_t)nwarps * J.sort_cap);  // [B*K]
     float* cand_p = reinterpret_cast<float*>(cand_id + B * K);         // [B*K]
     int32_t* ncand = reinterpret_cast<int32_t*>(cand_p + B * K);       // [B]
-    int32_t* fdep = ncand + B;                                         // [V + 1]
-    int32_t* fpar = fdep + V + 1;                                      // [V + 1]
-    int32_t* frank = fpar + V + 1;                                     // [V + 1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int r = blockIdx.x;
@@ -4188,7 +4184,7 @@ uno_status uno_tree_topk_expand(const int32_t* q_ids, const float* q_probs, cons
     J.node_depth = node_depth;
     J.node_score = node_score;
     J.num_nodes = num_nodes;
-    const size_t fixed = (size_t)(2 * V + 1) * 8 + (size_t)B * K * 8 + (size_t)B * 4 + (size_t)3 * (V + 1) * 4;
+    const size_t fixed = (size_t)V * 8 + (size_t)B * K * 8 + (size_t)B * 4;
     const size_t per_warp = align_up((size_t)J.sort_cap * 8, 8);
     // warps: one per marginal up to kTreeMaxWarps, as many as fit 200 KB
     int nw = B < kTreeMaxWarps ? B : kTreeMaxWarps;
