@@ -1880,6 +1880,7 @@ constexpr int kDynFinished = 4;  // rows finished
 constexpr int kDynWords = 8;     // then one word per posted retry (row + 1; 0 = not yet written)
 constexpr int kDynOffset = 1024; // counter words start here in the row-ticket area
 constexpr int kDynQ = 64;        // queue entries (the producer runs at most a few rows ahead)
+constexpr int kTicketAhead = 3;  // stages before a row's last copy at which the next ticket is taken
 constexpr int kPipeSlots = kPipeFinishers;
 constexpr int kPipeWarps = 1 + kPipeConsumers + kPipeFinishers;
 constexpr int kPipeThreads = 32 * kPipeWarps;
@@ -2528,8 +2529,12 @@ __device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring
     const uint32_t nst = (uint32_t)J.nst;
     uint32_t q = 0;
     bool ok = true;
-    auto issue = [&](const Piece& p) {
+    // ticket: when not null, the next row's ticket is taken kTicketAhead
+    // stages before this piece's last copy (its answer is needed only then)
+    auto issue = [&](const Piece& p, uint32_t* ticket) {
+        const int at = p.nstage > kTicketAhead ? p.nstage - kTicketAhead : 0;
         for (int st = 0; ok && st < p.nstage; ++st) {
+            if (ticket != nullptr && st == at) *ticket = atomicAdd(J.dyn + kDynNext, 1u);
             const uint32_t b = q % nst;
             if (q >= nst && !pipe_spin(&P.empty[b], ((q / nst) - 1u) & 1u, P)) {
                 ok = false;
@@ -2557,19 +2562,28 @@ __device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring
         };
         uint32_t* dc = J.dyn;
         int64_t i = 0;
+        // the counter only grows, so once past the rows it stays past them
+        uint32_t r = atomicAdd(dc + kDynNext, 1u);
         for (; ok; ++i) {
-            const uint32_t r = atomicAdd(dc + kDynNext, 1u);
             if ((int64_t)r < J.rows) {
                 post(i, (long long)r);
-                issue(whole_row<T>(J, L.cr, (int64_t)r));
+                uint32_t nx = 0xffffffffu;
+                issue(whole_row<T>(J, L.cr, (int64_t)r), &nx);
+                r = nx;
                 continue;
             }
             long long e = -1;
             bool found = false;
             for (uint32_t it = 0; it < kMaxWaitTries && !pipe_aborted(P); ++it) {
+                // the three counters in one round trip.  Every row finished
+                // means no retry is outstanding (a posted row counts as
+                // finished only once its second read has finished it).
+                const uint32_t put0 = *reinterpret_cast<volatile uint32_t*>(dc + kDynRetryPut);
+                uint32_t t = *reinterpret_cast<volatile uint32_t*>(dc + kDynRetryGet);
+                const uint32_t fin0 = *reinterpret_cast<volatile uint32_t*>(dc + kDynFinished);
+                if (t >= put0 && fin0 >= (uint32_t)J.rows) break;
                 // claim the next posted retry: the taken count only moves from t
                 // to t + 1 while t is below the posted count (which only grows)
-                uint32_t t = *reinterpret_cast<volatile uint32_t*>(dc + kDynRetryGet);
                 bool claimed = false;
                 while (t < *reinterpret_cast<volatile uint32_t*>(dc + kDynRetryPut)) {
                     const uint32_t seen = atomicCAS(dc + kDynRetryGet, t, t + 1u);
@@ -2591,12 +2605,11 @@ __device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring
                     }
                     break;
                 }
-                if (*reinterpret_cast<volatile uint32_t*>(dc + kDynFinished) >= (uint32_t)J.rows) break;
-                __nanosleep(256);
+                __nanosleep(64);
             }
             if (!found) break;
             post(i, e);
-            issue(whole_row<T>(J, L.cr, (int64_t)(e & ((1ll << 62) - 1))));
+            issue(whole_row<T>(J, L.cr, (int64_t)(e & ((1ll << 62) - 1))), nullptr);
         }
         post(i, -1);
         if (!ok) atomicExch(&P.abort, 1);
@@ -2605,12 +2618,13 @@ __device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring
     }
     for (int64_t i = 0; ok && i < L.nmain; ++i) {
         const int64_t row = main_row(L, i);
-        if (item_active<MODE>(J, row)) issue(piece_of<T>(J, L.cr, row));
+        if (item_active<MODE>(J, row)) issue(piece_of<T>(J, L.cr, row), nullptr);
     }
     // the redo pass: rows whose prediction failed, read whole
     if (ok && wait_flag(&P.redo_ready, P)) {
         const int n = *reinterpret_cast<volatile int*>(&P.redo_n);
-        for (int j = 0; ok && j < n; ++j) issue(whole_row<T>(J, L.cr, (int64_t)__ldcg(J.redo + L.rbase + j)));
+        for (int j = 0; ok && j < n; ++j)
+            issue(whole_row<T>(J, L.cr, (int64_t)__ldcg(J.redo + L.rbase + j)), nullptr);
     } else {
         ok = false;
     }
@@ -3339,9 +3353,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1) pipe_kernel(const __grid_cons
     __syncthreads();
     if (threadIdx.x < 2 && J.hint != nullptr && P.spec_set[threadIdx.x] != 0u && P.abort == 0)
         J.hint[(size_t)threadIdx.x * kPipeMaxGrid + blockIdx.x] = P.spec[threadIdx.x];
-    // run-time rows: the last CTA to exit puts the counters back to zero
-    // (every other CTA has stopped touching them)
-    if (J.dyn != nullptr && threadIdx.x == 0) {
+    // run-time rows: the request-tail kernel that follows puts the counters
+    // back to zero; without one, the last CTA to exit does (every other CTA
+    // has stopped touching them)
+    if (MODE == kModeFilter && J.dyn != nullptr && threadIdx.x == 0) {
         __threadfence();
         if (atomicAdd(J.dyn + kDynDone, 1u) == gridDim.x - 1) {
             for (int w = 0; w < kDynWords; ++w) atomicExch(J.dyn + w, 0u);
@@ -3366,6 +3381,8 @@ __global__ void __launch_bounds__(32 * kTailWarps) tail_kernel(const __grid_cons
     static_assert(sizeof(RowJob) % 4 == 0, "copied by words");
     for (int i = threadIdx.x; i < (int)(sizeof(RowJob) / 4); i += blockDim.x)
         reinterpret_cast<uint32_t*>(&sJ)[i] = reinterpret_cast<const uint32_t*>(&J)[i];
+    // the row kernel's run-time row counters, back to zero for the next call
+    if (blockIdx.x == 0 && threadIdx.x < kDynWords && J.dyn != nullptr) J.dyn[threadIdx.x] = 0u;
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t r = (int64_t)blockIdx.x * kTailWarps + warp;
