@@ -2533,6 +2533,8 @@ __device__ void pipe_produce(const RowJob& J, PipeShared& P, unsigned char* ring
     // stages before this piece's last copy (its answer is needed only then)
     auto issue = [&](const Piece& p, uint32_t* ticket) {
         const int at = p.nstage > kTicketAhead ? p.nstage - kTicketAhead : 0;
+        // a piece with no stage (a row of head and tail scalars only) still takes its ticket
+        if (ticket != nullptr && p.nstage == 0) *ticket = atomicAdd(J.dyn + kDynNext, 1u);
         for (int st = 0; ok && st < p.nstage; ++st) {
             if (ticket != nullptr && st == at) *ticket = atomicAdd(J.dyn + kDynNext, 1u);
             const uint32_t b = q % nst;
@@ -3783,8 +3785,6 @@ static size_t row_smem_bytes(RowJob& J) {
     return (size_t)J.fin_off + finish;
 }
 
-// The pipelined kernel: grid (balanced pieces), ring depth and shared memory.
-// Returns UNO_ERR_UNSUPPORTED (nothing launched) when it does not fit.
 // The joint order's per-row normalisers, ahead of the row kernels.
 template <typename T, int MODE>
 static uno_status launch_joint(const RowJob& J, cudaStream_t stream) {
@@ -3793,6 +3793,9 @@ static uno_status launch_joint(const RowJob& J, cudaStream_t stream) {
     return cudaGetLastError() == cudaSuccess ? UNO_OK : UNO_ERR_CUDA;
 }
 
+// The pipelined kernel: grid (balanced pieces or run-time rows), ring depth
+// and shared memory.  Returns UNO_ERR_UNSUPPORTED (nothing launched) when it
+// does not fit.
 template <typename T, int MODE>
 static uno_status launch_pipe(RowJob J, cudaStream_t stream) {
     J.hw = J.k + 16 > 64 ? J.k + 16 : 64;

@@ -43,6 +43,11 @@ CASES = [
     ("f32", 64, 300, 1.0, 1024, 1.0),
     ("bf16", 9, 7, 1.0, 50, 0.95),
     ("f32", 9, 1, 1.0, 50, 0.95),
+    # enough rows for run-time row hand-out, on rows of head and tail scalars
+    # only (no whole 16-byte unit) and on barely longer ones
+    ("bf16", 700, 7, 1.0, 50, 0.95),
+    ("f32", 650, 3, 1.0, 50, 0.95),
+    ("bf16", 640, 9, 0.8, 4, 0.9),
     ("f32", 33, 2000, 0.0, 50, 0.95),
     ("bf16", 33, 2000, 1.0, 1, 0.95),
     ("f32", 33, 2000, 1.0, 50, 1.0),

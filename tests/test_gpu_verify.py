@@ -6,8 +6,8 @@ import torch
 
 import oracle
 from _parity import Events, compare_filter, compare_requests, np_of, to_device
-from speculative_decoding_verification_filter_b200 import (uno_filter_softmax, uno_linear_verify,
-                                                          uno_tree_topk_expand, uno_tree_verify)
+from speculative_decoding_verification_filter_b200 import (LAYOUT_TWO_PASS, uno_filter_softmax, uno_linear_cycle,
+                                                          uno_linear_verify, uno_tree_topk_expand, uno_tree_verify)
 from speculative_decoding_verification_filter_b200.inputs import (Workload, linear_draft, linear_target,
                                                                  tree_draft, tree_target)
 
@@ -80,6 +80,9 @@ LINEAR_CASES = [
     # more than 32 draft positions (token slots beyond one warp)
     Workload("lin f32 B=40", "linear", R=3, B=40, vocab=600, dtype="f32", sigma=1.0, noise=0.05, top_k=10, seed=10),
     Workload("lin bf16 B=40 top-k 50", "linear", R=3, B=40, vocab=600, dtype="bf16", sigma=1.0, noise=0.05, seed=13),
+    # rows handed out at run time, each only head and tail scalars
+    Workload("lin bf16 tiny vocab many rows", "linear", R=100, B=6, vocab=6, dtype="bf16", sigma=1.0, noise=0.5,
+             seed=14),
 ]
 
 
@@ -189,4 +192,22 @@ def test_linear_draft_row_layouts(layout):
     r = oracle.linear_verify(p_np, w.dtype, w.R, w.B, w.temperature, w.top_k, w.top_p,
                              rq["sample"].reshape(w.R, w.B), rq["ids"], rq["probs"], rq["count"], rng=rng)
     compare_requests(g, r, ev, LINEAR_KEYS)
+    ev.check()
+
+
+def test_cycle_with_tiny_vocabulary_and_many_rows():
+    """uno_linear_cycle in the two-pass layout over 1,200 rows of 6 logits:
+    rows handed out at run time, none holding a whole 16-byte unit."""
+    w = Workload("cycle tiny vocab", "linear", R=100, B=6, vocab=6, dtype="bf16", sigma=1.0, noise=0.5, seed=15)
+    q_np = linear_draft(w)
+    p_np = np.ascontiguousarray(linear_target(w).reshape(w.R, w.B + 1, -1)[:, :w.B]).reshape(w.R * w.B, -1)
+    rng = (w.seed, 3, 1)
+    sp = dict(temperature=w.temperature, top_k=w.top_k, top_p=w.top_p)
+    g = uno_linear_cycle(to_device(q_np, w.dtype), to_device(p_np, w.dtype), R=w.R, B=w.B, rng=rng,
+                         layout=LAYOUT_TWO_PASS, **sp)
+    r = oracle.linear_cycle(q_np, p_np, w.dtype, w.R, w.B, w.temperature, w.top_k, w.top_p, rng)
+    ref = dict(tokens=r["tokens"], num_accepted=r["num_correct_drafts"], num_tokens=r["accept_len"],
+               flags=r["flags"], margin=r["margin"])
+    ev = Events("tiny vocabulary cycle, two-pass layout")
+    compare_requests(g, ref, ev, ("tokens", "num_accepted", "num_tokens", "flags"))
     ev.check()
