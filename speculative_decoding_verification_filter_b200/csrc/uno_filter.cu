@@ -2175,15 +2175,25 @@ struct StageScan<__nv_bfloat16> {
         const uint4 ninf = Elem<__nv_bfloat16>::neg_inf_unit();
         uint32_t ub = 0;
         B2 mx = ninf2(), nn = ninf2();
+        if (left >= 32 * kPLaneUnits) {  // every unit of the lane is present (all but a row's last stage)
 #pragma unroll 4
-        for (int u = 0; u < kPLaneUnits; ++u) {
-            const bool here = 32 * u < left;
-            const uint4 x = lds128(sa + (uint32_t)u * 512u);
-            const uint4 r = here ? x : ninf;
-            const B2 m = Elem<__nv_bfloat16>::umax(r);
-            nn = __hmax2_nan(nn, m);
-            mx = __hmax2(mx, m);
-            ub |= (here && __hgeu2_mask(m, tau) != 0u ? 1u : 0u) << u;
+            for (int u = 0; u < kPLaneUnits; ++u) {
+                const B2 m = Elem<__nv_bfloat16>::umax(lds128(sa + (uint32_t)u * 512u));
+                nn = __hmax2_nan(nn, m);
+                mx = __hmax2(mx, m);
+                ub |= (__hgeu2_mask(m, tau) != 0u ? 1u : 0u) << u;
+            }
+        } else {
+#pragma unroll 4
+            for (int u = 0; u < kPLaneUnits; ++u) {
+                const bool here = 32 * u < left;
+                const uint4 x = lds128(sa + (uint32_t)u * 512u);
+                const uint4 r = here ? x : ninf;
+                const B2 m = Elem<__nv_bfloat16>::umax(r);
+                nn = __hmax2_nan(nn, m);
+                mx = __hmax2(mx, m);
+                ub |= (here && __hgeu2_mask(m, tau) != 0u ? 1u : 0u) << u;
+            }
         }
         lm = gkey(mx);
         bad = nonfinite(nn);
@@ -2260,15 +2270,25 @@ struct StageScan<float> {
         const uint32_t sa = smem_u32(lsp);
         uint32_t ub = 0;
         float mx = -__int_as_float(0x7f800000), nn = -__int_as_float(0x7f800000);
+        if (left >= 32 * kPLaneUnits) {  // every unit of the lane is present (all but a row's last stage)
 #pragma unroll 4
-        for (int u = 0; u < kPLaneUnits; ++u) {
-            const bool here = 32 * u < left;
-            const uint4 x = lds128(sa + (uint32_t)u * 512u);
-            const uint4 r = here ? x : Elem<float>::neg_inf_unit();
-            const float m = Elem<float>::umax(r);
-            nn = Elem<float>::max_nan(nn, m);
-            mx = fmaxf(mx, m);
-            ub |= (here && !(m < tau) ? 1u : 0u) << u;
+            for (int u = 0; u < kPLaneUnits; ++u) {
+                const float m = Elem<float>::umax(lds128(sa + (uint32_t)u * 512u));
+                nn = Elem<float>::max_nan(nn, m);
+                mx = fmaxf(mx, m);
+                ub |= (!(m < tau) ? 1u : 0u) << u;
+            }
+        } else {
+#pragma unroll 4
+            for (int u = 0; u < kPLaneUnits; ++u) {
+                const bool here = 32 * u < left;
+                const uint4 x = lds128(sa + (uint32_t)u * 512u);
+                const uint4 r = here ? x : Elem<float>::neg_inf_unit();
+                const float m = Elem<float>::umax(r);
+                nn = Elem<float>::max_nan(nn, m);
+                mx = fmaxf(mx, m);
+                ub |= (here && !(m < tau) ? 1u : 0u) << u;
+            }
         }
         lm = gkey(mx);
         bad = !(nn < __int_as_float(0x7f800000));
