@@ -3023,17 +3023,50 @@ __device__ __noinline__ int warp_rank_topk(const uint64_t* g, int U, int k, uint
 }
 
 // The best min(k, U) of U distinct keys g[0..U) (U <= kPGather), into
-// sel[] in descending order: first cut g to the keys whose high half reaches
-// the k-th largest high half (a warp radix search), then rank the rest.
-__device__ __noinline__ int warp_select_topk(uint64_t* g, int U, int k, uint64_t* sel, int lane) {
+// sel[] in descending order: first cut g to the keys whose high half lies in
+// the k-th largest one's bucket or above, then rank the rest.  The buckets
+// split the keys' range of high halves [bot, top] into at most 64 classes
+// of 2^shift values each, counted into hist[64] (shared memory).  Whole
+// buckets are kept, so the cut keeps the best k and at least k keys.
+__device__ __noinline__ int warp_select_topk(uint64_t* g, int U, int k, uint64_t* sel, uint32_t* hist, int lane) {
     if (U > k + 8) {
         constexpr int PER = kPGather / 32;
         uint32_t v[PER];
+        uint32_t vmax = 0u, vmin = 0xffffffffu;
 #pragma unroll
-        for (int j = 0; j < PER; ++j) v[j] = lane + 32 * j < U ? (uint32_t)(g[lane + 32 * j] >> 32) : 0u;
-        const uint64_t x = (uint64_t)warp_kth_hi16<PER>(v, k) << 32;
+        for (int j = 0; j < PER; ++j) {
+            const bool here = lane + 32 * j < U;
+            v[j] = here ? (uint32_t)(g[lane + 32 * j] >> 32) : 0u;
+            vmax = here && v[j] > vmax ? v[j] : vmax;
+            vmin = here && v[j] < vmin ? v[j] : vmin;
+        }
+        const uint32_t top = __reduce_max_sync(kFull, vmax), bot = __reduce_min_sync(kFull, vmin);
+        const uint32_t span = top - bot;
+        const int shift = span < 64u ? 0 : 26 - __clz(span);  // span >> shift < 64
+        hist[lane] = 0u;
+        hist[lane + 32] = 0u;
         __syncwarp();
-        U = warp_keep_ge(g, U, x, lane);
+#pragma unroll
+        for (int j = 0; j < PER; ++j)
+            if (lane + 32 * j < U) atomicAdd(&hist[(top - v[j]) >> shift], 1u);  // bucket 0 holds top
+        __syncwarp();
+        // running counts from the top: lane l holds buckets 2l and 2l + 1
+        const uint32_t c0 = hist[2 * lane], c1 = hist[2 * lane + 1];
+        uint32_t incl = c0 + c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += t;
+        }
+        const bool first_half = incl - c1 >= (uint32_t)k;
+        const unsigned reach = __ballot_sync(kFull, incl >= (uint32_t)k);  // a suffix of the lanes (U >= k)
+        const int L = __ffs(reach) - 1;
+        const int bstar = 2 * L + (__shfl_sync(kFull, first_half, L) ? 0 : 1);
+        // keep the keys of buckets 0..bstar: top - hi < (bstar + 1) << shift
+        int64_t lo = (int64_t)top - ((int64_t)(bstar + 1) << shift) + 1;
+        lo = lo < 0 ? 0 : lo;
+        __syncwarp();
+        U = warp_keep_ge(g, U, (uint64_t)lo << 32, lane);
     }
     return warp_rank_topk(g, U, k, sel, lane);
 }
@@ -3223,7 +3256,7 @@ __device__ void pipe_finish(const RowJob& J, PipeShared& P, const uint64_t* slot
                     slot_reset(P, slot);
                     mbar_arrive(&P.slot_empty[slot]);
                 }
-                n = warp_select_topk(gat, U, J.k, sel, lane);
+                n = warp_select_topk(gat, U, J.k, sel, reinterpret_cast<uint32_t*>(wd), lane);
             } else {  // more keys than the scratch holds: select from the slot itself
                 int cw[kPipeConsumers];
                 U = 0;
