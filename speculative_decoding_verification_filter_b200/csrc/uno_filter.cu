@@ -3609,11 +3609,12 @@ __global__ void __launch_bounds__(32 * kTreeMaxWarps) tree_expand_kernel(const _
     // a frontier that holds every child.  The frontier holds at most as many
     // entries as the tree has nodes (V <= 128): entry j lives in registers of
     // lane j % 32, slot j / 32, as its score and its tie key (depth << 24 |
-    // parent << 12 | rank; lower ranks first at equal scores).
+    // parent << 12 | rank; lower ranks first at equal scores).  An empty slot
+    // holds score 0 and the largest tie key, so every entry ranks above it.
     constexpr int kSlots = (UNO_MAX_TREE_NODES + 31) / 32;
     double fs[kSlots];
     uint32_t ft[kSlots];
-    fs[0] = fs[1] = fs[2] = fs[3] = -1.0;  // empty (scores are positive)
+    fs[0] = fs[1] = fs[2] = fs[3] = 0.0;  // empty
     ft[0] = ft[1] = ft[2] = ft[3] = 0xffffffffu;
     auto tie_of = [](int d, int p, int rk) -> uint32_t {
         return ((uint32_t)d << 24) | ((uint32_t)p << 12) | (uint32_t)rk;
@@ -3660,14 +3661,17 @@ __global__ void __launch_bounds__(32 * kTreeMaxWarps) tree_expand_kernel(const _
         }
         UNO_TREE_BEST(1) UNO_TREE_BEST(2) UNO_TREE_BEST(3)
 #undef UNO_TREE_BEST
-        double ms = bs;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const double other = __shfl_xor_sync(kFull, ms, o);
-            ms = other > ms ? other : ms;
-        }
-        const uint32_t mt = __reduce_min_sync(kFull, bs == ms ? bt : 0xffffffffu);
-        const unsigned own = __ballot_sync(kFull, bs == ms && bt == mt);
+        // scores are >= 0, so their bit patterns order as their values: the
+        // warp's best is the largest high word, then low word, then the
+        // smallest tie key (three 32-bit warp reductions)
+        const uint64_t bb = (uint64_t)__double_as_longlong(bs);
+        const uint32_t bh = (uint32_t)(bb >> 32), bl = (uint32_t)bb;
+        const uint32_t mh = __reduce_max_sync(kFull, bh);
+        const uint32_t ml = __reduce_max_sync(kFull, bh == mh ? bl : 0u);
+        const bool best = bh == mh && bl == ml;
+        const double ms = __longlong_as_double((long long)(((uint64_t)mh << 32) | ml));
+        const uint32_t mt = __reduce_min_sync(kFull, best ? bt : 0xffffffffu);
+        const unsigned own = __ballot_sync(kFull, best && bt == mt);
         const int owner = __ffs(own) - 1;
         const int jo = owner + 32 * __shfl_sync(kFull, bslot, owner);
         const double sp = ms;
@@ -3679,7 +3683,7 @@ __global__ void __launch_bounds__(32 * kTreeMaxWarps) tree_expand_kernel(const _
         uint32_t lt = jt == 0 ? ft[0] : jt == 1 ? ft[1] : jt == 2 ? ft[2] : ft[3];
         ls = __shfl_sync(kFull, ls, jl & 31);
         lt = __shfl_sync(kFull, lt, jl & 31);
-        UNO_TREE_PUT(jl, -1.0, 0xffffffffu);
+        UNO_TREE_PUT(jl, 0.0, 0xffffffffu);
         if (jo != jl) UNO_TREE_PUT(jo, ls, lt);
         nf = jl;
         // the popped entry becomes node n
