@@ -3531,7 +3531,7 @@ struct TreeJob {
     int32_t* num_nodes;
 };
 
-constexpr int kTreeMaxWarps = 8;
+constexpr int kTreeMaxWarps = 16;
 constexpr int kTreeRankMax = 256;  // rows up to this many entries are ranked, longer ones sorted
 
 __global__ void __launch_bounds__(32 * kTreeMaxWarps) tree_expand_kernel(const __grid_constant__ TreeJob J) {
@@ -3683,6 +3683,14 @@ __global__ void __launch_bounds__(32 * kTreeMaxWarps) tree_expand_kernel(const _
         uint32_t lt = jt == 0 ? ft[0] : jt == 1 ? ft[1] : jt == 2 ? ft[2] : ft[3];
         ls = __shfl_sync(kFull, ls, jl & 31);
         lt = __shfl_sync(kFull, lt, jl & 31);
+        // everything the pushes below read, loaded at once (nothing of it is
+        // written in this step: the parent pp was stored steps ago)
+        const int nc_child = d < B ? ncand[d] : 0;
+        const float p_child = d < B ? cand_p[d * K] : 0.0f;
+        const int nc_sib = ncand[d - 1];
+        const float p_sib = rk + 1 < K ? cand_p[(d - 1) * K + rk + 1] : 0.0f;
+        const double s_par = nscore[pp];
+        const int32_t t_new = cand_id[(d - 1) * K + rk];
         UNO_TREE_PUT(jl, 0.0, 0xffffffffu);
         if (jo != jl) UNO_TREE_PUT(jo, ls, lt);
         nf = jl;
@@ -3690,18 +3698,18 @@ __global__ void __launch_bounds__(32 * kTreeMaxWarps) tree_expand_kernel(const _
         const int idx = n;
         if (lane == 0) {
             nscore[idx] = sp;
-            tok[idx] = cand_id[(d - 1) * K + rk];
+            tok[idx] = t_new;
             par[idx] = pp;
             dep[idx] = d;
             sco[idx] = (float)sp;
         }
         __syncwarp();
-        if (d < B && ncand[d] > 0) {  // its first child
-            UNO_TREE_PUT(nf, sp * (double)cand_p[d * K + 0], tie_of(d + 1, idx, 0));
+        if (nc_child > 0) {  // its first child
+            UNO_TREE_PUT(nf, sp * (double)p_child, tie_of(d + 1, idx, 0));
             ++nf;
         }
-        if (rk + 1 < ncand[d - 1]) {  // its next sibling
-            UNO_TREE_PUT(nf, nscore[pp] * (double)cand_p[(d - 1) * K + rk + 1], tie_of(d, pp, rk + 1));
+        if (rk + 1 < nc_sib) {  // its next sibling
+            UNO_TREE_PUT(nf, s_par * (double)p_sib, tie_of(d, pp, rk + 1));
             ++nf;
         }
         ++n;
