@@ -1896,8 +1896,13 @@ constexpr int kPGather = 256;                                   // keys a finish
 constexpr int kPipeMinStages = 6, kPipeMaxStages = 12;
 // The largest grid: part slots of split rows are sized for it.
 constexpr int kPipeMaxGrid = 256;
-// A piece of a row is at least this many units when rows are few.
-constexpr int64_t kPipeMinPieceUnits = 4 * kPStageUnits;
+// A piece of a row is at least this many units when rows are few.  A split
+// row costs a merge across CTAs after its pieces (about 8 us: the pieces'
+// keys published, a ticket, the last piece reading them back); a piece of
+// 19 stages (304 KB) streams about as long on one SM, so shorter pieces do
+// not pay for the merge (16 bf16 rows of 151,936 logits: 24.6 us whole
+// against 32.8 us in pieces of 4 stages).
+constexpr int64_t kPipeMinPieceUnits = 19 * kPStageUnits;
 // A row is cut into at most this many pieces (one merge warp).
 constexpr int kPipeMaxPieces = 32;
 // Suspend hint of the off-path waits (ns): the waiting thread sleeps until

@@ -40,6 +40,7 @@ CASES = [
     ("bf16", 6, 151936, 1.0, 50, 0.95),
     ("f32", 5, 151936, 0.7, 50, 0.95),
     ("bf16", 3, 65537, 1.0, 300, 0.999),
+    ("bf16", 2, 1000003, 1.0, 50, 0.95),  # long rows: about six pieces each, merged across CTAs
     ("f32", 64, 300, 1.0, 1024, 1.0),
     ("bf16", 9, 7, 1.0, 50, 0.95),
     ("f32", 9, 1, 1.0, 50, 0.95),
@@ -119,13 +120,14 @@ def test_non_finite_rows_are_flagged_not_trapped():
 
 
 def test_split_rows_and_single_cta_rows_agree():
-    """The same rows filtered alone (split across CTAs) and in a large batch
-    (one CTA per row) give identical results."""
+    """The same rows filtered alone (fp32 rows of 151,936 logits: each split
+    across two CTAs) and in a large batch (one CTA per row, rows handed out
+    at run time) give identical results."""
     rng = np.random.default_rng(8)
-    x = to_bf16_bits(_rows(rng, 4, 151936, scale=1.0, peak=8.0))
-    few = uno_filter_softmax(to_device(x, "bf16"), temperature=1.0, top_k=50, top_p=0.95, rng=(5, 0))
-    many_x = np.concatenate([x] * 300)
-    many = uno_filter_softmax(to_device(many_x, "bf16"), temperature=1.0, top_k=50, top_p=0.95, rng=(5, 0))
+    x = _rows(rng, 4, 151936, scale=1.0, peak=8.0)
+    few = uno_filter_softmax(to_device(x, "f32"), temperature=1.0, top_k=50, top_p=0.95, rng=(5, 0))
+    many_x = np.concatenate([x] * 150)
+    many = uno_filter_softmax(to_device(many_x, "f32"), temperature=1.0, top_k=50, top_p=0.95, rng=(5, 0))
     for key in ("ids", "probs", "count"):
         assert torch.equal(few[key], many[key][:4]), key
     assert torch.equal(few["sample"], many["sample"][:4])
