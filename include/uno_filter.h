@@ -396,10 +396,15 @@ uno_status uno_linear_verify_noalloc(const void* target_logits, uno_dtype dt, in
  * out_o        [R][V][H][d] float; out_lse [R][V][H] float.
  * out_flags    nullable [R]: UNO_FLAG_BAD_TREE when a node's parent breaks
  *              the rule above.  That node then attends to itself alone.
- * Limits: 1 <= V <= UNO_MAX_TREE_NODES, d <= 256, H a multiple of Hkv, and
- * the key and value tiles of one head, 2 * V * (d + 1) floats, within shared
- * memory; UNO_ERR_UNSUPPORTED otherwise.  One CTA runs per (request,
- * key/value head).  No workspace.
+ * Kernels: bf16 calls with d a multiple of 16, q, k, v, o_prefix and out_o
+ * 16-byte aligned and the operand tiles within 200 KB of shared memory run
+ * on the tensor cores (tcgen05, accumulators in tensor memory), one CTA per
+ * (request, key/value head, 128 stacked query rows).  Every other call runs
+ * on a CUDA-core kernel, one CTA per (request, key/value head), which needs
+ * the key and value tiles of one head, 2 * V * (d + 1) floats, within
+ * shared memory.  Arrays need only their element alignment.
+ * Limits: 1 <= V <= UNO_MAX_TREE_NODES, d <= 256, H a multiple of Hkv;
+ * UNO_ERR_UNSUPPORTED when neither kernel applies.  No workspace.
  * ---------------------------------------------------------------------- */
 #define UNO_FLAG_BAD_TREE 16u
 uno_status uno_tree_suffix_attention_merge(const void* q, const void* k, const void* v, uno_dtype dt, int32_t R,

@@ -571,9 +571,13 @@ extern "C" uno_status uno_tree_suffix_attention_merge(const void* q, const void*
         return UNO_ERR_INVALID_ARG;
     if (d > kMaxD) return UNO_ERR_UNSUPPORTED;
     // bf16 rows with d a multiple of 16 take the tensor cores; the rest the
-    // CUDA-core kernel
+    // CUDA-core kernel.  The tensor-core kernel moves q, k, v, o_prefix and
+    // out_o 16 bytes at a time (rows of d a multiple of 16 keep that
+    // alignment), so arrays that start off a 16-byte boundary go to the
+    // CUDA-core kernel, which reads and writes single elements.
     const size_t tc_smem = tc_smem_bytes(V, d);
-    const bool tc = dt == UNO_BF16 && d % 16 == 0 && tc_smem <= 200 * 1024;
+    const bool tc = dt == UNO_BF16 && d % 16 == 0 && tc_smem <= 200 * 1024 && aligned(q, 16) && aligned(k, 16) &&
+                    aligned(v, 16) && aligned(o_prefix, 16) && aligned(out_o, 16);
     const size_t smem = ((size_t)2 * V * (d + 1) + (size_t)kWarps * d) * 4 + (size_t)V * kMaskWords * 4;
     if (!tc && smem > 227 * 1024) return UNO_ERR_UNSUPPORTED;
     Job J{};

@@ -114,3 +114,21 @@ def test_bad_tree_is_flagged_and_confined_to_its_request():
 def test_tensor_core_shapes(R, V, H, Hkv, d, L, seed, kw):
     dev, host, scale = _case(R, V, H, Hkv, d, L, seed, "bf16", **kw)
     _check(dev, host, scale)
+
+
+def test_misaligned_arrays_take_the_cuda_core_kernel():
+    """The 8B-model shape with q, k, v and o_prefix starting one element past
+    a 16-byte boundary: the tensor-core kernel would move them 16 bytes at a
+    time, so the call runs on the CUDA-core kernel and matches the oracle."""
+    dev, host, scale = _case(2, 32, 32, 8, 128, 20, 5, "bf16")
+
+    def shifted(t):
+        flat = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+        view = flat[1:].view(t.shape)
+        view.copy_(t)
+        return view
+
+    for key in ("q", "k", "v", "o_prefix"):
+        dev[key] = shifted(dev[key])
+        assert dev[key].data_ptr() % 16 != 0, key
+    _check(dev, host, scale)
