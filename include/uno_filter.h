@@ -397,7 +397,7 @@ uno_status uno_linear_verify_noalloc(const void* target_logits, uno_dtype dt, in
  * out_flags    nullable [R]: UNO_FLAG_BAD_TREE when a node's parent breaks
  *              the rule above.  That node then attends to itself alone.
  * Kernels: bf16 calls with d a multiple of 16, q, k, v, o_prefix and out_o
- * 16-byte aligned and the operand tiles within 200 KB of shared memory run
+ * 16-byte aligned and the operand tiles within 220 KB of shared memory run
  * on the tensor cores (tcgen05, accumulators in tensor memory), one CTA per
  * (request, key/value head, 128 stacked query rows).  Every other call runs
  * on a CUDA-core kernel, one CTA per (request, key/value head), which needs

@@ -280,17 +280,28 @@ __device__ __forceinline__ uint32_t bf16_bits(float x) {
     return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
-// shared-memory bytes of the tensor-core form (0: it does not apply)
-// (the epilogue's O blocks of 128 x (cb + 4) floats reuse the operand area
-// and the ancestor masks)
-__host__ __device__ inline size_t tc_smem_bytes(int V, int d) {
+// shared-memory bytes of the tensor-core form: the operands (the
+// epilogue's O blocks of 128 x (cb + 4) floats reuse their area and the
+// ancestor masks), then a block of 128 x cb prefix floats that arrives by
+// asynchronous copies while the block before it is worked on
+__host__ __device__ inline int tc_block_cols(int d) { return d < 64 ? d : 64; }
+__host__ __device__ inline size_t tc_prefetch_offset(int V, int d) {
     const int Np = (V + 15) / 16 * 16;
     const size_t ops = (size_t)kTcRows * d * 2 + (size_t)Np * d * 2 * 2 + (size_t)3 * kTcRows * Np * 2 +
                        (size_t)V * kMaskWords * 4;
-    const int cb = d < 64 ? d : 64;
-    const size_t out = (size_t)kTcRows * (cb + 4) * 4;
+    const size_t out = (size_t)kTcRows * (tc_block_cols(d) + 4) * 4;
     return ops > out ? ops : out;
 }
+__host__ __device__ inline size_t tc_smem_bytes(int V, int d) {
+    return tc_prefetch_offset(V, d) + (size_t)kTcRows * tc_block_cols(d) * 4;
+}
+// 16 bytes global -> shared, asynchronously (both addresses 16-byte aligned)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const __grid_constant__ Job J) {
     extern __shared__ __align__(1024) unsigned char sm[];
@@ -322,39 +333,56 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
     int n = J.num_nodes[r];
     n = n < 1 ? 1 : (n > V ? V : n);
 
-    // staging: 16-byte chunks (8 elements), kTcBatch loads in flight per thread
+    // staging: 16-byte chunks (8 elements).  Q and K go straight to their
+    // K-major places by asynchronous copies (absent rows are zeroed); V is
+    // transposed through registers, kTcBatch loads in flight per thread.
     const int cpr = d >> 3;
     const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-    for (int e0 = tid; e0 < kTcRows * cpr; e0 += kTcThreads * kTcBatch) {
-        uint4 x[kTcBatch];
-#pragma unroll
-        for (int u = 0; u < kTcBatch; ++u) {
-            const int e = e0 + u * kTcThreads, ml = e / cpr, c = e - ml * cpr, m = m0 + ml;
-            x[u] = zero;
-            if (e < kTcRows * cpr && m < rows) {
-                const int hl = m / V, j = m - hl * V;
-                if (j < n) {
-                    const size_t row = ((size_t)r * V + j) * J.H + (size_t)g * G + hl;
-                    x[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.q) + row * d) + c);
-                }
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kTcBatch; ++u) {
-            const int e = e0 + u * kTcThreads, ml = e / cpr, c = e - ml * cpr;
-            if (e < kTcRows * cpr) *reinterpret_cast<uint4*>(sQ + kmajor_off(ml, c * 8, d)) = x[u];
+    for (int e = tid; e < kTcRows * cpr; e += kTcThreads) {
+        const int ml = e / cpr, c = e - ml * cpr, m = m0 + ml;
+        const int hl = m / V, j = m - hl * V;
+        unsigned char* dst = sQ + kmajor_off(ml, c * 8, d);
+        if (m < rows && j < n) {
+            const size_t row = ((size_t)r * V + j) * J.H + (size_t)g * G + hl;
+            cp_async16(dst, static_cast<const __nv_bfloat16*>(J.q) + row * d + c * 8);
+        } else {
+            *reinterpret_cast<uint4*>(dst) = zero;
         }
     }
+    for (int e = tid; e < Np * cpr; e += kTcThreads) {
+        const int i = e / cpr, c = e - i * cpr;
+        unsigned char* dst = sK + kmajor_off(i, c * 8, d);
+        if (i < n)
+            cp_async16(dst, static_cast<const __nv_bfloat16*>(J.k) + (((size_t)r * V + i) * J.Hkv + g) * d + c * 8);
+        else
+            *reinterpret_cast<uint4*>(dst) = zero;
+    }
+    cp_async_commit();
+    // the first block of the prefix state, for the epilogue: it lands while
+    // the products run (rows past num_nodes and past the stack are skipped)
+    const int cb = tc_block_cols(d);
+    float* sPre = reinterpret_cast<float*>(sm + tc_prefetch_offset(V, d));  // [128][cb]
+    auto prefetch = [&](int b0) {
+        const int f4 = cb >> 2;
+        for (int e = tid; e < kTcRows * f4; e += kTcThreads) {
+            const int pl = e / f4, c4 = e - pl * f4, pm = m0 + pl;
+            const int ph = pm / V, pj = pm - ph * V;
+            if (pm < rows && pj < n) {
+                const size_t orow = ((size_t)r * V + pj) * J.H + (size_t)g * G + ph;
+                cp_async16(sPre + (size_t)pl * cb + 4 * c4, J.o_prefix + orow * d + b0 + 4 * c4);
+            }
+        }
+        cp_async_commit();
+    };
+    prefetch(0);
     for (int e0 = tid; e0 < Np * cpr; e0 += kTcThreads * (kTcBatch / 2)) {
-        uint4 kx[kTcBatch / 2], vx[kTcBatch / 2];
+        uint4 vx[kTcBatch / 2];
 #pragma unroll
         for (int u = 0; u < kTcBatch / 2; ++u) {
             const int e = e0 + u * kTcThreads, i = e / cpr, c = e - i * cpr;
-            kx[u] = zero;
             vx[u] = zero;
             if (e < Np * cpr && i < n) {
                 const size_t src = (((size_t)r * V + i) * J.Hkv + g) * d;
-                kx[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.k) + src) + c);
                 vx[u] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(J.v) + src) + c);
             }
         }
@@ -362,7 +390,6 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
         for (int u = 0; u < kTcBatch / 2; ++u) {
             const int e = e0 + u * kTcThreads, i = e / cpr, c = e - i * cpr;
             if (e >= Np * cpr) continue;
-            *reinterpret_cast<uint4*>(sK + kmajor_off(i, c * 8, d)) = kx[u];
             const uint32_t w[4] = {vx[u].x, vx[u].y, vx[u].z, vx[u].w};
 #pragma unroll
             for (int q = 0; q < 8; ++q)  // V^T: element (column t of V, node i)
@@ -383,6 +410,7 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
         }
         s_bad = bad;
     }
+    cp_async_wait<1>();   // Q and K have landed (the prefix block may still be in flight)
     fence_proxy_async();  // the staged operands, for the tensor cores
     tc_fence_before();
     __syncthreads();
@@ -495,11 +523,12 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
         s_c2[ml] = c2;
         s_row[ml] = live ? (long long)orow : (m < rows ? -2 - (long long)orow : -1);
     }
-    const int cb = d < 64 ? d : 64, ld = cb + 4;
+    const int ld = cb + 4;
     float* sO = reinterpret_cast<float*>(sm);  // [128][cb + 4]
     for (int b0 = 0; b0 < d; b0 += cb) {
         tc_fence_before();
         __syncthreads();  // the operands (first block) or the previous block are consumed
+        if (b0 > 0) prefetch(b0);  // its copies land while O leaves the tensor memory
         for (int c0 = 0; c0 < cb; c0 += 16) {
             float ov[16];
             tc_ld16(lane_addr + kTcColO + (uint32_t)(b0 + c0), ov);
@@ -509,6 +538,7 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
                 *reinterpret_cast<float4*>(sO + (size_t)ml * ld + c0 + 4 * q) =
                     make_float4(ov[4 * q] * c2, ov[4 * q + 1] * c2, ov[4 * q + 2] * c2, ov[4 * q + 3] * c2);
         }
+        cp_async_wait<0>();
         __syncthreads();
         const int f4 = cb >> 2;
         for (int e0 = tid; e0 < kTcRows * f4; e0 += kTcThreads * 4) {
@@ -518,7 +548,7 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
                 const int e = e0 + u * kTcThreads, row = e / f4, c4 = e - row * f4;
                 pv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (e < kTcRows * f4 && s_row[row] >= 0 && s_c1[row] != 0.0f)
-                    pv[u] = __ldg(reinterpret_cast<const float4*>(J.o_prefix + (size_t)s_row[row] * d + b0) + c4);
+                    pv[u] = *reinterpret_cast<const float4*>(sPre + (size_t)row * cb + 4 * c4);
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -576,7 +606,7 @@ extern "C" uno_status uno_tree_suffix_attention_merge(const void* q, const void*
     // alignment), so arrays that start off a 16-byte boundary go to the
     // CUDA-core kernel, which reads and writes single elements.
     const size_t tc_smem = tc_smem_bytes(V, d);
-    const bool tc = dt == UNO_BF16 && d % 16 == 0 && tc_smem <= 200 * 1024 && aligned(q, 16) && aligned(k, 16) &&
+    const bool tc = dt == UNO_BF16 && d % 16 == 0 && tc_smem <= 220 * 1024 && aligned(q, 16) && aligned(k, 16) &&
                     aligned(v, 16) && aligned(o_prefix, 16) && aligned(out_o, 16);
     const size_t smem = ((size_t)2 * V * (d + 1) + (size_t)kWarps * d) * 4 + (size_t)V * kMaskWords * 4;
     if (!tc && smem > 227 * 1024) return UNO_ERR_UNSUPPORTED;
