@@ -54,6 +54,37 @@ __device__ __forceinline__ float load_elem(const void* base, int32_t bf16, size_
     return static_cast<const float*>(base)[idx];
 }
 
+// Ancestor masks of the first n nodes of one request: node j's mask holds j
+// and its ancestors, found by walking up the parent links from j.  A link
+// must point to an earlier node, and node 0's parent is -1; a node whose link
+// breaks that rule keeps itself alone (the walk from any node below it stops
+// there) and sets *s_bad.  Each thread walks its own nodes; s_par (n entries)
+// is shared scratch.  Every thread of the block calls it; the caller
+// synchronises the block before reading anc or *s_bad.
+__device__ void build_ancestor_masks(const int32_t* parent, int n, uint32_t* anc, int32_t* s_par, int* s_bad,
+                                     int tid, int nthreads) {
+    for (int j = tid; j < n; j += nthreads) s_par[j] = parent[j];
+    if (tid == 0) *s_bad = 0;
+    __syncthreads();
+    for (int j = tid; j < n; j += nthreads) {
+        uint32_t mk[kMaskWords];
+#pragma unroll
+        for (int w = 0; w < kMaskWords; ++w) mk[w] = (j >> 5) == w ? 1u << (j & 31) : 0u;
+        int cur = j;
+        for (int step = 0; step < n; ++step) {  // links only go down, so at most j steps
+            const int p = s_par[cur];
+            const bool ok = cur == 0 ? p == -1 : (p >= 0 && p < cur);
+            if (!ok && cur == j) *s_bad = 1;
+            if (!ok || cur == 0) break;
+#pragma unroll
+            for (int w = 0; w < kMaskWords; ++w) mk[w] |= (p >> 5) == w ? 1u << (p & 31) : 0u;
+            cur = p;
+        }
+#pragma unroll
+        for (int w = 0; w < kMaskWords; ++w) anc[j * kMaskWords + w] = mk[w];
+    }
+}
+
 __global__ void __launch_bounds__(32 * kWarps) suffix_attention_kernel(const __grid_constant__ Job J) {
     extern __shared__ float smem[];
     const int r = blockIdx.x, g = blockIdx.y;
@@ -63,6 +94,7 @@ __global__ void __launch_bounds__(32 * kWarps) suffix_attention_kernel(const __g
     float* sq = sv + (size_t)V * ld;                                     // [kWarps][d]
     uint32_t* anc = reinterpret_cast<uint32_t*>(sq + (size_t)kWarps * d);  // [V][kMaskWords]
     __shared__ int s_bad;
+    __shared__ int32_t s_par[UNO_MAX_TREE_NODES];
 
     int n = J.num_nodes[r];
     n = n < 1 ? 1 : (n > V ? V : n);
@@ -73,20 +105,7 @@ __global__ void __launch_bounds__(32 * kWarps) suffix_attention_kernel(const __g
         sk[i * ld + t] = load_elem(J.k, J.bf16, src);
         sv[i * ld + t] = load_elem(J.v, J.bf16, src);
     }
-    if (threadIdx.x == 0) {
-        // ancestors in node order: a parent precedes its child
-        const int32_t* par = J.parent + (size_t)r * V;
-        int bad = 0;
-        for (int j = 0; j < n; ++j) {
-            const int p = par[j];
-            const bool ok = j == 0 ? p == -1 : (p >= 0 && p < j);
-            uint32_t* a = anc + j * kMaskWords;
-            for (int w = 0; w < kMaskWords; ++w) a[w] = (ok && j > 0) ? anc[p * kMaskWords + w] : 0u;
-            a[j >> 5] |= 1u << (j & 31);
-            bad |= ok ? 0 : 1;
-        }
-        s_bad = bad;
-    }
+    build_ancestor_masks(J.parent + (size_t)r * V, n, anc, s_par, &s_bad, threadIdx.x, blockDim.x);
     __syncthreads();
     if (threadIdx.x == 0 && g == 0 && J.out_flags != nullptr) J.out_flags[r] = s_bad ? UNO_FLAG_BAD_TREE : 0u;
 
@@ -308,6 +327,7 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
     __shared__ uint64_t bar;
     __shared__ uint32_t tmem_base;
     __shared__ int s_bad;
+    __shared__ int32_t s_par[UNO_MAX_TREE_NODES];
     const int r = blockIdx.x, g = blockIdx.y, m0 = blockIdx.z * kTcRows;
     const int V = J.V, d = J.d, G = J.G, rows = G * V;
     const int Np = (V + 15) / 16 * 16;
@@ -397,19 +417,7 @@ __global__ void __launch_bounds__(kTcThreads) suffix_attention_tc_kernel(const _
                     (uint16_t)((q & 1) ? (w[q >> 1] >> 16) : (w[q >> 1] & 0xffffu));
         }
     }
-    if (tid == 0) {
-        const int32_t* par = J.parent + (size_t)r * V;
-        int bad = 0;
-        for (int j = 0; j < n; ++j) {
-            const int p = par[j];
-            const bool ok = j == 0 ? p == -1 : (p >= 0 && p < j);
-            uint32_t* a = anc + j * kMaskWords;
-            for (int w2 = 0; w2 < kMaskWords; ++w2) a[w2] = (ok && j > 0) ? anc[p * kMaskWords + w2] : 0u;
-            a[j >> 5] |= 1u << (j & 31);
-            bad |= ok ? 0 : 1;
-        }
-        s_bad = bad;
-    }
+    build_ancestor_masks(J.parent + (size_t)r * V, n, anc, s_par, &s_bad, tid, kTcThreads);
     cp_async_wait<1>();   // Q and K have landed (the prefix block may still be in flight)
     fence_proxy_async();  // the staged operands, for the tensor cores
     tc_fence_before();

@@ -92,8 +92,9 @@ def test_largest_tree_as_a_chain():
     _check(dev, host, scale)
 
 
-def test_bad_tree_is_flagged_and_confined_to_its_request():
-    dev, host, scale = _case(3, 8, 4, 2, 32, 9, 4, "f32")
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])  # the CUDA-core and the tensor-core kernel
+def test_bad_tree_is_flagged_and_confined_to_its_request(dtype):
+    dev, host, scale = _case(3, 8, 4, 2, 32, 9, 4, dtype)
     parent = dev["node_parent"].clone()
     parent[1, 3] = 6  # a parent after its child
     dev["node_parent"] = parent
