@@ -50,8 +50,8 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
 
 
 # (R, B, vocab, dtype, top_k): the batch shape of the linear 8/1/8 workload,
-# an fp32 vocabulary with a ragged tail, a few rows (split over many CTAs,
-# which uses the split-row tickets) and top_k above 64 (the general row kernel)
+# an fp32 vocabulary with a ragged tail, a few rows (fewer rows than SMs: one
+# CTA per row) and top_k above 64 (the general row kernel)
 CASES = [
     (64, 8, 151936, "bf16", 50),
     (64, 8, 5003, "f32", 50),
